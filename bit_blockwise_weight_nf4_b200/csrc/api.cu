@@ -1,0 +1,221 @@
+// api.cu -- the C ABI declared in include/bnb4.h: argument checks, buffer
+// size queries, the device error word, and the launches on the caller's
+// stream.  Nothing here allocates or synchronizes (bnb4_device_status aside).
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "bnb4.h"
+#include "kernels.h"
+
+namespace {
+
+// Set by kernels whose bounded waits expire; read by bnb4_device_status.
+__device__ int g_device_error = 0;
+
+constexpr int kMaxDevices = 64;
+
+bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+
+bool valid_blocksize(int32_t bs) {
+  return bs == 32 || bs == 64 || bs == 128 || bs == 256;
+}
+
+int64_t n_blocks(int64_t n, int64_t bs) { return (n + bs - 1) / bs; }
+
+int current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices)
+    return BNB4_ERR_CUDA;
+  return BNB4_OK;
+}
+
+int num_sms(int* out) {
+  static int cache[kMaxDevices];
+  int dev;
+  if (current_device(&dev) != BNB4_OK) return BNB4_ERR_CUDA;
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) !=
+            cudaSuccess || v <= 0)
+      return BNB4_ERR_CUDA;
+    cache[dev] = v;
+  }
+  *out = cache[dev];
+  return BNB4_OK;
+}
+
+int error_word(int** out) {
+  static int* cache[kMaxDevices];
+  int dev;
+  if (current_device(&dev) != BNB4_OK) return BNB4_ERR_CUDA;
+  if (cache[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess || !p)
+      return BNB4_ERR_CUDA;
+    cache[dev] = static_cast<int*>(p);
+  }
+  *out = cache[dev];
+  return BNB4_OK;
+}
+
+// Fields shared by every state check.
+int check_state_common(const bnb4_qstate* st) {
+  if (!st || !st->codes || st->n <= 0) return BNB4_ERR_INVALID_ARG;
+  if (st->qtype != BNB4_NF4 && st->qtype != BNB4_FP4)
+    return BNB4_ERR_INVALID_ARG;
+  if (st->double_quant != 0 && st->double_quant != 1)
+    return BNB4_ERR_INVALID_ARG;
+  if (st->reserved != 0) return BNB4_ERR_INVALID_ARG;
+  if (!valid_blocksize(st->blocksize)) return BNB4_ERR_UNSUPPORTED;
+  if (!aligned(st->codes, 16)) return BNB4_ERR_ALIGNMENT;
+  return BNB4_OK;
+}
+
+// A state a consumer reads: the scales it needs must be present.
+int check_state_read(const bnb4_qstate* st) {
+  int rc = check_state_common(st);
+  if (rc != BNB4_OK) return rc;
+  if (st->double_quant) {
+    if (!st->absmax_q || !st->scale2 || !st->offset) return BNB4_ERR_INVALID_ARG;
+    if (!aligned(st->scale2, 4) || !aligned(st->offset, 4))
+      return BNB4_ERR_ALIGNMENT;
+  } else {
+    if (!st->absmax) return BNB4_ERR_INVALID_ARG;
+    if (!aligned(st->absmax, 4)) return BNB4_ERR_ALIGNMENT;
+  }
+  return BNB4_OK;
+}
+
+int check_weight(const bnb4_qstate* W, int64_t N, int64_t K) {
+  int rc = check_state_read(W);
+  if (rc != BNB4_OK) return rc;
+  if (N <= 0 || K <= 0) return BNB4_ERR_SHAPE;
+  if (N > INT64_MAX / K || W->n != N * K) return BNB4_ERR_SHAPE;
+  if (K % 64 != 0 || K % W->blocksize != 0) return BNB4_ERR_SHAPE;
+  return BNB4_OK;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? BNB4_OK : BNB4_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int bnb4_abi_version(void) { return BNB4_ABI_VERSION; }
+
+const char* bnb4_strerror(int status) {
+  switch (status) {
+    case BNB4_OK: return "ok";
+    case BNB4_ERR_INVALID_ARG: return "invalid argument (null pointer, n <= 0 or bad enum)";
+    case BNB4_ERR_UNSUPPORTED: return "unsupported blocksize or dtype";
+    case BNB4_ERR_ALIGNMENT: return "pointer misaligned (16 bytes for vector data)";
+    case BNB4_ERR_SHAPE: return "shape constraint violated";
+    case BNB4_ERR_WORKSPACE: return "workspace missing or too small";
+    case BNB4_ERR_CUDA: return "CUDA runtime error";
+    case BNB4_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait expired";
+    default: return "unknown status";
+  }
+}
+
+int bnb4_query_sizes(int64_t n, int32_t blocksize, int32_t double_quant,
+                     bnb4_sizes* out) {
+  if (!out || n <= 0 || (double_quant != 0 && double_quant != 1))
+    return BNB4_ERR_INVALID_ARG;
+  if (!valid_blocksize(blocksize)) return BNB4_ERR_UNSUPPORTED;
+  const int64_t nb = n_blocks(n, blocksize);
+  const int64_t ng = n_blocks(nb, 256);
+  out->codes = static_cast<size_t>((n + 1) / 2);
+  out->absmax = static_cast<size_t>(4 * nb);
+  out->absmax_q = double_quant ? static_cast<size_t>(nb) : 0;
+  out->scale2 = double_quant ? static_cast<size_t>(4 * ng) : 0;
+  out->offset = double_quant ? 4 : 0;
+  out->workspace =
+      double_quant ? sizeof(double) * static_cast<size_t>(bnb4::kMaxPartials) : 0;
+  return BNB4_OK;
+}
+
+int bnb_quantize_4bit(const void* x, int32_t x_dtype, const bnb4_qstate* st,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+  if (!x) return BNB4_ERR_INVALID_ARG;
+  if (x_dtype != BNB4_F32 && x_dtype != BNB4_BF16) return BNB4_ERR_UNSUPPORTED;
+  int rc = check_state_common(st);
+  if (rc != BNB4_OK) return rc;
+  if (!st->absmax) return BNB4_ERR_INVALID_ARG;
+  if (!aligned(x, 16)) return BNB4_ERR_ALIGNMENT;
+  if (!aligned(st->absmax, 4)) return BNB4_ERR_ALIGNMENT;
+  if (st->double_quant) {
+    if (!st->absmax_q || !st->scale2 || !st->offset) return BNB4_ERR_INVALID_ARG;
+    if (!aligned(st->scale2, 4) || !aligned(st->offset, 4))
+      return BNB4_ERR_ALIGNMENT;
+    if (!workspace ||
+        workspace_bytes < sizeof(double) * static_cast<size_t>(bnb4::kMaxPartials))
+      return BNB4_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return BNB4_ERR_ALIGNMENT;
+  }
+  int sms;
+  if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
+  const int grid = bnb4::quant_grid(st->n, x_dtype, sms);
+  return from_cuda(bnb4::launch_quantize(x, x_dtype, *st,
+                                         static_cast<double*>(workspace), grid,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+int bnb_dequantize_4bit(const bnb4_qstate* st, void* out, int32_t out_dtype,
+                        void* stream) {
+  if (!out) return BNB4_ERR_INVALID_ARG;
+  if (out_dtype != BNB4_F32 && out_dtype != BNB4_BF16) return BNB4_ERR_UNSUPPORTED;
+  int rc = check_state_read(st);
+  if (rc != BNB4_OK) return rc;
+  if (!aligned(out, 16)) return BNB4_ERR_ALIGNMENT;
+  int sms;
+  if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
+  const int grid = bnb4::dequant_grid(st->n, out_dtype, sms);
+  return from_cuda(bnb4::launch_dequantize(*st, out, out_dtype, grid,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstate* W,
+                  int64_t N, void* y, void* stream) {
+  if (!x || !y) return BNB4_ERR_INVALID_ARG;
+  int rc = check_weight(W, N, K);
+  if (rc != BNB4_OK) return rc;
+  if (B < 1 || B > 8) return BNB4_ERR_SHAPE;
+  if (!aligned(x, 16) || !aligned(y, 2)) return BNB4_ERR_ALIGNMENT;
+  int sms;
+  if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
+  return from_cuda(bnb4::launch_gemv(x, B, K, *W, N, y, sms,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstate* W,
+                  int64_t N, void* Y, void* stream) {
+  if (!X || !Y) return BNB4_ERR_INVALID_ARG;
+  int rc = check_weight(W, N, K);
+  if (rc != BNB4_OK) return rc;
+  if (M < 1 || N % 8 != 0 || M > (int64_t(1) << 31) || N > (int64_t(1) << 31))
+    return BNB4_ERR_SHAPE;
+  if (!aligned(X, 16) || !aligned(Y, 16)) return BNB4_ERR_ALIGNMENT;
+  int sms;
+  if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
+  int* err;
+  if ((rc = error_word(&err)) != BNB4_OK) return rc;
+  return from_cuda(bnb4::launch_gemm(X, M, K, *W, N, Y, err, sms,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
+int bnb4_device_status(void* stream, int32_t clear) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return BNB4_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess)
+    return BNB4_ERR_CUDA;
+  if (clear && v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess)
+      return BNB4_ERR_CUDA;
+  }
+  return v ? BNB4_ERR_DEVICE_TIMEOUT : BNB4_OK;
+}
+
+}  // extern "C"

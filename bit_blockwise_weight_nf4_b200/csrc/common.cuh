@@ -1,0 +1,86 @@
+// common.cuh -- device-side constants and helpers shared by the kernels of the
+// 4-bit blockwise quantization library (sm_100a).
+//
+// The codebooks follow the CSDN article on bitsandbytes, section "数学原理对比"
+// (NF4: 16 normal-quantile values normalised to [-1, 1] with an exact 0) and
+// its closing remarks (FP4: an E2M1-like format; here E2M1 magnitudes / 6 with
+// a sign bit).  The NF4 values are the QLoRA quantile construction:
+// positives = inverse normal CDF at 8 evenly spaced probabilities in
+// (1/2, 1 - delta], negatives = the same at 7 points, mirrored, plus 0,
+// all divided by the largest; delta = (1/32 + 1/30) / 2.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "bnb4.h"
+
+namespace bnb4 {
+
+constexpr int kQtNF4 = BNB4_NF4;
+constexpr int kQtFP4 = BNB4_FP4;
+
+// NF4 codebook, ascending; index 7 is the exact zero.
+__device__ __forceinline__ float nf4_value(int i) {
+  constexpr float t[16] = {
+      -0x1p+0f,        -0x1.647362p-1f, -0x1.0cd65cp-1f, -0x1.94653cp-2f,
+      -0x1.234496p-2f, -0x1.7a6a7ap-3f, -0x1.74f0d2p-4f, 0x0p+0f,
+      0x1.45f602p-4f,  0x1.4995bep-3f,  0x1.f809b4p-3f,  0x1.5a066cp-2f,
+      0x1.c3496ap-2f,  0x1.200f52p-1f,  0x1.722760p-1f,  0x1p+0f};
+  return t[i];
+}
+
+// FP4 magnitudes: E2M1 values {0, .5, 1, 1.5, 2, 3, 4, 6} divided by 6.
+__device__ __forceinline__ float fp4_magnitude(int m) {
+  constexpr float t[8] = {0x0p+0f,        0x1.555556p-4f, 0x1.555556p-3f,
+                          0x1p-2f,        0x1.555556p-2f, 0x1p-1f,
+                          0x1.555556p-1f, 0x1p+0f};
+  return t[m];
+}
+
+// Dequantization value of 4-bit code c (FP4: bit 3 is the sign).
+__device__ __forceinline__ float code_value(int qtype, int c) {
+  if (qtype == kQtNF4) return nf4_value(c);
+  const float m = fp4_magnitude(c & 7);
+  return (c & 8) ? -m : m;
+}
+
+// Decoded absmax of block b: fma(u - 128, s, offset) rounded once with double
+// quantization, the exact absmax without.
+template <bool DQ>
+__device__ __forceinline__ float decoded_absmax(int64_t b, const float* absmax,
+                                                const uint8_t* absmax_q,
+                                                const float* scale2,
+                                                float offset) {
+  if constexpr (DQ) {
+    const int u = __ldg(absmax_q + b);
+    return __fmaf_rn(static_cast<float>(u - 128), __ldg(scale2 + (b >> 8)),
+                     offset);
+  } else {
+    return __ldg(absmax + b);
+  }
+}
+
+__device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) {
+  return __uint_as_float(w << 16);
+}
+__device__ __forceinline__ float bf16_hi(uint32_t w) {
+  return __uint_as_float(w & 0xffff0000u);
+}
+
+// Two fp32 -> packed bf16x2 (lo in bits 0..15), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+}  // namespace bnb4

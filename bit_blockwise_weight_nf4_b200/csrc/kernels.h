@@ -1,0 +1,32 @@
+// kernels.h -- internal launcher interface between the C ABI (api.cu) and the
+// kernel translation units.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "bnb4.h"
+
+namespace bnb4 {
+
+// Upper bound on the quantize grid; the double-quant workspace holds one fp64
+// partial sum per CTA.
+constexpr int kMaxPartials = 4096;
+
+int quant_grid(int64_t n, int x_dtype, int num_sms);
+cudaError_t launch_quantize(const void* x, int x_dtype, const bnb4_qstate& st,
+                            double* partials, int grid, cudaStream_t s);
+
+int dequant_grid(int64_t n, int out_dtype, int num_sms);
+cudaError_t launch_dequantize(const bnb4_qstate& st, void* out, int out_dtype,
+                              int grid, cudaStream_t s);
+
+cudaError_t launch_gemv(const void* x, int64_t B, int64_t K,
+                        const bnb4_qstate& W, int64_t N, void* y, int num_sms,
+                        cudaStream_t s);
+
+cudaError_t launch_gemm(const void* X, int64_t M, int64_t K,
+                        const bnb4_qstate& W, int64_t N, void* Y, int* err,
+                        int num_sms, cudaStream_t s);
+
+}  // namespace bnb4

@@ -1,0 +1,199 @@
+/*
+ * bnb4.h -- C ABI of the B200 (sm_100a) library for 4-bit blockwise weight
+ * quantization (NF4 / FP4), double quantization of the per-block absmax,
+ * dequantization, and the fused 4-bit-weight x bf16-activation GEMV (decode)
+ * and GEMM (prefill).
+ *
+ * Sources, by page title and section:
+ *  - CSDN article "bitsandbytes 是一个用于高效量化和加载大型语言模型（LLM）的开源库",
+ *    section "数学原理对比": the NF4 codebook of 16 normal-quantile values in
+ *    [-1, 1] with an exact 0, the per-block absmax scale, no zero-point; the
+ *    closing remarks: fp4 as an E2M1-like format; section "实际性能差异":
+ *    double quantization (weights to 4 bits, then the scales to 8 bits).
+ *  - ossradar repository page for bitsandbytes, release notes 0.50.0 (fused
+ *    4-bit dequantize + GEMM for inference; nested quantization fused in),
+ *    0.50.2 (absmax store of a partial last block is masked), 0.49.2
+ *    (blocksize 32 and 64 for 4-bit), and the gemv_4bit / quantize /
+ *    dequantize op names.
+ *
+ * Conventions for every entry point:
+ *  - All data pointers are DEVICE pointers owned and allocated by the caller.
+ *    The library never allocates, frees or synchronizes (except
+ *    bnb4_device_status, which synchronizes the stream it is given).
+ *  - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *    stream.  Work is enqueued asynchronously on it.
+ *  - Every call returns a status (BNB4_OK = 0, negative on error).  On an
+ *    argument error nothing is launched and no memory is touched.  No C++
+ *    exception crosses the ABI.
+ *  - Tensors are dense and row-major.  A weight W[N, K] (out features N, in
+ *    features K) is quantized as the flat array of N*K elements, so its
+ *    blocks run along K.
+ *  - Alignment: x / out / codes / X / Y pointers must be 16-byte aligned;
+ *    fp32 arrays 4-byte aligned.  Misalignment returns BNB4_ERR_ALIGNMENT.
+ *  - Results are deterministic for a given input and device: codes, absmax,
+ *    double-quant fields and dequantized values are bit-identical to the
+ *    reference definition below.  The GEMV / GEMM accumulate in fp32 and round
+ *    once to bf16 at the end.
+ */
+#ifndef BNB4_H_
+#define BNB4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BNB4_ABI_VERSION 1
+
+/* Every entry point is exported from the shared library (the library is
+ * built with hidden visibility by default). */
+#if defined(__GNUC__)
+#define BNB4_API __attribute__((visibility("default")))
+#else
+#define BNB4_API
+#endif
+
+/* ----------------------------------------------------------- status codes */
+#define BNB4_OK 0
+#define BNB4_ERR_INVALID_ARG (-1)    /* null pointer, n <= 0, bad enum value */
+#define BNB4_ERR_UNSUPPORTED (-2)    /* blocksize not 32/64/128/256, dtype */
+#define BNB4_ERR_ALIGNMENT (-3)      /* a pointer misses its alignment */
+#define BNB4_ERR_SHAPE (-4)          /* shape constraint (see each call) */
+#define BNB4_ERR_WORKSPACE (-5)      /* workspace missing or too small */
+#define BNB4_ERR_CUDA (-6)           /* a CUDA runtime call or launch failed */
+#define BNB4_ERR_DEVICE_TIMEOUT (-7) /* a kernel's bounded wait expired */
+
+/* -------------------------------------------------------------- enums */
+#define BNB4_NF4 0  /* normal-quantile codebook */
+#define BNB4_FP4 1  /* E2M1 magnitudes / 6, sign-magnitude codes */
+#define BNB4_F32 0  /* fp32 element type */
+#define BNB4_BF16 1 /* bf16 element type (raw 16-bit patterns) */
+
+/*
+ * Quantization state of n elements: the packed codes plus the block scales.
+ * nb = ceil(n / blocksize) blocks of `blocksize` consecutive elements (the
+ * last may be short); ng = ceil(nb / 256) double-quant groups.
+ *
+ *  codes     uint8[ceil(n/2)]: byte j = code[2j] << 4 | code[2j+1]; an odd n
+ *            leaves the low nibble of the last byte 0.  16-byte aligned.
+ *  absmax    float[nb]: exact per-block max |x|.  Written by quantize in both
+ *            modes; read by the consumers only when double_quant == 0.
+ *  absmax_q  uint8[nb]: u = q + 128, q = clamp(rint((absmax - offset) / s),
+ *            -127, 127) with s the scale of the block's group (double quant).
+ *  scale2    float[ng]: s = max |absmax - offset| over the group / 127.
+ *  offset    float[1]: mean of absmax (fp64 sum, rounded to fp32).
+ * The decoded scale of block b is fma(u_b - 128, scale2[b/256], offset) with
+ * double quant, absmax[b] without.
+ */
+typedef struct bnb4_qstate {
+  uint8_t* codes;
+  float* absmax;
+  uint8_t* absmax_q;
+  float* scale2;
+  float* offset;
+  int64_t n;
+  int32_t blocksize;
+  int32_t qtype;
+  int32_t double_quant;
+  int32_t reserved; /* must be 0 */
+} bnb4_qstate;
+
+/* Byte sizes of every buffer of a quantization state of n elements. */
+typedef struct bnb4_sizes {
+  size_t codes;     /* ceil(n/2) */
+  size_t absmax;    /* 4 * nb */
+  size_t absmax_q;  /* nb (0 without double quant) */
+  size_t scale2;    /* 4 * ng (0 without double quant) */
+  size_t offset;    /* 4 (0 without double quant) */
+  size_t workspace; /* scratch bnb_quantize_4bit needs (0 without dq) */
+} bnb4_sizes;
+
+/*
+ * Fills *out with the buffer sizes for n elements.  Pure host function.
+ * Errors: INVALID_ARG (n <= 0, out NULL), UNSUPPORTED (blocksize).
+ */
+BNB4_API int bnb4_query_sizes(int64_t n, int32_t blocksize, int32_t double_quant,
+                     bnb4_sizes* out);
+
+/*
+ * Blockwise 4-bit quantization (NF4 article, section "数学原理对比": absmax
+ * scale per block, nearest codebook entry, 16 codes packed two per byte;
+ * section "实际性能差异": double quantization of the scales to 8 bits).
+ *
+ *  x           device, st->n elements of x_dtype (BNB4_F32 or BNB4_BF16),
+ *              16-byte aligned.
+ *  st          state whose buffers receive the result: codes and absmax
+ *              always; absmax_q, scale2 and offset when st->double_quant.
+ *  workspace   device scratch of at least bnb4_query_sizes(...).workspace
+ *              bytes, 16-byte aligned (may be NULL when the size is 0).
+ *              Its contents on entry do not matter.
+ * Per block: a = max|x|; r = RN(1/a) (0 for a = 0); v = RN(x*r); code =
+ * number of fp32 codebook midpoints RN(RN(t[i]+t[i+1])*0.5) strictly below v
+ * (FP4: of magnitude midpoints below |v|, sign bit set for v < 0 with a
+ * non-zero magnitude).  Ties at a midpoint go to the lower index.
+ * Bit-exact: codes, absmax, absmax_q, scale2 and offset equal the reference
+ * definition for finite inputs; the offset equals it whenever the fp64 sum
+ * of absmax is exact in every order (true for absmax values within ~29 -
+ * log2(nb) binades of each other).
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, WORKSPACE, CUDA.
+ */
+BNB4_API int bnb_quantize_4bit(const void* x, int32_t x_dtype, const bnb4_qstate* st,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Dequantization (NF4 article, section "实际性能差异": the 4-bit codes times
+ * the decoded block scale).  w = RN(t[code] * a_hat) in fp32; with out_dtype
+ * BNB4_BF16 the output is round-to-nearest-even of w.  out: device, st->n
+ * elements, 16-byte aligned.  Bit-exact to the reference definition.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA.
+ */
+BNB4_API int bnb_dequantize_4bit(const bnb4_qstate* st, void* out, int32_t out_dtype,
+                        void* stream);
+
+/*
+ * Decode GEMV (release notes 0.50.0 / gemv_4bit):
+ *   y[b, n] = bf16( sum_k x[b, k] * What[n, k] ),  b < B, n < N,
+ * What[n, k] = bf16(RN(t[code] * a_hat)) the dequantized weight, products
+ * exact, fp32 accumulation (order unspecified), one final rounding to bf16.
+ *  x  device bf16 [B, K], 16-byte aligned;   y  device bf16 [B, N].
+ *  W  quantization state of the weight [N, K] (W->n == N*K).
+ * Constraints: 1 <= B <= 8; K % 64 == 0; K % W->blocksize == 0.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, SHAPE, CUDA.
+ */
+BNB4_API int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstate* W,
+                  int64_t N, void* y, void* stream);
+
+/*
+ * Prefill GEMM with the dequantization fused in (release notes 0.50.0):
+ *   Y[m, n] = bf16( sum_k X[m, k] * What[n, k] ),  fp32 accumulation in
+ * tensor memory (tcgen05 bf16 MMA), What as in bnb_gemv_4bit.
+ *  X  device bf16 [M, K], 16-byte aligned;   Y  device bf16 [M, N],
+ *     16-byte aligned.
+ *  W  quantization state of the weight [N, K] (W->n == N*K).
+ * Constraints: M >= 1; N % 8 == 0; K % 64 == 0; K % W->blocksize == 0.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, SHAPE, CUDA.
+ */
+BNB4_API int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstate* W,
+                  int64_t N, void* Y, void* stream);
+
+/*
+ * Synchronizes `stream`, then reads the library's device error word of the
+ * current device: BNB4_OK, or BNB4_ERR_DEVICE_TIMEOUT when a kernel gave up a
+ * bounded wait (its output is then incomplete).  clear != 0 resets the word.
+ * Errors: CUDA.
+ */
+BNB4_API int bnb4_device_status(void* stream, int32_t clear);
+
+/* Static description of a status code; never NULL. */
+BNB4_API const char* bnb4_strerror(int status);
+
+/* BNB4_ABI_VERSION of the built library. */
+BNB4_API int bnb4_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BNB4_H_ */

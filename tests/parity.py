@@ -1,0 +1,99 @@
+"""Helpers shared by the GPU parity tests: unpacking, guard (canary) buffers
+and the linear-layer tolerance of the method's brief (relative Frobenius
+error <= 2e-3, per-row max abs error <= 1e-2 * ||x_b||_2 * max|What|)."""
+import numpy as np
+import torch
+
+import bit_blockwise_weight_nf4_b200 as bnb4
+import oracle
+
+REL_FROB_TOL = 2e-3
+MAX_ABS_FACTOR = 1e-2
+CANARY = 0xA5
+GUARD = 64  # bytes of canary after every output buffer
+
+
+def bits_to_f64(bits):
+    return oracle.bf16_bits_to_f64(bits)
+
+
+def cpu_bits(t):
+    """uint16 bit patterns of a bf16 tensor (any device)."""
+    return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
+
+
+class GuardedState:
+    """A device quantization state whose buffers are followed by canary
+    bytes, to catch writes past the end."""
+
+    def __init__(self, n, blocksize, qtype, dq):
+        rc, sz = bnb4.bnb4_query_sizes(n, blocksize, dq)
+        assert rc == 0
+        self.n, self.blocksize, self.qtype, self.dq = n, blocksize, qtype, dq
+        self.sizes = {"codes": sz.codes, "absmax": sz.absmax,
+                      "absmax_q": sz.absmax_q, "scale2": sz.scale2,
+                      "offset": sz.offset}
+        self.buf = {k: torch.full((v + GUARD,), CANARY, dtype=torch.uint8,
+                                  device="cuda")
+                    for k, v in self.sizes.items() if v > 0}
+        self.workspace = torch.empty(sz.workspace, dtype=torch.uint8,
+                                     device="cuda") if sz.workspace else None
+
+    def cstruct(self):
+        p = lambda k: self.buf[k].data_ptr() if k in self.buf else None
+        return bnb4.QState(p("codes"), p("absmax"), p("absmax_q"), p("scale2"),
+                           p("offset"), self.n, self.blocksize, self.qtype,
+                           int(self.dq), 0)
+
+    def quantize(self, x, x_dtype):
+        rc = bnb4.bnb_quantize_4bit(
+            x.data_ptr(), x_dtype, self.cstruct(),
+            None if self.workspace is None else self.workspace.data_ptr(),
+            0 if self.workspace is None else self.workspace.numel(),
+            torch.cuda.current_stream().cuda_stream)
+        assert rc == 0, bnb4.bnb4_strerror(rc)
+        torch.cuda.synchronize()
+
+    def arrays(self):
+        host = {k: b.cpu().numpy() for k, b in self.buf.items()}
+        for k, b in host.items():
+            assert np.all(b[self.sizes[k]:] == CANARY), "write past the end of " + k
+        out = {"codes": host["codes"][:self.sizes["codes"]],
+               "absmax": host["absmax"][:self.sizes["absmax"]].view(np.float32)}
+        if self.dq:
+            out["absmax_q"] = host["absmax_q"][:self.sizes["absmax_q"]]
+            out["scale2"] = host["scale2"][:self.sizes["scale2"]].view(np.float32)
+            out["offset"] = host["offset"][:4].view(np.float32)
+        return out
+
+
+def assert_state_equal(gpu, orc, dq):
+    keys = ["codes", "absmax"] + (["absmax_q", "scale2", "offset"] if dq else [])
+    for k in keys:
+        a, b = gpu[k], orc[k]
+        assert a.shape == b.shape, k
+        if not np.array_equal(a.view(np.uint8), b.view(np.uint8)):
+            bad = np.nonzero(a.view(np.uint8) != b.view(np.uint8))[0]
+            raise AssertionError("%s differs at %d bytes, first %s" % (k, bad.size, bad[:8]))
+
+
+def check_linear(y_gpu_bits, y64, x_bits, What_bits, rows=None):
+    """Tolerance of the method's brief for y = x What^T (rows of x optionally
+    subsampled; y64 is the fp64 oracle for those rows)."""
+    y = bits_to_f64(y_gpu_bits).reshape(y64.shape)
+    err = y - y64
+    rel = np.linalg.norm(err) / max(np.linalg.norm(y64), 1e-300)
+    assert rel <= REL_FROB_TOL, "relative Frobenius error %.3g" % rel
+    x = bits_to_f64(x_bits)
+    if rows is not None:
+        x = x[rows]
+    wmax = np.abs(bits_to_f64(What_bits)).max()
+    bound = MAX_ABS_FACTOR * np.linalg.norm(x, axis=1) * wmax
+    assert np.all(np.abs(err).max(axis=1) <= bound + 1e-30), "max abs error"
+    # the rounding of the exact fp64 result to bf16 is the dominant error:
+    # almost every output must equal it (a wrong What would not)
+    ref16 = torch.from_numpy(y64).to(torch.bfloat16).view(torch.int16).numpy() \
+        .view(np.uint16).reshape(-1)
+    match = np.mean(ref16 == np.asarray(y_gpu_bits).reshape(-1))
+    assert match >= 0.98, "only %.4f of outputs equal bf16(fp64 reference)" % match
+    return rel, match

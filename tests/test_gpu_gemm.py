@@ -1,0 +1,61 @@
+"""GPU prefill GEMM (tcgen05, fused dequantization) against the fp64 oracle
+over the dequantized bf16 weight, with the tolerance of the method's brief.
+Full-size shapes are checked on a seeded sample of rows of X (all columns);
+small shapes, including ragged M, are checked in full."""
+import numpy as np
+import pytest
+import torch
+
+import bit_blockwise_weight_nf4_b200 as bnb4
+import oracle
+import synth
+from parity import check_linear, cpu_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def case(M, N, K, bs, qtype, dq, seed, n_rows=None):
+    W = synth.weight_bf16(N, K, seed=seed)
+    X = synth.activations_bf16(M, K, seed=seed + 1)
+    st = oracle.quantize(synth.bf16_bits(W.view(-1)), bs, qtype, dq)
+    What = oracle.dequantize(st, oracle.BF16).reshape(N, K)
+    Xb = synth.bf16_bits(X)
+    rows = None
+    if n_rows is not None and n_rows < M:
+        rng = np.random.default_rng(seed)
+        rows = np.unique(np.concatenate([[0, M - 1],
+                                         rng.choice(M, n_rows - 2, replace=False)]))
+    y64 = oracle.linear_ref(Xb, What, rows=rows)
+    g = bnb4.state_from_arrays(st)
+    Y = bnb4.gemm_4bit(X.cuda(), g, N)
+    torch.cuda.synchronize()
+    assert bnb4.bnb4_device_status(torch.cuda.current_stream().cuda_stream) == 0
+    Yb = cpu_bits(Y)
+    if rows is not None:
+        Yb = Yb[rows]
+    return check_linear(Yb, y64, Xb, What, rows=rows)
+
+
+@pytest.mark.parametrize("N,K", synth.GEMM_SHAPES)
+def test_prefill_shapes_nf4_bs64(N, K):
+    """X bf16 [2048, K] ~ N(0, 1); NF4 weight ~ N(0, 0.02^2), blocksize 64,
+    double quant."""
+    case(synth.GEMM_M, N, K, 64, bnb4.NF4, True, seed=N + 3 * K, n_rows=48)
+
+
+@pytest.mark.parametrize("qtype,bs", [(bnb4.NF4, 128), (bnb4.FP4, 64),
+                                      (bnb4.FP4, 128)])
+def test_prefill_variants(qtype, bs):
+    case(synth.GEMM_M, 4096, 4096, bs, qtype, True, seed=bs + qtype, n_rows=48)
+
+
+@pytest.mark.parametrize("qtype", [bnb4.NF4, bnb4.FP4])
+@pytest.mark.parametrize("bs", [32, 64, 128, 256])
+@pytest.mark.parametrize("dq", [True, False])
+@pytest.mark.parametrize("M,N,K", [(1, 8, 256), (100, 264, 512),
+                                   (300, 520, 192), (256, 256, 64),
+                                   (513, 16, 1024)])
+def test_small_ragged(qtype, bs, dq, M, N, K):
+    if K % bs:
+        pytest.skip("K must be a multiple of the blocksize")
+    case(M, N, K, bs, qtype, dq, seed=M + N + K)

@@ -1,0 +1,60 @@
+"""GPU GEMV (decode) against the fp64 oracle over the dequantized bf16
+weight: relative Frobenius error <= 2e-3, per-row max abs error <=
+1e-2 ||x_b|| max|What|, and nearly every output equal to the bf16 rounding of
+the exact result."""
+import numpy as np
+import pytest
+import torch
+
+import bit_blockwise_weight_nf4_b200 as bnb4
+import oracle
+import synth
+from parity import check_linear, cpu_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def case(N, K, B, bs, qtype, dq, seed):
+    W = synth.weight_bf16(N, K, seed=seed)
+    x = synth.activations_bf16(B, K, seed=seed + 1)
+    st = oracle.quantize(synth.bf16_bits(W.view(-1)), bs, qtype, dq)
+    What = oracle.dequantize(st, oracle.BF16).reshape(N, K)
+    xb = synth.bf16_bits(x)
+    y64 = oracle.linear_ref(xb, What)
+    g = bnb4.state_from_arrays(st)
+    y = bnb4.gemv_4bit(x.cuda(), g, N)
+    return check_linear(cpu_bits(y), y64, xb, What)
+
+
+@pytest.mark.parametrize("N,K", [(11008, 4096), (4096, 11008)])
+@pytest.mark.parametrize("B", [1, 8])
+def test_llama_mlp_shapes(N, K, B):
+    """Decode GEMV: x bf16 [B, K] ~ N(0, 1); NF4 weight ~ N(0, 0.02^2),
+    blocksize 64, double quant (Llama-7B MLP shapes)."""
+    case(N, K, B, 64, bnb4.NF4, True, seed=N + K)
+
+
+@pytest.mark.parametrize("qtype", [bnb4.NF4, bnb4.FP4])
+@pytest.mark.parametrize("bs", [32, 64, 128, 256])
+@pytest.mark.parametrize("dq", [True, False])
+@pytest.mark.parametrize("N,K,B", [(1, 256, 1), (13, 320, 3), (100, 576, 8),
+                                   (257, 1024, 5), (8, 64, 2)])
+def test_small_ragged(qtype, bs, dq, N, K, B):
+    if K % bs:
+        pytest.skip("K must be a multiple of the blocksize")
+    case(N, K, B, bs, qtype, dq, seed=N * 31 + K)
+
+
+def test_gpu_quantized_weight_end_to_end():
+    """GPU quantize then GEMV on the GPU state (the codes equal the oracle's,
+    so the same fp64 reference applies)."""
+    N, K = 4096, 4096
+    W = synth.weight_bf16(N, K, seed=5, outlier_frac=synth.OUTLIER_FRAC)
+    x = synth.activations_bf16(1, K, seed=6)
+    st = oracle.quantize(synth.bf16_bits(W.view(-1)), 64, bnb4.NF4, True)
+    What = oracle.dequantize(st, oracle.BF16).reshape(N, K)
+    xb = synth.bf16_bits(x)
+    y64 = oracle.linear_ref(xb, What)
+    g = bnb4.quantize_4bit(W.cuda().view(-1), 64, bnb4.NF4, True)
+    y = bnb4.gemv_4bit(x.cuda(), g, N)
+    check_linear(cpu_bits(y), y64, xb, What)

@@ -1,0 +1,104 @@
+"""GPU parity of bnb_quantize_4bit against the CPU oracle: codes, absmax,
+absmax_q, scale2 and offset must be bit-identical, and nothing may be written
+past any output buffer."""
+import numpy as np
+import pytest
+import torch
+
+import bit_blockwise_weight_nf4_b200 as bnb4
+import oracle
+import synth
+from parity import GuardedState, assert_state_equal
+
+pytestmark = pytest.mark.gpu
+
+
+def run_both(x_cpu, bs, qtype, dq):
+    """x_cpu: fp32 or bf16 CPU tensor. Returns (gpu arrays, oracle state)."""
+    if x_cpu.dtype == torch.float32:
+        host, dt = x_cpu.contiguous().view(-1).numpy(), bnb4.F32
+    else:
+        host, dt = synth.bf16_bits(x_cpu.view(-1)), bnb4.BF16
+    orc = oracle.quantize(host, bs, qtype, dq)
+    g = GuardedState(host.size, bs, qtype, dq)
+    g.quantize(x_cpu.cuda(), dt)
+    return g.arrays(), orc
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("qtype", [bnb4.NF4, bnb4.FP4])
+@pytest.mark.parametrize("bs", [32, 64, 128, 256])
+@pytest.mark.parametrize("dq", [True, False])
+@pytest.mark.parametrize("n", [1, 2, 63, 64, 65, 257, 4097, 100003])
+def test_quantize_small_ragged(dtype, qtype, bs, dq, n):
+    x = synth.normal_f32((n,), seed=n + bs, std=0.02)
+    if dtype == "bf16":
+        x = x.to(torch.bfloat16)
+    gpu, orc = run_both(x, bs, qtype, dq)
+    assert_state_equal(gpu, orc, dq)
+
+
+def test_roundtrip_vector_1m():
+    """fp32 vector of 2^20 ~ N(0, 0.02^2), seed 0, blocksize 64, double
+    quant (mean-subtracted absmax in groups of 256)."""
+    x = synth.normal_f32((synth.ROUNDTRIP_N,), seed=0, std=0.02)
+    gpu, orc = run_both(x, 64, bnb4.NF4, True)
+    assert orc["sum_exact"]
+    assert_state_equal(gpu, orc, True)
+
+
+@pytest.mark.parametrize("qtype", [bnb4.NF4, bnb4.FP4])
+def test_matrix_4096_with_outliers(qtype):
+    """bf16 4096 x 4096 ~ N(0, 0.02^2), 0.1% of positions x20, blocksize 64,
+    double quant."""
+    W = synth.weight_bf16(4096, 4096, seed=1000, outlier_frac=synth.OUTLIER_FRAC)
+    gpu, orc = run_both(W, 64, qtype, True)
+    assert orc["sum_exact"]
+    assert_state_equal(gpu, orc, True)
+
+
+@pytest.mark.parametrize("qtype", [bnb4.NF4, bnb4.FP4])
+@pytest.mark.parametrize("bs", [32, 64, 256])
+def test_exact_midpoint_ties(qtype, bs):
+    """Blocks with max 2^k and the other elements exactly on fp32 codebook
+    midpoints times 2^k: v lands on the midpoint, the lower code wins."""
+    t = oracle.codebook(qtype).astype(np.float32)
+    if qtype == bnb4.NF4:
+        mids = [(t[i] + t[i + 1]) * np.float32(0.5) for i in range(15)]
+    else:
+        mids = [(t[i] + t[i + 1]) * np.float32(0.5) for i in range(7)]
+        mids += [-m for m in mids]
+    mids = np.array(mids, np.float32)
+    rng = np.random.default_rng(bs)
+    blocks = []
+    for k in range(-20, 21, 5):
+        blk = rng.choice(mids, bs).astype(np.float32) * np.float32(2.0 ** k)
+        blk[rng.integers(bs)] = np.float32(2.0 ** k)
+        blocks.append(blk)
+    x = torch.from_numpy(np.concatenate(blocks))
+    gpu, orc = run_both(x, bs, qtype, True)
+    assert_state_equal(gpu, orc, True)
+
+
+@pytest.mark.parametrize("qtype", [bnb4.NF4, bnb4.FP4])
+def test_zero_tiny_and_signed_zero_blocks(qtype):
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal(64 * 12) * 0.02).astype(np.float32)
+    x[0:64] = 0.0                                   # all-zero block
+    x[64:128] = -0.0                                # all negative zero
+    x[128:192] = rng.standard_normal(64) * 1e-40    # subnormal block
+    x[192:256] = 0.0
+    x[200] = 3e-39                                  # single tiny value
+    x[256:320] = rng.standard_normal(64) * 1e30     # huge block
+    gpu, orc = run_both(torch.from_numpy(x), 64, qtype, False)
+    assert_state_equal(gpu, orc, False)
+
+
+def test_codes_are_deterministic_and_independent_of_dq():
+    x = synth.weight_bf16(512, 1024, seed=77).cuda().view(-1)
+    a = bnb4.quantize_4bit(x, 64, bnb4.NF4, True)
+    b = bnb4.quantize_4bit(x, 64, bnb4.NF4, False)
+    c = bnb4.quantize_4bit(x, 64, bnb4.NF4, True)
+    assert torch.equal(a.codes, b.codes) and torch.equal(a.absmax, b.absmax)
+    for k in ("codes", "absmax", "absmax_q", "scale2", "offset"):
+        assert torch.equal(getattr(a, k), getattr(c, k))
