@@ -1,6 +1,18 @@
 """Helpers shared by the GPU parity tests: unpacking, guard (canary) buffers
-and the linear-layer tolerance of the method's brief (relative Frobenius
-error <= 2e-3, per-row max abs error <= 1e-2 * ||x_b||_2 * max|What|)."""
+and the linear-layer tolerance.
+
+Tolerance for y = bf16(fp32 sum of x * What) against the fp64 oracle y64:
+  * relative Frobenius error <= 2e-3 and per-row max abs error <=
+    1e-2 * ||x_b||_2 * max|What| (the method's brief).  The Frobenius bound is
+    statistical -- rounding one value to bf16 alone can cost up to 2^-8
+    relative -- so it is applied to outputs of at least 1024 elements;
+  * for every output, the bound the arithmetic gives: the fp32 accumulation
+    of exact bf16 x bf16 products errs by at most gamma * S (S = sum |x w|,
+    gamma = K 2^-22, a loose bound for any summation order and for the
+    tensor cores' accumulation), and the final bf16 rounding by 2^-8 of the
+    value: |y - y64| <= 2^-8 (|y64| + gamma S) + gamma S;
+  * with at least 1024 outputs, 98% of them equal bf16(y64) exactly (a wrong
+    What, or unrounded weights, would not)."""
 import numpy as np
 import torch
 
@@ -77,23 +89,35 @@ def assert_state_equal(gpu, orc, dq):
             raise AssertionError("%s differs at %d bytes, first %s" % (k, bad.size, bad[:8]))
 
 
+FROB_MIN_ELEMENTS = 1024
+
+
 def check_linear(y_gpu_bits, y64, x_bits, What_bits, rows=None):
-    """Tolerance of the method's brief for y = x What^T (rows of x optionally
-    subsampled; y64 is the fp64 oracle for those rows)."""
+    """Tolerance for y = x What^T (rows of x optionally subsampled; y64 is
+    the fp64 oracle for those rows).  See the module docstring."""
     y = bits_to_f64(y_gpu_bits).reshape(y64.shape)
     err = y - y64
     rel = np.linalg.norm(err) / max(np.linalg.norm(y64), 1e-300)
-    assert rel <= REL_FROB_TOL, "relative Frobenius error %.3g" % rel
+    if y64.size >= FROB_MIN_ELEMENTS:
+        assert rel <= REL_FROB_TOL, "relative Frobenius error %.3g" % rel
     x = bits_to_f64(x_bits)
     if rows is not None:
         x = x[rows]
-    wmax = np.abs(bits_to_f64(What_bits)).max()
+    W = bits_to_f64(What_bits)
+    wmax = np.abs(W).max()
     bound = MAX_ABS_FACTOR * np.linalg.norm(x, axis=1) * wmax
     assert np.all(np.abs(err).max(axis=1) <= bound + 1e-30), "max abs error"
+    K = x.shape[1]
+    gamma = K * 2.0 ** -22
+    S = np.abs(x) @ np.abs(W).T
+    elem = 2.0 ** -8 * (np.abs(y64) + gamma * S) + gamma * S
+    bad = np.abs(err) > elem
+    assert not bad.any(), "elementwise bound violated at %d outputs" % bad.sum()
     # the rounding of the exact fp64 result to bf16 is the dominant error:
     # almost every output must equal it (a wrong What would not)
     ref16 = torch.from_numpy(y64).to(torch.bfloat16).view(torch.int16).numpy() \
         .view(np.uint16).reshape(-1)
     match = np.mean(ref16 == np.asarray(y_gpu_bits).reshape(-1))
-    assert match >= 0.98, "only %.4f of outputs equal bf16(fp64 reference)" % match
+    if y64.size >= FROB_MIN_ELEMENTS:
+        assert match >= 0.98, "only %.4f of outputs equal bf16(fp64 reference)" % match
     return rel, match
