@@ -4,7 +4,7 @@ Two layers, both argument marshalling only -- every step of the
 quantize / dequantize / GEMV / GEMM path runs in the CUDA library:
 
 * raw ctypes entry points with the C names (``bnb_quantize_4bit``,
-  ``bnb_dequantize_4bit``, ``bnb_gemv_4bit``, ``bnb_gemm_4bit``,
+  ``bnb_quantize_4bit_noalloc``, ``bnb_dequantize_4bit``, ``bnb_gemv_4bit``, ``bnb_gemm_4bit``,
   ``bnb4_query_sizes``, ``bnb4_device_status``, ``bnb4_strerror``,
   ``bnb4_abi_version``), returning the C status;
 * torch helpers (``QuantState``, ``quantize_4bit``, ``dequantize_4bit``,
@@ -29,6 +29,9 @@ ERR_SHAPE = -4
 ERR_WORKSPACE = -5
 ERR_CUDA = -6
 ERR_DEVICE_TIMEOUT = -7
+ERR_SCRATCH_LIMIT = -8
+
+NOALLOC_MAX_BLOCKS = 1 << 20
 
 NF4 = 0
 FP4 = 1
@@ -79,6 +82,7 @@ def load():
     sig = {
         "bnb4_query_sizes": ([i64, i32, i32, ctypes.POINTER(Sizes)], ctypes.c_int),
         "bnb_quantize_4bit": ([p, i32, QP, p, sz, p], ctypes.c_int),
+        "bnb_quantize_4bit_noalloc": ([p, i32, QP, p], ctypes.c_int),
         "bnb_dequantize_4bit": ([QP, p, i32, p], ctypes.c_int),
         "bnb_gemv_4bit": ([p, i64, i64, QP, i64, p, p], ctypes.c_int),
         "bnb_gemm_4bit": ([p, i64, i64, QP, i64, p, p], ctypes.c_int),
@@ -115,6 +119,13 @@ def bnb4_query_sizes(n, blocksize, double_quant):
 def bnb_quantize_4bit(x, x_dtype, st, workspace, workspace_bytes, stream):
     return load().bnb_quantize_4bit(x, x_dtype, ctypes.byref(st), workspace,
                                     workspace_bytes, stream)
+
+
+def bnb_quantize_4bit_noalloc(x, x_dtype, st, stream):
+    """Allocation-free double-quantized quantize (see include/bnb4.h): the
+    library keeps its scratch in its own fixed device array, so the caller
+    passes no workspace and st.absmax is ignored."""
+    return load().bnb_quantize_4bit_noalloc(x, x_dtype, ctypes.byref(st), stream)
 
 
 def bnb_dequantize_4bit(st, out, out_dtype, stream):

@@ -114,6 +114,8 @@ const char* bnb4_strerror(int status) {
     case BNB4_ERR_WORKSPACE: return "workspace missing or too small";
     case BNB4_ERR_CUDA: return "CUDA runtime error";
     case BNB4_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait expired";
+    case BNB4_ERR_SCRATCH_LIMIT:
+      return "input exceeds the fixed scratch of the allocation-free entry point";
     default: return "unknown status";
   }
 }

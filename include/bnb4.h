@@ -64,6 +64,8 @@ extern "C" {
 #define BNB4_ERR_WORKSPACE (-5)      /* workspace missing or too small */
 #define BNB4_ERR_CUDA (-6)           /* a CUDA runtime call or launch failed */
 #define BNB4_ERR_DEVICE_TIMEOUT (-7) /* a kernel's bounded wait expired */
+#define BNB4_ERR_SCRATCH_LIMIT (-8)  /* input larger than the fixed scratch of
+                                        bnb_quantize_4bit_noalloc */
 
 /* -------------------------------------------------------------- enums */
 #define BNB4_NF4 0  /* normal-quantile codebook */
@@ -141,6 +143,39 @@ BNB4_API int bnb4_query_sizes(int64_t n, int32_t blocksize, int32_t double_quant
  */
 BNB4_API int bnb_quantize_4bit(const void* x, int32_t x_dtype, const bnb4_qstate* st,
                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Allocation-free variant of bnb_quantize_4bit with double quantization.
+ * The pages describe no such call; it exists for callers that cannot
+ * allocate device memory or pass a workspace -- for example a plugin whose
+ * host framework owns every device allocation, or a latency-critical loader
+ * that must not call cudaMalloc (which can synchronize the device or fail
+ * under memory pressure).
+ *
+ * Same method and bit-identical results as bnb_quantize_4bit with
+ * st->double_quant = 1, except that the exact fp32 absmax is not returned:
+ * st->absmax is ignored (may be NULL) and the intermediate absmax and the
+ * per-CTA fp64 partial sums live in a fixed array in the library's own
+ * device memory (32 KiB + 4 MiB per GPU that loads the library, held until
+ * the process exits).  The caller passes x and the outputs codes, absmax_q,
+ * scale2 and offset, with the alignment rules of bnb_quantize_4bit.
+ *  - Limit: at most BNB4_NOALLOC_MAX_BLOCKS blocks (ceil(n / blocksize));
+ *    larger inputs return BNB4_ERR_SCRATCH_LIMIT and launch nothing.
+ *  - st->double_quant must be 1 (without double quantization
+ *    bnb_quantize_4bit needs no workspace anyway): else INVALID_ARG.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, once per device, with that device current); make
+ *    that first call before any stream capture on the device.
+ *  - Every call shares the one array, and a call overwrites all of the
+ *    scratch it reads, so nothing carries over from the previous call; calls
+ *    that overlap on the GPU (different streams, or devices sharing a
+ *    context) race on it and must be serialized by the caller.
+ * Allocates nothing and calls no allocating routine.
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, SCRATCH_LIMIT, CUDA.
+ */
+#define BNB4_NOALLOC_MAX_BLOCKS (1 << 20)
+BNB4_API int bnb_quantize_4bit_noalloc(const void* x, int32_t x_dtype,
+                                       const bnb4_qstate* st, void* stream);
 
 /*
  * Dequantization (NF4 article, section "实际性能差异": the 4-bit codes times
