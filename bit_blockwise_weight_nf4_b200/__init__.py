@@ -87,6 +87,7 @@ def load():
         "bnb_gemv_4bit": ([p, i64, i64, QP, i64, p, p], ctypes.c_int),
         "bnb_gemm_4bit": ([p, i64, i64, QP, i64, p, p], ctypes.c_int),
         "bnb4_device_status": ([p, i32], ctypes.c_int),
+        "bnb4_debug_gemm_withhold": ([p, i64, i64, QP, i64, p, i32, p], ctypes.c_int),
         "bnb4_strerror": ([ctypes.c_int], ctypes.c_char_p),
         "bnb4_abi_version": ([], ctypes.c_int),
     }
@@ -138,6 +139,12 @@ def bnb_gemv_4bit(x, B, K, W, N, y, stream):
 
 def bnb_gemm_4bit(X, M, K, W, N, Y, stream):
     return load().bnb_gemm_4bit(X, M, K, ctypes.byref(W), N, Y, stream)
+
+
+def bnb4_debug_gemm_withhold(X, M, K, W, N, Y, wait_limit_us, stream):
+    """Failure-detection diagnostic (see include/bnb4.h)."""
+    return load().bnb4_debug_gemm_withhold(X, M, K, ctypes.byref(W), N, Y,
+                                           wait_limit_us, stream)
 
 
 def bnb4_device_status(stream, clear=True):

@@ -206,6 +206,25 @@ int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstate* W,
                                      static_cast<cudaStream_t>(stream)));
 }
 
+int bnb4_debug_gemm_withhold(const void* X, int64_t M, int64_t K,
+                             const bnb4_qstate* W, int64_t N, void* Y,
+                             int32_t wait_limit_us, void* stream) {
+  if (!X || !Y) return BNB4_ERR_INVALID_ARG;
+  int rc = check_weight(W, N, K);
+  if (rc != BNB4_OK) return rc;
+  if (M < 1 || N % 8 != 0 || M > (int64_t(1) << 31) || N > (int64_t(1) << 31))
+    return BNB4_ERR_SHAPE;
+  if (wait_limit_us < 1 || wait_limit_us > 1000000) return BNB4_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(Y, 16)) return BNB4_ERR_ALIGNMENT;
+  int sms;
+  if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
+  int* err;
+  if ((rc = error_word(&err)) != BNB4_OK) return rc;
+  return from_cuda(bnb4::launch_gemm(X, M, K, *W, N, Y, err, sms,
+                                     static_cast<cudaStream_t>(stream),
+                                     static_cast<uint64_t>(wait_limit_us) * 1000u, 1));
+}
+
 int bnb4_device_status(void* stream, int32_t clear) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return BNB4_ERR_CUDA;

@@ -7,28 +7,33 @@
 // 0.50.0 (ossradar page), nested quantization decoded inside, over the NF4 /
 // FP4 blockwise format of the CSDN article (section "数学原理对比").
 //
-// Design (one CTA per 256 x 256 output tile, 10 warps, 3-stage pipeline):
-//  * warp 0: producer.  Lane 0 issues the TMA loads of a 64-wide K step --
-//    two 128 x 64 bf16 tiles of X (128-byte swizzle) and the 256 x 32-byte
-//    packed weight tile; meanwhile all 32 lanes decode the 256 block scales of
-//    the step (nested quantization) into shared memory, so the dequantizers
-//    never wait on a global load.  One mbarrier (32 arrivals + the TMA bytes)
-//    marks the stage full.
-//  * warps 2..9 (256 threads): dequantizers.  Thread r turns weight row r of
-//    the stage (64 codes) into 64 bf16 values through a per-block 16-entry
-//    table (byte-permute lookups, as in the GEMV) and stores them in the
-//    128-byte-swizzled K-major layout the MMA reads; then fence.proxy.async
-//    and an arrive on the stage's "weights ready" barrier.
-//  * warp 1 (one lane): allocates 512 TMEM columns (two 128 x 256 fp32
-//    accumulators), waits for both barriers of a stage, issues 2 x 4
-//    tcgen05.mma (M 128, N 256, K 16) -- the dequantized tile is used by both
-//    M halves, halving the dequantization work per flop -- and commits to the
-//    stage's "empty" barrier.
-//  * epilogue: the 8 dequant warps read the accumulators with tcgen05.ld
-//    (warp w owns TMEM lanes 32 (w % 4)..+31), round to bf16 and store.
+// Design: CTA pairs (clusters of 2) with tcgen05.mma.cta_group::2.  A pair
+// owns a 512 x 256 output tile: two M = 256 accumulators (each CTA holds 128
+// rows of each in its TMEM, 2 x 256 columns) and N = 256 weight rows split in
+// halves -- each CTA dequantizes only its 128 weight rows, so the
+// dequantization work per flop is a quarter of a one-CTA 128 x 256 MMA.
+// Per CTA, 19 warps and three smem rings:
+//  * ring A (3 stages): the CTA's two 128 x 64 bf16 tiles of X per 64-wide K
+//    step, TMA (128-byte swizzle) completing on the leader CTA's barrier;
+//    warp 0 produces it (the leader also arms the barrier with the bytes of
+//    both CTAs).
+//  * ring W (8 stages): the CTA's 128 x 32-byte packed weight tile (TMA) plus
+//    its 128 decoded block scales (nested quantization decoded by the 32
+//    lanes of warp 2, whose scale loads run two steps ahead).
+//  * ring B (4 stages): the CTA's dequantized 128 x 64 bf16 weight half,
+//    written by warps 3..18 in four groups of 4 warps (group g takes the K
+//    steps kt = g mod 4 and owns B slot g; thread r of a group owns weight
+//    row r) in the 128-byte-swizzled K-major layout, then fence.proxy.async
+//    and one cluster-scope arrive per warp on the leader's barrier.
+//  * warp 1: allocates 512 TMEM columns in both CTAs; in the leader one lane
+//    waits for the A and B stages of both CTAs and issues 2 x 4
+//    tcgen05.mma.cta_group::2 (M 256, N 256, K 16), then commits to the
+//    "empty" barriers of both CTAs (multicast commit).
+//  * epilogue: warps 3..18 of each CTA read its accumulator rows with
+//    tcgen05.ld, round to bf16 and store.
 //  * Every mbarrier wait is bounded in time; on expiry the CTA sets the
 //    library's device error word, drains what it started and exits.
-//  No TMA multicast is used.
+//  No TMA load uses cluster multicast.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -38,30 +43,44 @@
 namespace bnb4 {
 namespace {
 
-constexpr int BM = 128;     // rows of one accumulator (M of one MMA)
-constexpr int MSUB = 2;     // accumulators per CTA (M tile 256)
-constexpr int BN = 256;     // weight rows per CTA (N of one MMA)
-constexpr int BK = 64;      // K per stage (one 128-byte swizzle row of bf16)
-constexpr int STAGES = 3;
-constexpr int A_BYTES = BM * BK * 2;    // 16 KB
-constexpr int B_BYTES = BN * BK * 2;    // 32 KB
-constexpr int WP_BYTES = BN * BK / 2;   // 8 KB packed codes
-constexpr int STAGE_BYTES = MSUB * A_BYTES + B_BYTES + WP_BYTES;
-constexpr int SCALE_FLOATS = 2 * BN;  // decoded scales of a stage (2 per row
-                                      // for blocksize 32)
-constexpr int kDeqWarps = 8;
-constexpr int kThreads = 64 + kDeqWarps * 32;
+constexpr int BM = 128;      // rows of one accumulator per CTA
+constexpr int MSUB = 2;      // accumulators (M = 256 each across the pair)
+constexpr int BNP = 256;     // weight rows per pair (N of one MMA)
+constexpr int BNC = 128;     // weight rows per CTA
+constexpr int BK = 64;       // K per stage (one 128-byte swizzle row of bf16)
+constexpr int SA = 3;        // X stages
+constexpr int SB = 4;        // dequantized weight stages (one per group)
+constexpr int SW = 8;        // packed weight + scale stages
+constexpr int NGROUPS = 4;   // dequant groups (one K step each in flight)
+constexpr int A_BYTES = BM * BK * 2;     // 16 KB
+constexpr int A_STAGE = MSUB * A_BYTES;  // 32 KB
+constexpr int B_BYTES = BNC * BK * 2;    // 16 KB
+constexpr int WP_BYTES = BNC * BK / 2;   // 4 KB packed codes
+constexpr int SCALE_FLOATS = 2 * BNC;    // 2 per row for blocksize 32
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + SA * A_STAGE;
+constexpr int OFF_W = OFF_B + SB * B_BYTES;
+constexpr int OFF_S = OFF_W + SW * WP_BYTES;
+constexpr int OFF_BARS = OFF_S + SW * SCALE_FLOATS * 4;
+constexpr int kDeqWarps = 16;
+constexpr int kGroupThreads = BNC;  // threads per group = weight rows of a CTA
+constexpr int kFirstDeqWarp = 3;
+constexpr int kThreads = (kFirstDeqWarp + kDeqWarps) * 32;
 constexpr int TMEM_COLS = 512;
-constexpr int SMEM_BYTES =
-    STAGES * STAGE_BYTES + STAGES * SCALE_FLOATS * 4 + 1024 /*align*/ + 256;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
-static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
+constexpr int SMEM_BYTES = OFF_BARS + 256 + 1024 /*align*/;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s (normal launches)
+constexpr uint32_t kSuspendHintNs = 1000000;       // 1 ms per try_wait
+static_assert(OFF_B % 1024 == 0 && OFF_W % 1024 == 0, "swizzled tiles need 1024-byte alignment");
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(kDeqWarps * 32 == NGROUPS * kGroupThreads, "groups");
+static_assert(SB == NGROUPS && SW % NGROUPS == 0, "group ownership of slots");
 
 struct Bars {
-  uint64_t full[STAGES];    // TMA bytes of the stage landed
-  uint64_t bready[STAGES];  // dequantized weights of the stage written
-  uint64_t empty[STAGES];   // MMAs reading the stage finished
-  uint64_t accum;           // all MMAs finished
+  uint64_t afull[SA], aempty[SA];  // X tiles of both CTAs landed (leader) / consumed
+  uint64_t wfull[SW], wempty[SW];  // codes + scales ready / read (local)
+  uint64_t bfull[SB], bempty[SB];  // dequantized halves written (leader) / consumed
+  uint64_t accum;                  // all MMAs finished
+  uint64_t wait_limit_ns;  // bound of every wait of this launch
   uint32_t tmem_base;
   int abort;
 };
@@ -69,9 +88,28 @@ struct Bars {
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
-
+__device__ __forceinline__ uint32_t cta_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same smem offset in CTA `rank` of the pair
+__device__ __forceinline__ uint32_t map_to(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+               "r"(bytes)
+               : "memory");
 }
 __device__ __forceinline__ void mbar_expect_tx_only(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes)
@@ -80,15 +118,37 @@ __device__ __forceinline__ void mbar_expect_tx_only(uint32_t bar, uint32_t bytes
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// arrive on a barrier of either CTA of the pair (cluster address), with
+// release at cluster scope
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cbar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cbar)
+               : "memory");
+}
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or the hint (ns) expires, instead of polling.  CTA-scope acquire
+// for barriers only this CTA (or the MMA commit) arrives on; cluster scope
+// only where the peer CTA arrives (the leader's A and B "full" barriers) --
+// a cluster-scope acquire also invalidates L1, which the producers' scale
+// loads rely on.
+template <bool kCluster>
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
+  if constexpr (kCluster)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
+        : "memory");
   return ok != 0;
 }
 __device__ __forceinline__ uint64_t global_ns() {
@@ -99,28 +159,51 @@ __device__ __forceinline__ uint64_t global_ns() {
 
 // Bounded wait for the phase of `parity`; false when the CTA is aborting or
 // the time limit expired (then the device error word is set).
+template <bool kCluster = false>
 __device__ bool wait_bounded(uint32_t bar, uint32_t parity, Bars* bars, int* err) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait<kCluster>(bar, parity)) return true;
   const uint64_t t0 = global_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
-      if (*reinterpret_cast<volatile int*>(&bars->abort)) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
-        atomicExch(err, 1);
-        *reinterpret_cast<volatile int*>(&bars->abort) = 1;
-        return false;
-      }
+  for (;;) {
+    if (mbar_try_wait<kCluster>(bar, parity)) return true;
+    if (*reinterpret_cast<volatile int*>(&bars->abort)) return false;
+    if (global_ns() - t0 > bars->wait_limit_ns) {
+      atomicExch(err, 1);
+      *reinterpret_cast<volatile int*>(&bars->abort) = 1;
+      return false;
     }
   }
 }
 
+// Wait for operations this CTA started (TMA loads, MMAs) to land before it
+// tears down: unlike wait_bounded it ignores the abort flag -- those
+// operations complete on their own within microseconds -- and gives up after
+// min(limit, 10 ms) when the phase cannot complete because an arrival is
+// missing on the abort path.
+template <bool kCluster = false>
+__device__ void wait_drain(uint32_t bar, uint32_t parity, Bars* bars) {
+  const uint64_t lim = bars->wait_limit_ns < 10000000ull ? bars->wait_limit_ns : 10000000ull;
+  const uint64_t t0 = global_ns();
+  while (!mbar_try_wait<kCluster>(bar, parity))
+    if (global_ns() - t0 > lim) return;
+}
+
+// TMA 2D load into this CTA's smem, completing on this CTA's barrier.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map,
                                             int x, int y, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+// TMA 2D load into this CTA's smem, completing on a barrier of either CTA of
+// the pair (`cbar` is a shared::cluster address; no multicast).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
+                                                 int x, int y, uint32_t cbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(cbar)
       : "memory");
 }
 
@@ -137,24 +220,28 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
 }
 
 // Instruction descriptor: kind::f16, D fp32, A and B bf16, both K-major,
-// N = 256, M = 128.
+// N = 256, M = 256 (two CTAs).
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
-                            (static_cast<uint32_t>(BN >> 3) << 17) |
-                            (static_cast<uint32_t>(BM >> 4) << 24);
+                            (static_cast<uint32_t>(BNP >> 3) << 17) |
+                            (static_cast<uint32_t>((2 * BM) >> 4) << 24);
 
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc,
-                                          uint64_t bdesc, uint32_t accumulate) {
+__device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc,
+                                               uint64_t bdesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
       "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate));
 }
 
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
+// Arrive on the barrier at `bar`'s offset in both CTAs of the pair once all
+// previously issued MMAs have completed.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
   asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          bar)
+      "{\n\t.reg .b16 m;\n\t"
+      "mov.b16 m, 3;\n\t"
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], m;\n\t}" ::"r"(bar)
       : "memory");
 }
 
@@ -190,16 +277,19 @@ __device__ __forceinline__ Lut make_lut(float ah) {
 }
 
 // 8 codes of one packed 32-bit word (natural order k0..k7) -> 8 bf16 in k
-// order as 4 words.
+// order as 4 words.  The low 3 bits of each code select from the two
+// 8-entry halves of the table, bit 3 picks the half; one mask / shift of the
+// whole word serves both 4-code halves (prmt reads the low 16 selector bits).
 __device__ __forceinline__ uint4 dq8(const Lut& l, uint32_t w) {
+  const uint32_t sel = w & 0x77777777u;
+  const uint32_t mix = ((w >> 1) & 0x44444444u) | 0x32103210u;
   uint4 o;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const uint32_t v = h ? (w >> 16) : w;
-    const uint32_t sel = v & 0x7777u;
-    const uint32_t mix = ((v >> 1) & 0x4444u) | 0x3210u;
-    const uint32_t lo = prmt(prmt(l.L[0], l.L[1], sel), prmt(l.L[2], l.L[3], sel), mix);
-    const uint32_t hi = prmt(prmt(l.H[0], l.H[1], sel), prmt(l.H[2], l.H[3], sel), mix);
+    const uint32_t s = h ? sel >> 16 : sel;
+    const uint32_t m = h ? mix >> 16 : mix;
+    const uint32_t lo = prmt(prmt(l.L[0], l.L[1], s), prmt(l.L[2], l.L[3], s), m);
+    const uint32_t hi = prmt(prmt(l.H[0], l.H[1], s), prmt(l.H[2], l.H[3], s), m);
     if (h == 0) {
       o.x = prmt(lo, hi, 0x4051);
       o.y = prmt(lo, hi, 0x6273);
@@ -215,170 +305,255 @@ template <int BS, int QT, bool DQ>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm4_kernel(const __grid_constant__ CUtensorMap map_x,
                  const __grid_constant__ CUtensorMap map_w, int M, int N, int K,
-                 const float* __restrict__ absmax,
+                 int n_pair_cols, const float* __restrict__ absmax,
                  const uint8_t* __restrict__ absmax_q,
                  const float* __restrict__ scale2,
                  const float* __restrict__ offset, uint16_t* __restrict__ Y,
-                 int* err) {
+                 int* err, uint64_t wait_limit_ns, int withhold_first_x) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* scales = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES);
-  Bars* bars = reinterpret_cast<Bars*>(smem + STAGES * STAGE_BYTES +
-                                       STAGES * SCALE_FLOATS * 4);
+  // 1024-byte aligned base, derived from the shared array by pointer
+  // arithmetic (not an integer cast) so every access stays a shared-memory
+  // access rather than a generic one
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+  Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BARS);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.y * (BM * MSUB);
-  const int n0 = blockIdx.x * BN;
+  const uint32_t rank = cta_rank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1;
+  const int m_pair = (pair / n_pair_cols) * (2 * MSUB * BM);
+  const int n_pair = (pair % n_pair_cols) * BNP;
+  const int n0 = n_pair + static_cast<int>(rank) * BNC;  // this CTA's weight rows
   const int k_tiles = K / BK;
 
-  auto stage_a = [&](int s, int j) { return smem + s * STAGE_BYTES + j * A_BYTES; };
-  auto stage_b = [&](int s) { return smem + s * STAGE_BYTES + MSUB * A_BYTES; };
-  auto stage_wp = [&](int s) {
-    return smem + s * STAGE_BYTES + MSUB * A_BYTES + B_BYTES;
+  auto a_tile = [&](int s, int j) { return smem + OFF_A + s * A_STAGE + j * A_BYTES; };
+  auto b_tile = [&](int s) { return smem + OFF_B + s * B_BYTES; };
+  auto w_tile = [&](int s) { return smem + OFF_W + s * WP_BYTES; };
+  auto scales = [&](int s) {
+    return reinterpret_cast<float*>(smem + OFF_S) + s * SCALE_FLOATS;
   };
+  auto bar = [&](uint64_t& b) { return smem_u32(&b); };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(smem_u32(&bars->full[s]), 32);
-      mbar_init(smem_u32(&bars->bready[s]), kDeqWarps * 32);
-      mbar_init(smem_u32(&bars->empty[s]), 1);
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(bar(bars->afull[s]), 1);
+      mbar_init(bar(bars->aempty[s]), 1);
     }
-    mbar_init(smem_u32(&bars->accum), 1);
+    for (int s = 0; s < SW; ++s) {
+      mbar_init(bar(bars->wfull[s]), 32);
+      mbar_init(bar(bars->wempty[s]), kGroupThreads / 32);
+    }
+    for (int s = 0; s < SB; ++s) {
+      mbar_init(bar(bars->bfull[s]), 2 * kGroupThreads / 32);
+      mbar_init(bar(bars->bempty[s]), 1);
+    }
+    mbar_init(bar(bars->accum), 1);
     bars->abort = 0;
+    bars->wait_limit_ns = wait_limit_ns;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&bars->tmem_base)),
                  "r"(TMEM_COLS));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
   }
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0) {
-    // ---------------------------------------------------------- producer
-    const float off = DQ ? __ldg(offset) : 0.0f;
-    int last_round[STAGES];
-    for (int s = 0; s < STAGES; ++s) last_round[s] = -1;
-    for (int kt = 0; kt < k_tiles; ++kt) {
-      const int s = kt % STAGES, round = kt / STAGES;
-      if (!wait_bounded(smem_u32(&bars->empty[s]), (round & 1) ^ 1, bars, err)) break;
-      const uint32_t fb = smem_u32(&bars->full[s]);
-      if (lane == 0) {
-        mbar_expect_tx_only(fb, MSUB * A_BYTES + WP_BYTES);
+    // ------------------------------------------------------ X producer
+    if (lane == 0) {
+      int last = -1;
+      for (int kt = 0; kt < k_tiles; ++kt) {
+        const int s = kt % SA, round = kt / SA;
+        if (!wait_bounded(bar(bars->aempty[s]), (round & 1) ^ 1, bars, err)) break;
+        // failure-detection diagnostic: the first X stage is never armed or
+        // loaded, so the MMA's wait for it runs out (nothing else changes)
+        if (withhold_first_x && kt == 0) continue;
+        const uint32_t fb = bar(bars->afull[s]);
+        if (leader) mbar_arrive_expect_tx(fb, 2 * A_STAGE);  // bytes of both CTAs
+        const uint32_t cfb = map_to(fb, 0);
         for (int j = 0; j < MSUB; ++j)
-          tma_load_2d(smem_u32(stage_a(s, j)), &map_x, kt * BK, m0 + j * BM, fb);
-        tma_load_2d(smem_u32(stage_wp(s)), &map_w, kt * (BK / 2), n0, fb);
+          tma_load_2d_pair(smem_u32(a_tile(s, j)), &map_x, kt * BK,
+                           m_pair + j * 2 * BM + static_cast<int>(rank) * BM, cfb);
+        last = kt;
       }
-      last_round[s] = round;
-      float* sc = scales + s * SCALE_FLOATS;
+      // drain: the loads this CTA issued have landed (the leader's barrier
+      // completes only when both CTAs' bytes arrived)
+      for (int kt = last - SA + 1 > 0 ? last - SA + 1 : 0; kt <= last; ++kt)
+        if (leader) wait_drain<true>(bar(bars->afull[kt % SA]), (kt / SA) & 1, bars);
+    }
+  } else if (warp == 2) {
+    // ------------------------------- packed weight + scale producer
+    // The raw scale inputs of a step are loaded two steps ahead into one of
+    // two register sets, so their latency overlaps the waits and the TMAs.
+    const float off = DQ ? __ldg(offset) : 0.0f;
+    constexpr int RPL = BNC / 32;  // rows per lane
+    constexpr int NBLK = BS == 32 ? 2 : 1;
+    auto fetch = [&](int kt, uint32_t (&u)[RPL][NBLK], float (&g)[RPL][NBLK]) {
 #pragma unroll
-      for (int i = 0; i < BN / 32; ++i) {
-        const int row = lane + 32 * i;
-        const int64_t n = static_cast<int64_t>(n0) + row;
-        float a0 = 0.0f, a1 = 0.0f;
-        if (n < N) {
-          const int64_t b = (n * K + static_cast<int64_t>(kt) * BK) / BS;
-          a0 = decoded_absmax<DQ>(b, absmax, absmax_q, scale2, off);
-          if constexpr (BS == 32) a1 = decoded_absmax<DQ>(b + 1, absmax, absmax_q, scale2, off);
+      for (int i = 0; i < RPL; ++i) {
+        const int64_t n = static_cast<int64_t>(n0) + lane + 32 * i;
+#pragma unroll
+        for (int j = 0; j < NBLK; ++j) {
+          u[i][j] = 0u;
+          g[i][j] = 0.0f;
+          if (n < N && kt < k_tiles) {
+            const int64_t b = (n * K + static_cast<int64_t>(kt) * BK) / BS + j;
+            if constexpr (DQ) {
+              u[i][j] = __ldg(absmax_q + b);
+              g[i][j] = __ldg(scale2 + (b >> 8));
+            } else {
+              u[i][j] = __float_as_uint(__ldg(absmax + b));
+            }
+          }
         }
-        sc[row] = a0;
-        if constexpr (BS == 32) sc[BN + row] = a1;
+      }
+    };
+    // two register sets, each refilled two steps ahead of its use
+    uint32_t ua[RPL][NBLK], ub[RPL][NBLK];
+    float ga[RPL][NBLK], gb[RPL][NBLK];
+    fetch(0, ua, ga);
+    fetch(1, ub, gb);
+    int last = -1;
+    bool ok = true;
+    auto step = [&](int kt, const uint32_t (&u)[RPL][NBLK], const float (&g)[RPL][NBLK]) {
+      const int s = kt % SW, round = kt / SW;
+      if (!wait_bounded(bar(bars->wempty[s]), (round & 1) ^ 1, bars, err)) {
+        ok = false;
+        return;
+      }
+      const uint32_t fb = bar(bars->wfull[s]);
+      if (lane == 0) {
+        mbar_expect_tx_only(fb, WP_BYTES);
+        tma_load_2d(smem_u32(w_tile(s)), &map_w, kt * (BK / 2), n0, fb);
+      }
+      last = kt;
+      float* sc = scales(s);
+#pragma unroll
+      for (int i = 0; i < RPL; ++i) {
+        const int row = lane + 32 * i;
+#pragma unroll
+        for (int j = 0; j < NBLK; ++j) {
+          float a;
+          if constexpr (DQ)
+            a = __fmaf_rn(static_cast<float>(static_cast<int>(u[i][j]) - 128), g[i][j], off);
+          else
+            a = __uint_as_float(u[i][j]);
+          sc[j * BNC + row] = a;
+        }
       }
       mbar_arrive(fb);
+    };
+    for (int kt = 0; kt < k_tiles && ok; kt += 2) {
+      step(kt, ua, ga);
+      fetch(kt + 2, ua, ga);
+      if (kt + 1 < k_tiles && ok) {
+        step(kt + 1, ub, gb);
+        fetch(kt + 3, ub, gb);
+      }
     }
-    // drain: every load issued has landed before the CTA may exit
     if (lane == 0)
-      for (int s = 0; s < STAGES; ++s)
-        if (last_round[s] >= 0)
-          wait_bounded(smem_u32(&bars->full[s]), last_round[s] & 1, bars, err);
+      for (int kt = last - SW + 1 > 0 ? last - SW + 1 : 0; kt <= last; ++kt)
+        wait_drain(bar(bars->wfull[kt % SW]), (kt / SW) & 1, bars);
   } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      bool ok = true;
-      for (int kt = 0; kt < k_tiles && ok; ++kt) {
-        const int s = kt % STAGES, round = kt / STAGES;
-        ok = wait_bounded(smem_u32(&bars->full[s]), round & 1, bars, err) &&
-             wait_bounded(smem_u32(&bars->bready[s]), round & 1, bars, err);
-        if (!ok) break;
+    // ------------------------------------------- MMA issuer (leader CTA)
+    if (leader && lane == 0) {
+      for (int kt = 0; kt < k_tiles; ++kt) {
+        const int sa = kt % SA, sb = kt % SB;
+        if (!wait_bounded<true>(bar(bars->afull[sa]), (kt / SA) & 1, bars, err) ||
+            !wait_bounded<true>(bar(bars->bfull[sb]), (kt / SB) & 1, bars, err))
+          break;
         asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-        const uint32_t b_addr = smem_u32(stage_b(s));
+        const uint32_t b_addr = smem_u32(b_tile(sb));
 #pragma unroll
         for (int j = 0; j < MSUB; ++j) {
-          const uint32_t a_addr = smem_u32(stage_a(s, j));
+          const uint32_t a_addr = smem_u32(a_tile(sa, j));
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_bf16(tmem + j * BN, sw128_desc(a_addr + 32 * k),
-                      sw128_desc(b_addr + 32 * k), (kt > 0 || k > 0) ? 1u : 0u);
+            umma_bf16_pair(tmem + j * BNP, sw128_desc(a_addr + 32 * k),
+                           sw128_desc(b_addr + 32 * k), (kt > 0 || k > 0) ? 1u : 0u);
         }
-        umma_commit(smem_u32(&bars->empty[s]));
+        umma_commit_pair(bar(bars->aempty[sa]));
+        umma_commit_pair(bar(bars->bempty[sb]));
       }
-      // completion of every MMA issued (also on the abort path, before the
-      // TMEM is released)
-      umma_commit(smem_u32(&bars->accum));
-      wait_bounded(smem_u32(&bars->accum), 0, bars, err);
+      // completion of every MMA issued, signalled to both CTAs (also on the
+      // abort path, before the TMEM is released)
+      umma_commit_pair(bar(bars->accum));
     }
   } else {
     // ------------------------------------------------- dequant + epilogue
-    const int r = threadIdx.x - 64;  // weight row of the tile
-    const int64_t n = static_cast<int64_t>(n0) + r;
-    const bool row_ok = n < N;
+    const int dq = threadIdx.x - kFirstDeqWarp * 32;
+    const int grp = dq / kGroupThreads;   // takes K steps kt = grp (mod 4)
+    const int r = dq % kGroupThreads;     // weight row of this CTA's half
+    const bool row_ok = static_cast<int64_t>(n0) + r < N;
     bool ok = true;
-    for (int kt = 0; kt < k_tiles; ++kt) {
-      const int s = kt % STAGES, round = kt / STAGES;
-      if (!wait_bounded(smem_u32(&bars->full[s]), round & 1, bars, err)) {
+    for (int kt = grp; kt < k_tiles; kt += NGROUPS) {
+      const int sw = kt % SW, sb = kt % SB;
+      if (!wait_bounded(bar(bars->wfull[sw]), (kt / SW) & 1, bars, err)) {
         ok = false;
         break;
       }
-      uint8_t* brow = stage_b(s) + r * 128;
-      const int sw = r & 7;
+      const uint4* wp = reinterpret_cast<const uint4*>(w_tile(sw) + r * 32);
+      const uint4 c0 = wp[0], c1 = wp[1];
+      const float* sc = scales(sw);
+      const float s0 = sc[r];
+      const float s1 = BS == 32 ? sc[BNC + r] : s0;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(bars->wempty[sw]));
+      if (!wait_bounded(bar(bars->bempty[sb]), ((kt / SB) & 1) ^ 1, bars, err)) {
+        ok = false;
+        break;
+      }
+      uint8_t* brow = b_tile(sb) + r * 128;
+      const int swz = r & 7;
       if (row_ok) {
-        const uint4* wp = reinterpret_cast<const uint4*>(stage_wp(s) + r * 32);
-        const uint4 c0 = wp[0], c1 = wp[1];
-        const float* sc = scales + s * SCALE_FLOATS;
-        const Lut l0 = make_lut<QT>(sc[r]);
+        const Lut l0 = make_lut<QT>(s0);
         Lut l1 = l0;
-        if constexpr (BS == 32) l1 = make_lut<QT>(sc[BN + r]);
+        if constexpr (BS == 32) l1 = make_lut<QT>(s1);
         const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
           const uint4 v = dq8(p < 4 ? l0 : l1, cw[p]);
-          *reinterpret_cast<uint4*>(brow + ((p ^ sw) << 4)) = v;
+          *reinterpret_cast<uint4*>(brow + ((p ^ swz) << 4)) = v;
         }
       } else {
 #pragma unroll
         for (int p = 0; p < 8; ++p)
-          *reinterpret_cast<uint4*>(brow + ((p ^ sw) << 4)) = make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(brow + ((p ^ swz) << 4)) = make_uint4(0, 0, 0, 0);
       }
+      // every lane makes its stores visible to the tensor core (async proxy),
+      // then one cluster-scope release per warp signals the leader
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(smem_u32(&bars->bready[s]));
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to(bar(bars->bfull[sb]), 0));
     }
-    // epilogue: accumulator j, TMEM lanes 32 q .. 32 q + 31, columns of half h.
-    // tcgen05.ld is warp-collective, so the go / no-go decision is made
-    // uniform across the warp.
+    // epilogue: accumulator j, TMEM lanes 32 q .. 32 q + 31 (rows of this
+    // CTA), a 64-column quarter h.  tcgen05.ld is warp-collective, so the
+    // go / no-go decision is uniform across the warp.
     bool go = __all_sync(0xffffffffu, ok);
     if (go) {
       bool w = true;
-      if (lane == 0) w = wait_bounded(smem_u32(&bars->accum), 0, bars, err);
+      if (lane == 0) w = wait_bounded(bar(bars->accum), 0, bars, err);
       go = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
     }
     if (go) {
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-      const int q = warp & 3;
-      const int h = (warp - 2) >> 2;
+      const int q = warp & 3;                     // TMEM lane quarter
+      const int h = (warp - kFirstDeqWarp) >> 2;  // 64-column quarter
 #pragma unroll 1
       for (int j = 0; j < MSUB; ++j) {
-        const int row = m0 + j * BM + q * 32 + lane;
+        const int row = m_pair + j * 2 * BM + static_cast<int>(rank) * BM + q * 32 + lane;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          const int col = h * 128 + c * 32;
+        for (int c = 0; c < 2; ++c) {
+          const int col = h * 64 + c * 32;
           uint32_t v[32];
           const uint32_t taddr =
-              tmem + (static_cast<uint32_t>(q * 32) << 16) + j * BN + col;
+              tmem + (static_cast<uint32_t>(q * 32) << 16) + j * BNP + col;
           asm volatile(
               "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
               "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -392,11 +567,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 "=r"(v[30]), "=r"(v[31])
               : "r"(taddr));
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-          if (row < M && n0 + col < N) {
-            uint16_t* dst = Y + static_cast<int64_t>(row) * N + n0 + col;
+          if (row < M && n_pair + col < N) {
+            uint16_t* dst = Y + static_cast<int64_t>(row) * N + n_pair + col;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              if (n0 + col + 8 * i < N) {
+              if (n_pair + col + 8 * i < N) {
                 const uint4 o = make_uint4(
                     pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1])),
                     pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
@@ -411,12 +586,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  // Teardown: every MMA of the pair has completed (the accum barrier of this
+  // CTA) before either CTA releases TMEM or exits, and neither exits while
+  // the other may still arrive on its barriers.
+  if (warp == 1 && lane == 0) wait_drain(bar(bars->accum), 0, bars);
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
   __syncthreads();
+  cluster_sync();
   if (warp == 1) {
     __syncwarp();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(TMEM_COLS));
   }
 }
@@ -451,7 +631,8 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base,
 
 template <int BS, int QT, bool DQ>
 cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W,
-                     int64_t N, void* Y, int* err, cudaStream_t s) {
+                     int64_t N, void* Y, int* err, uint64_t wait_limit_ns, int withhold,
+                     cudaStream_t s) {
   static bool attr_set[64] = {};  // per device
   auto kern = gemm4_kernel<BS, QT, DQ>;
   int dev = 0;
@@ -468,24 +649,37 @@ cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (!make_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.codes, K / 2, N, K / 2,
-                   BK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE))
+                   BK / 2, BNC, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
-  const dim3 grid(static_cast<unsigned>((N + BN - 1) / BN),
-                  static_cast<unsigned>((M + BM * MSUB - 1) / (BM * MSUB)));
-  kern<<<grid, kThreads, SMEM_BYTES, s>>>(mx, mw, static_cast<int>(M), static_cast<int>(N),
-                                          static_cast<int>(K), W.absmax, W.absmax_q,
-                                          W.scale2, W.offset, static_cast<uint16_t*>(Y), err);
-  return cudaGetLastError();
+  const int n_pair_cols = static_cast<int>((N + BNP - 1) / BNP);
+  const int m_pairs = static_cast<int>((M + 2 * MSUB * BM - 1) / (2 * MSUB * BM));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * n_pair_cols * m_pairs));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, mx, mw, static_cast<int>(M), static_cast<int>(N),
+                            static_cast<int>(K), n_pair_cols, W.absmax, W.absmax_q,
+                            W.scale2, W.offset, static_cast<uint16_t*>(Y), err,
+                            wait_limit_ns, withhold);
 }
 
 template <int QT, bool DQ>
 cudaError_t launch_bs(const void* X, int64_t M, int64_t K, const bnb4_qstate& W,
-                      int64_t N, void* Y, int* err, cudaStream_t s) {
+                      int64_t N, void* Y, int* err, uint64_t lim, int withhold,
+                      cudaStream_t s) {
   switch (W.blocksize) {
-    case 32: return launch_t<32, QT, DQ>(X, M, K, W, N, Y, err, s);
-    case 64: return launch_t<64, QT, DQ>(X, M, K, W, N, Y, err, s);
-    case 128: return launch_t<128, QT, DQ>(X, M, K, W, N, Y, err, s);
-    default: return launch_t<256, QT, DQ>(X, M, K, W, N, Y, err, s);
+    case 32: return launch_t<32, QT, DQ>(X, M, K, W, N, Y, err, lim, withhold, s);
+    case 64: return launch_t<64, QT, DQ>(X, M, K, W, N, Y, err, lim, withhold, s);
+    case 128: return launch_t<128, QT, DQ>(X, M, K, W, N, Y, err, lim, withhold, s);
+    default: return launch_t<256, QT, DQ>(X, M, K, W, N, Y, err, lim, withhold, s);
   }
 }
 
@@ -493,13 +687,16 @@ cudaError_t launch_bs(const void* X, int64_t M, int64_t K, const bnb4_qstate& W,
 
 cudaError_t launch_gemm(const void* X, int64_t M, int64_t K,
                         const bnb4_qstate& W, int64_t N, void* Y, int* err,
-                        int num_sms, cudaStream_t s) {
+                        int num_sms, cudaStream_t s, uint64_t wait_limit_ns,
+                        int withhold_first_x) {
   (void)num_sms;
+  const uint64_t lim = wait_limit_ns ? wait_limit_ns : kWaitLimitNs;
+  const int wh = withhold_first_x;
   if (W.qtype == kQtNF4)
-    return W.double_quant ? launch_bs<kQtNF4, true>(X, M, K, W, N, Y, err, s)
-                          : launch_bs<kQtNF4, false>(X, M, K, W, N, Y, err, s);
-  return W.double_quant ? launch_bs<kQtFP4, true>(X, M, K, W, N, Y, err, s)
-                        : launch_bs<kQtFP4, false>(X, M, K, W, N, Y, err, s);
+    return W.double_quant ? launch_bs<kQtNF4, true>(X, M, K, W, N, Y, err, lim, wh, s)
+                          : launch_bs<kQtNF4, false>(X, M, K, W, N, Y, err, lim, wh, s);
+  return W.double_quant ? launch_bs<kQtFP4, true>(X, M, K, W, N, Y, err, lim, wh, s)
+                        : launch_bs<kQtFP4, false>(X, M, K, W, N, Y, err, lim, wh, s);
 }
 
 }  // namespace bnb4

@@ -7,30 +7,35 @@
 // "数学原理对比"), nested (double) quantization decoded in-kernel.
 //
 // Design (HBM-bound on the packed bytes; integer-ALU heavy):
-//  * A warp owns 8 weight rows and a share of K; its 4 lanes of one quad hold
-//    one row, each lane a contiguous 64-element (32-byte) segment per
-//    256-wide K step, loaded with two 128-bit loads.
-//  * Per (row, quant block) each lane builds a 16-entry bf16 table of
+//  * A CTA (8 warps) owns 16 weight rows; its warps split K in 256-wide
+//    steps.  The 4 lanes of a quad own two rows (g and g + 8) and a
+//    contiguous 64-element segment of each per step (2 x 2 128-bit loads);
+//    every lane keeps 2 steps of loads (codes and raw scales) in flight.
+//  * Per (row, quant block) a lane builds the 16-entry bf16 table of
 //    bf16(RN(t[i] * a_hat)) -- bit-identical to dequantizing every element --
 //    split into low-byte and high-byte tables held in 8 registers.
 //  * 8 packed codes become 4 bf16x2 words with byte permutes (prmt): the low
 //    3 bits of each code select from the two 8-entry halves, bit 3 picks the
 //    half, a last permute interleaves low/high bytes.
-//  * The products go through mma.sync m16n8k16 (bf16 -> fp32) with the weight
-//    as the B operand (8 rows) and x as the A operand (batch rows, zero
-//    padded).  K is permuted identically in both operands, which leaves the
-//    dot products unchanged.
-//  * The 8 warps of a CTA split K; partial sums are reduced in shared memory
-//    in a fixed order and rounded once to bf16.
+//  * The products run on mma.sync m16n8k16 (bf16 -> fp32) with the weight as
+//    the A operand (16 rows) and x as B (batch columns): one 128-bit load of
+//    x feeds two MMAs straight from its register pairs, and batch columns
+//    beyond B simply read a valid row whose outputs are discarded.  K is
+//    permuted identically in both operands, which leaves the dot products
+//    unchanged; two accumulator chains keep consecutive MMAs independent.
+//  * Partial sums of the 8 warps are reduced in shared memory in a fixed
+//    order and rounded once to bf16.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace bnb4 {
 namespace {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 8;       // warps per CTA; they split K of one 16-row group
 constexpr int kThreads = kWarps * 32;
+constexpr int kRowsPerCta = 16;
 constexpr int kKStep = 256;  // K covered by one warp step (4 lanes x 64)
+constexpr int kChains = 2;   // independent MMA accumulators per warp
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
   uint32_t d;
@@ -66,29 +71,78 @@ __device__ __forceinline__ Lut make_lut(float ah) {
   return l;
 }
 
-// Four codes in the low 16 bits of w (nibble order k1 k0 k3 k2) -> two bf16x2
-// words {k0, k1}, {k2, k3}.
-__device__ __forceinline__ void dq4(const Lut& l, uint32_t w, uint32_t& o01,
-                                    uint32_t& o23) {
-  const uint32_t sel = w & 0x7777u;
-  const uint32_t mix = ((w >> 1) & 0x4444u) | 0x3210u;
+// Four codes (nibble order k1 k0 k3 k2 in the low 16 bits of the word they
+// came from) -> two bf16x2 words {k0, k1}, {k2, k3}.  `sel` holds the codes'
+// low 3 bits (the index into an 8-entry half), `mix` picks, per byte, the
+// half given by bit 3: nibble p of mix = p + 4 * bit3(code p).
+__device__ __forceinline__ void dq4(const Lut& l, uint32_t sel, uint32_t mix,
+                                    uint32_t& o01, uint32_t& o23) {
   const uint32_t lo = prmt(prmt(l.L[0], l.L[1], sel), prmt(l.L[2], l.L[3], sel), mix);
   const uint32_t hi = prmt(prmt(l.H[0], l.H[1], sel), prmt(l.H[2], l.H[3], sel), mix);
   o01 = prmt(lo, hi, 0x4051);
   o23 = prmt(lo, hi, 0x6273);
 }
 
-__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a2,
-                                         uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+// 8 packed codes -> 4 bf16x2 words in k order.  The selectors of both halves
+// come from one mask / shift of the whole word (prmt reads only the low 16
+// bits of its selector).
+__device__ __forceinline__ void dq8(const Lut& l, uint32_t w, uint32_t (&o)[4]) {
+  const uint32_t sel = w & 0x77777777u;
+  const uint32_t mix = ((w >> 1) & 0x44444444u) | 0x32103210u;
+  dq4(l, sel, mix, o[0], o[1]);
+  dq4(l, sel >> 16, mix >> 16, o[2], o[3]);
 }
 
-template <int BS, int QT, bool DQ>
-__global__ void __launch_bounds__(kThreads)
+// D[16 x 8] += A[16 x 16] (weight rows) * B[16 x 8] (x columns), bf16 in,
+// fp32 accumulate.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1,
+                                         uint32_t a2, uint32_t a3, uint32_t b0,
+                                         uint32_t b1) {
+  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Raw scale inputs of one quant block, loaded ahead and decoded when used
+// (so the decode never waits on a load issued just before it).
+struct RawScale {
+  uint32_t u;  // absmax_q byte (double quant) or absmax bits
+  float s;     // scale2 of the block's group (double quant)
+};
+
+template <bool DQ>
+__device__ __forceinline__ RawScale load_scale(int64_t b, const float* absmax,
+                                               const uint8_t* absmax_q,
+                                               const float* scale2) {
+  RawScale r;
+  if constexpr (DQ) {
+    r.u = __ldg(absmax_q + b);
+    r.s = __ldg(scale2 + (b >> 8));
+  } else {
+    r.u = __float_as_uint(__ldg(absmax + b));
+    r.s = 0.0f;
+  }
+  return r;
+}
+
+template <bool DQ>
+__device__ __forceinline__ float decode(const RawScale& r, float off) {
+  if constexpr (DQ)
+    return __fmaf_rn(static_cast<float>(static_cast<int>(r.u) - 128), r.s, off);
+  else
+    return __uint_as_float(r.u);
+}
+
+// Loads of one K step of one lane: 64 codes of each of its two rows and the
+// scales of their blocks, issued kDepth steps ahead of their use.
+struct StepBuf {
+  uint4 c[2][2];       // [row g / g+8][16-byte half]
+  RawScale a[2][2];    // [row][block within the segment (blocksize 32)]
+};
+
+template <int BS, int QT, bool DQ, int kDepth>
+__global__ void __launch_bounds__(kThreads, 2)
     gemv4_kernel(const uint16_t* __restrict__ x, int B, int64_t K,
                  const uint8_t* __restrict__ codes,
                  const float* __restrict__ absmax,
@@ -96,90 +150,135 @@ __global__ void __launch_bounds__(kThreads)
                  const float* __restrict__ scale2,
                  const float* __restrict__ offset, int64_t N,
                  uint16_t* __restrict__ y) {
-  __shared__ float red[kWarps][32][2];
+  __shared__ float red[kWarps][32][4];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int g = lane >> 2;  // weight row within the group / batch row of x
+  const int g = lane >> 2;  // rows g and g + 8 of the group; batch column g of x
   const int t = lane & 3;   // K segment of the step
-  const int64_t n = static_cast<int64_t>(blockIdx.x) * 8 + g;
-  const bool row_ok = n < N;
-  const bool x_ok = g < B;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRowsPerCta;
+  const int64_t n[2] = {row0 + g, row0 + g + 8};
+  const bool ok[2] = {n[0] < N, n[1] < N};
   const float off = DQ ? __ldg(offset) : 0.0f;
   const int64_t steps = (K + kKStep - 1) / kKStep;
-  const uint8_t* wrow = codes + n * (K / 2);
-  const uint16_t* xrow = x + static_cast<int64_t>(g) * K;
+  const int my_steps =
+      warp < steps ? static_cast<int>((steps - warp + kWarps - 1) / kWarps) : 0;
+  // batch columns beyond B read row B-1 (valid memory); their outputs are
+  // never stored
+  const uint16_t* xrow = x + static_cast<int64_t>(g < B ? g : B - 1) * K;
 
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-
-  for (int64_t s = warp; s < steps; s += kWarps) {
-    // this lane's segment; past a ragged K edge (K % 256 != 0) the lane
-    // feeds zeros, since mma.sync needs every lane of the warp
-    const int64_t k0 = s * kKStep + 64 * t;
-    const bool seg_ok = k0 < K;
-    uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
-    Lut lut0, lut1;
-    if (row_ok && seg_ok) {
-      c0 = ldg_stream_v4(wrow + k0 / 2);
-      c1 = ldg_stream_v4(wrow + k0 / 2 + 16);
-      const int64_t b = (n * K + k0) / BS;
-      lut0 = make_lut<QT>(decoded_absmax<DQ>(b, absmax, absmax_q, scale2, off));
-      if constexpr (BS == 32)
-        lut1 = make_lut<QT>(decoded_absmax<DQ>(b + 1, absmax, absmax_q, scale2, off));
-      else
-        lut1 = lut0;
-    } else {
-      lut0 = make_lut<QT>(0.0f);
-      lut1 = lut0;
-    }
-    const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  auto issue = [&](int i, StepBuf& b) {
+    const int64_t k0 = (static_cast<int64_t>(i) * kWarps + warp) * kKStep + 64 * t;
 #pragma unroll
-    for (int p = 0; p < 8; ++p) {  // 8 codes = k0 + 8p .. +7: two MMAs
-      uint4 xa = make_uint4(0, 0, 0, 0);
-      if (x_ok && seg_ok)
-        xa = __ldg(reinterpret_cast<const uint4*>(xrow + k0 + 8 * p));
-      const Lut& l = (BS == 32 && p >= 4) ? lut1 : lut0;
-      uint32_t b0, b1, b2, b3;
-      dq4(l, cw[p], b0, b1);
-      dq4(l, cw[p] >> 16, b2, b3);
-      mma_bf16(acc, xa.x, xa.y, b0, b1);
-      mma_bf16(acc, xa.z, xa.w, b2, b3);
+    for (int r = 0; r < 2; ++r) {
+      if (ok[r] && k0 < K) {
+        const uint8_t* src = codes + n[r] * (K / 2) + k0 / 2;
+        b.c[r][0] = ldg_stream_v4(src);
+        b.c[r][1] = ldg_stream_v4(src + 16);
+        const int64_t blk = (n[r] * K + k0) / BS;
+        b.a[r][0] = load_scale<DQ>(blk, absmax, absmax_q, scale2);
+        if constexpr (BS == 32) b.a[r][1] = load_scale<DQ>(blk + 1, absmax, absmax_q, scale2);
+      } else {
+        b.c[r][0] = make_uint4(0, 0, 0, 0);
+        b.c[r][1] = b.c[r][0];
+        b.a[r][0] = RawScale{0u, 0.0f};
+        b.a[r][1] = b.a[r][0];
+      }
+    }
+  };
+
+  float acc[kChains][4] = {};
+  StepBuf buf[kDepth];
+#pragma unroll
+  for (int d = 0; d < kDepth; ++d)
+    if (d < my_steps) issue(d, buf[d]);
+
+  for (int base = 0; base < my_steps; base += kDepth) {
+#pragma unroll
+    for (int d = 0; d < kDepth; ++d) {
+      const int i = base + d;
+      if (i < my_steps) {  // warp-uniform
+        const int64_t k0 = (static_cast<int64_t>(i) * kWarps + warp) * kKStep + 64 * t;
+        const bool seg = k0 < K;
+        // past a ragged K edge or the N edge the lane's rows are zero codes
+        // with a zero scale: mma.sync needs every lane of the warp
+        Lut lut[2][2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          lut[r][0] = make_lut<QT>(ok[r] && seg ? decode<DQ>(buf[d].a[r][0], off) : 0.0f);
+          lut[r][1] = BS == 32
+                          ? make_lut<QT>(ok[r] && seg ? decode<DQ>(buf[d].a[r][1], off) : 0.0f)
+                          : lut[r][0];
+        }
+        const int64_t kx = seg ? k0 : 0;  // x stays in bounds on a ragged edge
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {  // codes k0 + 8p .. +7 of both rows: two MMAs
+          const uint4 xb = __ldg(reinterpret_cast<const uint4*>(xrow + kx + 8 * p));
+          const int h = p >> 2, wi = p & 3;
+          const uint32_t w0 = wi == 0 ? buf[d].c[0][h].x : wi == 1 ? buf[d].c[0][h].y
+                            : wi == 2 ? buf[d].c[0][h].z : buf[d].c[0][h].w;
+          const uint32_t w1 = wi == 0 ? buf[d].c[1][h].x : wi == 1 ? buf[d].c[1][h].y
+                            : wi == 2 ? buf[d].c[1][h].z : buf[d].c[1][h].w;
+          uint32_t o0[4], o1[4];
+          dq8(lut[0][BS == 32 ? h : 0], w0, o0);
+          dq8(lut[1][BS == 32 ? h : 0], w1, o1);
+          mma_bf16(acc[(2 * p) % kChains], o0[0], o1[0], o0[1], o1[1], xb.x, xb.y);
+          mma_bf16(acc[(2 * p + 1) % kChains], o0[2], o1[2], o0[3], o1[3], xb.z, xb.w);
+        }
+        if (i + kDepth < my_steps) issue(i + kDepth, buf[d]);
+      }
     }
   }
 
-  // acc[0], acc[1]: batch g, rows 2t, 2t+1 of the group (acc[2..3] padding)
-  red[warp][lane][0] = acc[0];
-  red[warp][lane][1] = acc[1];
+  // acc[.]: rows g (0, 1) and g + 8 (2, 3) of the group, batch columns 2t and
+  // 2t + 1
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    float sum = 0.f;
+#pragma unroll
+    for (int c = 0; c < kChains; ++c) sum += acc[c][v];
+    red[warp][lane][v] = sum;
+  }
   __syncthreads();
   if (warp == 0) {
-    float s0 = 0.f, s1 = 0.f;
+    float s[4];
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      s0 += red[w][lane][0];
-      s1 += red[w][lane][1];
+    for (int v = 0; v < 4; ++v) {
+      s[v] = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) s[v] += red[w][lane][v];
     }
-    if (g < B) {
-      const int64_t r0 = static_cast<int64_t>(blockIdx.x) * 8 + 2 * t;
-      const uint32_t o = pack_bf16x2(s0, s1);
-      if (r0 < N) y[static_cast<int64_t>(g) * N + r0] = static_cast<uint16_t>(o);
-      if (r0 + 1 < N)
-        y[static_cast<int64_t>(g) * N + r0 + 1] = static_cast<uint16_t>(o >> 16);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+#pragma unroll
+      for (int cb = 0; cb < 2; ++cb) {
+        const int bcol = 2 * t + cb;
+        if (ok[r] && bcol < B) {
+          const uint32_t o = pack_bf16x2(s[2 * r + cb], 0.0f);
+          y[static_cast<int64_t>(bcol) * N + n[r]] = static_cast<uint16_t>(o);
+        }
+      }
     }
   }
+}
+
+template <int BS, int QT, bool DQ, int kDepth>
+cudaError_t launch_t(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
+                     int64_t N, void* y, cudaStream_t s) {
+  const int64_t grid = (N + kRowsPerCta - 1) / kRowsPerCta;
+  return launch_kernel(gemv4_kernel<BS, QT, DQ, kDepth>, dim3(static_cast<unsigned>(grid)),
+             dim3(kThreads), 0, s, false, static_cast<const uint16_t*>(x), static_cast<int>(B), K,
+             static_cast<const uint8_t*>(W.codes), static_cast<const float*>(W.absmax),
+             static_cast<const uint8_t*>(W.absmax_q), static_cast<const float*>(W.scale2),
+             static_cast<const float*>(W.offset), N, static_cast<uint16_t*>(y));
 }
 
 template <int BS, int QT>
 cudaError_t launch_bs(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
                       int64_t N, void* y, cudaStream_t s) {
-  const int64_t grid = (N + 7) / 8;
-  if (W.double_quant)
-    gemv4_kernel<BS, QT, true><<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
-        static_cast<const uint16_t*>(x), static_cast<int>(B), K, W.codes,
-        W.absmax, W.absmax_q, W.scale2, W.offset, N, static_cast<uint16_t*>(y));
-  else
-    gemv4_kernel<BS, QT, false><<<static_cast<unsigned>(grid), kThreads, 0, s>>>(
-        static_cast<const uint16_t*>(x), static_cast<int>(B), K, W.codes,
-        W.absmax, W.absmax_q, W.scale2, W.offset, N, static_cast<uint16_t*>(y));
-  return cudaGetLastError();
+  // two K steps of loads in flight per lane (for K <= 4096 that is all of a
+  // warp's share), 2 CTAs of 8 warps resident per SM
+  if (W.double_quant) return launch_t<BS, QT, true, 2>(x, B, K, W, N, y, s);
+  return launch_t<BS, QT, false, 2>(x, B, K, W, N, y, s);
 }
 
 template <int QT>

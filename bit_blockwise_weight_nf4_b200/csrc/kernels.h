@@ -25,8 +25,12 @@ cudaError_t launch_gemv(const void* x, int64_t B, int64_t K,
                         const bnb4_qstate& W, int64_t N, void* y, int num_sms,
                         cudaStream_t s);
 
+// wait_limit_ns = 0 selects the normal bound of every mbarrier wait (2 s);
+// withhold_first_x != 0 is the failure-detection diagnostic (the first X
+// stage is never loaded, so the kernel's waits run out).
 cudaError_t launch_gemm(const void* X, int64_t M, int64_t K,
                         const bnb4_qstate& W, int64_t N, void* Y, int* err,
-                        int num_sms, cudaStream_t s);
+                        int num_sms, cudaStream_t s, uint64_t wait_limit_ns = 0,
+                        int withhold_first_x = 0);
 
 }  // namespace bnb4

@@ -221,6 +221,20 @@ BNB4_API int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstat
  */
 BNB4_API int bnb4_device_status(void* stream, int32_t clear);
 
+/*
+ * Failure-detection diagnostic (no counterpart on the pages).  Runs the
+ * kernel of bnb_gemm_4bit (same arguments and checks) with its first X tile
+ * never loaded and every mbarrier wait bounded by wait_limit_us (1 ..
+ * 1,000,000): the kernel's waits run out, it sets the device error word,
+ * drains what it started, releases its tensor memory and exits.  A following
+ * bnb4_device_status reports BNB4_ERR_DEVICE_TIMEOUT and the context stays
+ * usable.  Y receives no defined values.  Nothing traps or hangs.
+ * Errors: as bnb_gemm_4bit, INVALID_ARG for the limit.
+ */
+BNB4_API int bnb4_debug_gemm_withhold(const void* X, int64_t M, int64_t K,
+                                      const bnb4_qstate* W, int64_t N, void* Y,
+                                      int32_t wait_limit_us, void* stream);
+
 /* Static description of a status code; never NULL. */
 BNB4_API const char* bnb4_strerror(int status);
 
