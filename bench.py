@@ -41,6 +41,28 @@ WORKLOAD = ("llama7b-shaped stack, 32 layers x 7 linears (224): per linear "
 GEMM_M = 2048
 BS = 64
 
+# DRAM bytes (read + write) per GEMM launch, averaged over the seven GEMMs of
+# one layer, from one ncu capture (profiles/gemm4_dram_traffic_llama7b_layer.md).
+# Reported only while the GEMM kernel's sources are the ones captured.
+GEMM_TRAFFIC_BYTES = 36508050
+GEMM_TRAFFIC_SOURCES = ("bit_blockwise_weight_nf4_b200/csrc/gemm.cu",
+                        "bit_blockwise_weight_nf4_b200/csrc/common.cuh")
+GEMM_TRAFFIC_SHA256 = "0e7d60c90f099d82488609b0055cbdbef27b70c1834f0dff3f0eb61a98f6e6ed"
+
+
+def gemm_traffic():
+    """Measured DRAM bytes per GEMM launch, or None when the kernel sources
+    changed since the capture."""
+    import hashlib
+    h = hashlib.sha256()
+    try:
+        for p in GEMM_TRAFFIC_SOURCES:
+            with open(os.path.join(ROOT, p), "rb") as f:
+                h.update(f.read())
+    except OSError:
+        return None
+    return GEMM_TRAFFIC_BYTES if h.hexdigest() == GEMM_TRAFFIC_SHA256 else None
+
 
 def parse():
     ap = argparse.ArgumentParser()
@@ -423,7 +445,8 @@ def run_ours(args):
                    "parallelism": "replicas x%d" % world},
         "roofline": {"bound": "tensor", "kernel": "gemm4 (fused dequant + tcgen05)",
                      "achieved": gemm_tflops, "peak": tf_sus, "unit": "TFLOP/s",
-                     "frac": gemm_tflops / tf_sus, "traffic": None,
+                     "frac": gemm_tflops / tf_sus, "traffic": gemm_traffic(),
+                     "traffic_unit": "bytes per launch (dram read + write, ncu)",
                      "peak_source": "%s bf16 sustained (kernel inside a long step)"
                                     % peak_src,
                      "per_launch": "2*2048*N*K flops; %d launches per step" % n_gemm},

@@ -88,6 +88,7 @@ def load():
         "bnb_gemm_4bit": ([p, i64, i64, QP, i64, p, p], ctypes.c_int),
         "bnb4_device_status": ([p, i32], ctypes.c_int),
         "bnb4_debug_gemm_withhold": ([p, i64, i64, QP, i64, p, i32, p], ctypes.c_int),
+        "bnb4_debug_check_rcp": ([p, p], ctypes.c_int),
         "bnb4_strerror": ([ctypes.c_int], ctypes.c_char_p),
         "bnb4_abi_version": ([], ctypes.c_int),
     }
@@ -145,6 +146,12 @@ def bnb4_debug_gemm_withhold(X, M, K, W, N, Y, wait_limit_us, stream):
     """Failure-detection diagnostic (see include/bnb4.h)."""
     return load().bnb4_debug_gemm_withhold(X, M, K, ctypes.byref(W), N, Y,
                                            wait_limit_us, stream)
+
+
+def bnb4_debug_check_rcp(result, stream):
+    """Self-check of the quantize kernel's reciprocal over its whole input
+    range (see include/bnb4.h); result = 16-byte device buffer."""
+    return load().bnb4_debug_check_rcp(result, stream)
 
 
 def bnb4_device_status(stream, clear=True):

@@ -225,6 +225,12 @@ int bnb4_debug_gemm_withhold(const void* X, int64_t M, int64_t K,
                                      static_cast<uint64_t>(wait_limit_us) * 1000u, 1));
 }
 
+int bnb4_debug_check_rcp(void* result, void* stream) {
+  if (!result) return BNB4_ERR_INVALID_ARG;
+  if (!aligned(result, 8)) return BNB4_ERR_ALIGNMENT;
+  return from_cuda(bnb4::launch_check_rcp(result, static_cast<cudaStream_t>(stream)));
+}
+
 int bnb4_device_status(void* stream, int32_t clear) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return BNB4_ERR_CUDA;

@@ -21,6 +21,10 @@ int dequant_grid(int64_t n, int out_dtype, int num_sms);
 cudaError_t launch_dequantize(const bnb4_qstate& st, void* out, int out_dtype,
                               int grid, cudaStream_t s);
 
+// Compares the quantize kernel's reciprocal with the correctly rounded one
+// over its whole input range; result = {u64 mismatches, u32 first, u32 0}.
+cudaError_t launch_check_rcp(void* result, cudaStream_t s);
+
 cudaError_t launch_gemv(const void* x, int64_t B, int64_t K,
                         const bnb4_qstate& W, int64_t N, void* y, int num_sms,
                         cudaStream_t s);

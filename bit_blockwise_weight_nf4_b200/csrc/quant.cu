@@ -12,18 +12,29 @@
 //   absmax (fp64 sum), c = RN(a - offset), per group of 256: s = RN(max|c| /
 //   127), u = clamp(rint(RN(c / s)), -127, 127) + 128.
 //
-// Design (HBM-bound): a persistent grid of 256-thread CTAs, exactly the
-// resident ones (3 per SM); each warp streams tiles of 8 x 512 contiguous
-// bytes with 128-bit non-allocating loads, refilling each row's register slot
-// with the next tile's row as soon as it is consumed (8 loads in flight per
-// lane at all times), reduces each block's absmax with xor shuffles among the
-// lanes that hold it, and writes the packed codes with one coalesced
-// 16/32-bit store per lane and row.  The nearest-code search is one
-// fused multiply-add that buckets v into 1/32-wide intervals, one shared-
-// memory lookup of {candidate midpoint, codes below it} (lane-replicated, so
-// conflict free) and one compare.  The double quantization runs as a second,
-// tiny kernel that first reduces the per-CTA fp64 partial sums in a fixed
-// order.
+// Design (HBM-bound; the instruction budget per element decides how close to
+// the bound it runs): a persistent grid of 256-thread CTAs, exactly the
+// resident ones (3 per SM).  Each warp streams whole tiles of 8 rows x 512
+// contiguous bytes with 128-bit non-allocating loads, refilling each row's
+// register slot with the next tile's row as soon as it is consumed (8 loads
+// in flight per lane at all times).  Per row a lane holds one 16-byte chunk
+// of a block; the block absmax is an xor-shuffle reduction among the lanes
+// that hold it.  Addresses are lane pointers advanced once per tile, rows
+// are immediate offsets.  The common case -- an absmax in [2^-126, 2^126),
+// warp-uniformly -- takes a branch-free path:
+//   * 1/a from the approximate reciprocal refined to the correctly rounded
+//     value (Newton-Raphson step plus Markstein's final correction);
+//   * nearest code: one FMA buckets v into 1/32-wide intervals (the integer
+//     lands in the mantissa bits of 1.5 * 2^23 + v * 32), one lane-private
+//     shared-memory lookup of {candidate midpoint, midpoints below the
+//     bucket}, one compare;
+//   * the chunk's packed word is built by a Horner chain p = 16 p + code in
+//     the nibble order of the byte layout, so no shifts or ors are needed.
+// Any other row group (zero, subnormal or huge absmax, infinities) and the
+// one ragged tile at the end take an exact out-of-line path with the
+// correctly rounded reciprocal and a clamped lookup.  The double
+// quantization runs as a second, tiny kernel that first reduces the per-CTA
+// fp64 partial sums in a fixed order.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -33,40 +44,51 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kCtasPerSm = 3;       // resident CTAs per SM (register cap)
 constexpr int kRows = 8;            // 16-byte chunks per lane per tile
-constexpr int kLutBuckets = 65;     // buckets j = 0..64 reached by finite values
 constexpr int kLutEntries = 128;    // the fast path masks the bucket to 7 bits
 // v is bucketed as j = rint(32 v) + 32 (NF4) or rint(32 |v|) (FP4) with one
 // FMA against 1.5 * 2^23 (+32): the integer lands in the mantissa bits.
 constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr int kMagicBits = 0x4B400000;
+// FP4: the smallest magnitude midpoint, RN(RN(0 + 1/12) * 0.5).  A value
+// gets the sign bit exactly when v < -kFp4Mid0 (negative with a non-zero
+// magnitude index).
+constexpr float kFp4Mid0 = 0x1.555556p-5f;
+
+template <int QT>
+__host__ __device__ constexpr int lut_buckets() {  // buckets reached by |v| <= 1 (+ rounding)
+  return QT == kQtNF4 ? 65 : 33;
+}
 
 // Bucket table, replicated per lane: entry (j, lane) at lut[j * 32 + lane].
 // For every v whose bucket is j, code = base + (v > cand), where base counts
 // the midpoints below the bucket and cand is the only midpoint inside it (or
 // +inf).  Buckets are 1/32 wide; codebook midpoints are at least 0.08 apart, so
-// a bucket widened by 1e-3 on each side holds at most one.
+// a bucket widened by 1e-3 on each side holds at most one.  Entries past the
+// reachable buckets are {+inf, 0}: only a NaN lands there, and its code is
+// 0 (no midpoint is below NaN).
 template <int QT>
 __device__ void build_lut(uint2* lut) {
   constexpr int nm = QT == kQtNF4 ? 15 : 7;
-  // one thread per bucket computes its entry into lane slot 0 (entries past
-  // the last reachable bucket repeat it: only non-finite input lands there)
+  // one thread per entry computes it into lane slot 0 ...
   if (threadIdx.x < kLutEntries) {
-    const int j = threadIdx.x < kLutBuckets ? threadIdx.x : kLutBuckets - 1;
-    const float center = QT == kQtNF4 ? static_cast<float>(j - 32)
-                                      : static_cast<float>(j);
-    const float lo = (center - 0.5f) / 32.0f - 1e-3f;
-    const float hi = (center + 0.5f) / 32.0f + 1e-3f;
+    const int j = threadIdx.x;
     int base = 0;
     float cand = __int_as_float(0x7f800000);
+    if (j < lut_buckets<QT>()) {
+      const float center = QT == kQtNF4 ? static_cast<float>(j - 32)
+                                        : static_cast<float>(j);
+      const float lo = (center - 0.5f) / 32.0f - 1e-3f;
+      const float hi = (center + 0.5f) / 32.0f + 1e-3f;
 #pragma unroll
-    for (int i = 0; i < nm; ++i) {
-      const float a = QT == kQtNF4 ? nf4_value(i) : fp4_magnitude(i);
-      const float b = QT == kQtNF4 ? nf4_value(i + 1) : fp4_magnitude(i + 1);
-      const float mid = __fmul_rn(__fadd_rn(a, b), 0.5f);
-      if (mid < lo) ++base;
-      else if (mid <= hi) cand = mid;
+      for (int i = 0; i < nm; ++i) {
+        const float a = QT == kQtNF4 ? nf4_value(i) : fp4_magnitude(i);
+        const float b = QT == kQtNF4 ? nf4_value(i + 1) : fp4_magnitude(i + 1);
+        const float mid = __fmul_rn(__fadd_rn(a, b), 0.5f);
+        if (mid < lo) ++base;
+        else if (mid <= hi) cand = mid;
+      }
     }
-    lut[threadIdx.x * 32] = make_uint2(__float_as_uint(cand), static_cast<uint32_t>(base));
+    lut[j * 32] = make_uint2(__float_as_uint(cand), static_cast<uint32_t>(base));
   }
   __syncthreads();
   // ... and every thread replicates entries to the other lane slots
@@ -74,11 +96,12 @@ __device__ void build_lut(uint2* lut) {
     if (idx & 31) lut[idx] = lut[idx & ~31];
 }
 
+// Exact nearest code for any v (infinite and NaN included): the bucket is
+// clamped in the float domain (maxNum drops a NaN), which reproduces the
+// midpoint count.
 template <int QT>
 __device__ __forceinline__ uint32_t code_of(float v, const uint2* lut_lane) {
   if constexpr (QT == kQtNF4) {
-    // clamp in the float domain: keeps NaN (maxNum drops it) and out-of-range
-    // values inside the table, with the same result as counting midpoints.
     const float f = fminf(fmaxf(__fmaf_rn(v, 32.0f, kMagic + 32.0f), kMagic),
                           kMagic + 64.0f);
     const int j = __float_as_int(f) - kMagicBits;
@@ -91,7 +114,7 @@ __device__ __forceinline__ uint32_t code_of(float v, const uint2* lut_lane) {
     const int j = __float_as_int(f) - kMagicBits;
     const uint2 e = lut_lane[j * 32];
     const uint32_t m = e.y + (a > __uint_as_float(e.x) ? 1u : 0u);
-    return (v < 0.0f && m != 0u) ? (m | 8u) : m;
+    return m + (v < -kFp4Mid0 ? 8u : 0u);
   }
 }
 
@@ -101,11 +124,10 @@ __device__ __forceinline__ uint2 lds_v2(uint32_t addr) {
   return r;
 }
 
-// Fast nearest code for |v| <= 1 + 2^-23, which holds whenever the block's
-// reciprocal 1/absmax is finite and the input finite: the bucket index is
-// then 0..64 without clamping.  The 7-bit mask only keeps non-finite input
-// inside the table (its code is unspecified).  lut_addr = shared address of
-// this lane's slot of bucket 0.
+// Nearest code for |v| <= 1 + 2^-23 (finite block, absmax in the normal
+// range) or NaN: the bucket index is then 0..64 (or 127 for NaN) without
+// clamping; the 7-bit mask only keeps the address inside the table.
+// lut_addr = shared address of this lane's slot of bucket 0.
 template <int QT>
 __device__ __forceinline__ uint32_t code_fast(float v, uint32_t lut_addr) {
   if constexpr (QT == kQtNF4) {
@@ -117,8 +139,31 @@ __device__ __forceinline__ uint32_t code_fast(float v, uint32_t lut_addr) {
     const float f = __fmaf_rn(a, 32.0f, kMagic);
     const uint2 e = lds_v2(lut_addr + ((__float_as_uint(f) & 0x7fu) << 8));
     const uint32_t m = e.y + (a > __uint_as_float(e.x) ? 1u : 0u);
-    return (v < 0.0f && m != 0u) ? (m | 8u) : m;
+    return m + (v < -kFp4Mid0 ? 8u : 0u);
   }
+}
+
+// Correctly rounded 1/a for a in [2^-126, 2^126): the hardware approximate
+// reciprocal y0 (within an ulp), one Newton-Raphson step y1 = y0 + y0 (1 -
+// a y0), then Markstein's correction y1 + y1 (1 - a y1), whose residual is
+// exact in one fma and whose last fma rounds once (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990).  The result equals the
+// correctly rounded reciprocal for every input of the range (checked
+// exhaustively against the round-to-nearest division by the library's
+// debug entry point bnb4_debug_check_rcp).
+__device__ __forceinline__ float rcp_rn_normal(float a) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(a));
+  float e = __fmaf_rn(-a, y, 1.0f);
+  y = __fmaf_rn(e, y, y);
+  e = __fmaf_rn(-a, y, 1.0f);
+  return __fmaf_rn(e, y, y);
+}
+
+// a in [2^-126, 2^126) -- the range of rcp_rn_normal.
+__device__ __forceinline__ bool normal_scale(float a) {
+  return __float_as_uint(a) - 0x00800000u < 0x7e000000u;
 }
 
 template <typename T>
@@ -159,89 +204,55 @@ struct Elem<uint16_t> {  // bf16 bit patterns
   }
 };
 
-// One warp tile: per absmax group of rows, the block absmax (per chunk, then
-// across the lanes -- and for LPB == 64 the two rows -- holding the block),
-// the masked absmax store, the codes and the packed store.  As soon as a row
-// is consumed its register slot is refilled with the same row of the warp's
-// next tile.  FULL (the tile lies entirely inside n) removes every bounds
-// check from the element loops.
-template <bool FULL, typename T, int BS, int QT, bool DQ, typename LoadRow>
-__device__ __forceinline__ void quant_tile(uint4 (&c)[kRows], int64_t e0, int64_t n,
-                                           int64_t nb, int64_t next, int64_t n_tiles,
-                                           int lane, const uint2* lut_lane, uint32_t lut_addr,
-                                           uint8_t* __restrict__ codes,
-                                           float* __restrict__ absmax, double& acc,
-                                           const LoadRow& load_row) {
+// Block absmax of a row group: the lane's chunk(s), then an xor-shuffle
+// reduction over the lanes holding the block (for LPB = 64 the two rows of
+// the group hold one block across the whole warp).
+template <typename T, int LPB, int RG>
+__device__ __forceinline__ float group_absmax(const uint4* ch) {
   constexpr int EPL = Elem<T>::kPerChunk;
-  constexpr int LPB = BS / EPL;
-  constexpr int ROW = 32 * EPL;
-  constexpr int RG = LPB == 64 ? 2 : 1;
+  float m = 0.0f;
 #pragma unroll
-  for (int r0 = 0; r0 < kRows; r0 += RG) {
-    float m = 0.0f;
+  for (int rr = 0; rr < RG; ++rr)
 #pragma unroll
-    for (int rr = 0; rr < RG; ++rr)
+    for (int i = 0; i < EPL; ++i) m = fmaxf(m, fabsf(Elem<T>::get(ch[rr], i)));
+  constexpr int kFirst = LPB == 64 ? 16 : LPB / 2;
 #pragma unroll
-      for (int i = 0; i < EPL; ++i) m = fmaxf(m, fabsf(Elem<T>::get(c[r0 + rr], i)));
-    constexpr int kFirst = LPB == 64 ? 16 : LPB / 2;
+  for (int o = kFirst; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  return m;
+}
+
+// Exact path for one chunk (any absmax, any bounds): the correctly rounded
+// reciprocal (0 for a zero block), the clamped lookup, padding nibbles of
+// elements at or past n set to 0, and a store that stays inside the
+// ceil(n/2) code bytes.  Out of line: it runs for rare row groups and the
+// one ragged tile, and keeps the streaming loop small.
+template <typename T, int QT>
+__device__ __noinline__ void chunk_exact(uint4 ch, float m, int64_t e, int64_t n,
+                                         uint8_t* codes, const uint2* lut_lane) {
+  constexpr int EPL = Elem<T>::kPerChunk;
+  const float inv = m == 0.0f ? 0.0f : __frcp_rn(m);
+  uint32_t p = 0;
 #pragma unroll
-    for (int o = kFirst; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    {
-      const bool writer = LPB == 64 ? lane == 0 : (lane % LPB) == 0;
-      const int64_t b = (e0 + static_cast<int64_t>(r0) * ROW) / BS +
-                        (LPB == 64 ? 0 : lane / LPB);
-      if (writer && (FULL || b < nb)) {
-        absmax[b] = m;
-        if constexpr (DQ) acc += static_cast<double>(m);
-      }
+  for (int q = EPL / 2 - 1; q >= 0; --q) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = 2 * q + h;
+      uint32_t c = code_of<QT>(__fmul_rn(Elem<T>::get(ch, i), inv), lut_lane);
+      if (e + i >= n) c = 0u;
+      p = p * 16u + c;
     }
-    const float inv = m == 0.0f ? 0.0f : __frcp_rn(m);
-    // a subnormal absmax below 2^-128 makes the reciprocal infinite: such
-    // rows (warp-uniform choice) take the clamped search, which reproduces
-    // the midpoint count for infinite and NaN products
-    const bool slow = __any_sync(0xffffffffu, isinf(inv));
+  }
+  uint8_t* dst = codes + e / 2;
+  if (e + EPL <= n) {
+    if constexpr (EPL == 8)
+      *reinterpret_cast<uint32_t*>(dst) = p;
+    else
+      *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(p);
+  } else {
+    const int64_t nbytes = (n + 1) / 2;
 #pragma unroll
-    for (int rr = 0; rr < RG; ++rr) {
-      const int r = r0 + rr;
-      const int64_t e = e0 + static_cast<int64_t>(r * 32 + lane) * EPL;
-      uint32_t packed = 0;
-      if (!slow) {
-#pragma unroll
-        for (int i = 0; i < EPL; i += 2) {
-          uint32_t c0 = code_fast<QT>(__fmul_rn(Elem<T>::get(c[r], i), inv), lut_addr);
-          uint32_t c1 = code_fast<QT>(__fmul_rn(Elem<T>::get(c[r], i + 1), inv), lut_addr);
-          if constexpr (!FULL) {  // padding nibbles of the ragged tail are 0
-            if (e + i >= n) c0 = 0u;
-            if (e + i + 1 >= n) c1 = 0u;
-          }
-          packed |= (c0 * 16u + c1) << (4 * i);
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < EPL; i += 2) {
-          uint32_t c0 = code_of<QT>(__fmul_rn(Elem<T>::get(c[r], i), inv), lut_lane);
-          uint32_t c1 = code_of<QT>(__fmul_rn(Elem<T>::get(c[r], i + 1), inv), lut_lane);
-          if constexpr (!FULL) {
-            if (e + i >= n) c0 = 0u;
-            if (e + i + 1 >= n) c1 = 0u;
-          }
-          packed |= (c0 * 16u + c1) << (4 * i);
-        }
-      }
-      if (next < n_tiles) c[r] = load_row(next, r);
-      uint8_t* dst = codes + e / 2;
-      if (FULL || e + EPL <= n) {
-        if constexpr (EPL == 8)
-          *reinterpret_cast<uint32_t*>(dst) = packed;
-        else
-          *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(packed);
-      } else {
-        const int64_t nbytes = (n + 1) / 2;
-#pragma unroll
-        for (int j = 0; j < EPL / 2; ++j)
-          if (e / 2 + j < nbytes) dst[j] = static_cast<uint8_t>(packed >> (8 * j));
-      }
-    }
+    for (int j = 0; j < EPL / 2; ++j)
+      if (e / 2 + j < nbytes) dst[j] = static_cast<uint8_t>(p >> (8 * j));
   }
 }
 
@@ -254,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   constexpr int LPB = BS / EPL;            // lanes (chunks) per block
   constexpr int ROW = 32 * EPL;            // elements per warp row
   constexpr int TILE = kRows * ROW;        // elements per warp tile
+  constexpr int RG = LPB == 64 ? 2 : 1;    // rows per block group
   static_assert(LPB == 64 || (LPB >= 4 && LPB <= 32), "blocksize");
   static_assert(TILE % BS == 0, "tile must hold whole blocks");
 
@@ -268,32 +280,86 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   const uint2* lut_lane = lut + lane;
   const uint32_t lut_addr = static_cast<uint32_t>(__cvta_generic_to_shared(lut_lane));
   const int64_t nb = (n + BS - 1) / BS;
-  const int64_t n_tiles = (n + TILE - 1) / TILE;
+  const int64_t n_full = n / TILE;  // tiles entirely inside n
   const int64_t n_warps = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
+  const bool writer = LPB == 64 ? lane == 0 : (lane % LPB) == 0;
   double acc = 0.0;
 
-  auto load_row = [&](int64_t tile, int r) -> uint4 {
-    const int64_t t0 = tile * TILE;
-    const int64_t e = t0 + static_cast<int64_t>(r * 32 + lane) * EPL;
-    if (t0 + TILE <= n) return ldg_stream_v4(x + e);
-    return Elem<T>::load_partial(x, e, n);
-  };
-
   int64_t tile = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + warp;
-  uint4 c[kRows];
-  if (tile < n_tiles) {
+  if (tile < n_full) {
+    // lane pointers at row 0 of the current tile; rows are immediate offsets
+    const int64_t e0 = tile * TILE + lane * EPL;
+    const T* xp = x + e0;
+    uint8_t* cp = codes + e0 / 2;
+    float* ap = absmax + tile * (TILE / BS) + (LPB == 64 ? 0 : lane / LPB);
+    const int64_t stride = n_warps * TILE;
+    uint4 c[kRows];
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) c[r] = load_row(tile, r);
+    for (int r = 0; r < kRows; ++r) c[r] = ldg_stream_v4(xp + r * ROW);
+    for (; tile < n_full; tile += n_warps) {
+      // the last tile of the warp refills from itself (the loads are unused)
+      const T* xn = tile + n_warps < n_full ? xp + stride : xp;
+#pragma unroll
+      for (int r0 = 0; r0 < kRows; r0 += RG) {
+        const float m = group_absmax<T, LPB, RG>(c + r0);
+        if (writer) ap[r0 * ROW / BS] = m;
+        if constexpr (DQ) acc += static_cast<double>(writer ? m : 0.0f);
+        if (__any_sync(0xffffffffu, !normal_scale(m))) {
+#pragma unroll
+          for (int rr = 0; rr < RG; ++rr)
+            chunk_exact<T, QT>(c[r0 + rr], m, tile * TILE + lane * EPL + (r0 + rr) * ROW,
+                               n, codes, lut_lane);
+        } else {
+          const float inv = rcp_rn_normal(m);
+#pragma unroll
+          for (int rr = 0; rr < RG; ++rr) {
+            const int r = r0 + rr;
+            uint32_t p = 0;
+#pragma unroll
+            for (int q = EPL / 2 - 1; q >= 0; --q) {
+              p = p * 16u +
+                  code_fast<QT>(__fmul_rn(Elem<T>::get(c[r], 2 * q), inv), lut_addr);
+              p = p * 16u +
+                  code_fast<QT>(__fmul_rn(Elem<T>::get(c[r], 2 * q + 1), inv), lut_addr);
+            }
+            if constexpr (EPL == 8)
+              *reinterpret_cast<uint32_t*>(cp + r * ROW / 2) = p;
+            else
+              *reinterpret_cast<uint16_t*>(cp + r * ROW / 2) = static_cast<uint16_t>(p);
+          }
+        }
+#pragma unroll
+        for (int rr = 0; rr < RG; ++rr) c[r0 + rr] = ldg_stream_v4(xn + (r0 + rr) * ROW);
+      }
+      xp = xn;
+      cp += stride / 2;
+      ap += stride / BS;
+    }
   }
-  for (; tile < n_tiles; tile += n_warps) {
-    const int64_t e0 = tile * TILE;
-    const int64_t next = tile + n_warps;
-    if (e0 + TILE <= n)
-      quant_tile<true, T, BS, QT, DQ>(c, e0, n, nb, next, n_tiles, lane, lut_lane,
-                                      lut_addr, codes, absmax, acc, load_row);
-    else
-      quant_tile<false, T, BS, QT, DQ>(c, e0, n, nb, next, n_tiles, lane, lut_lane,
-                                       lut_addr, codes, absmax, acc, load_row);
+
+  // the ragged tile (elements n_full * TILE .. n - 1) belongs to the warp
+  // whose tile sequence reaches it
+  if (n % TILE != 0 && tile == n_full) {
+    const int64_t t0 = n_full * TILE;
+#pragma unroll 1
+    for (int r0 = 0; r0 < kRows; r0 += RG) {
+      uint4 ch[RG];
+#pragma unroll
+      for (int rr = 0; rr < RG; ++rr)
+        ch[rr] = Elem<T>::load_partial(x, t0 + static_cast<int64_t>((r0 + rr) * 32 + lane) * EPL, n);
+      const float m = group_absmax<T, LPB, RG>(ch);
+      const int64_t b = (t0 + static_cast<int64_t>(r0) * ROW) / BS +
+                        (LPB == 64 ? 0 : lane / LPB);
+      if (writer && b < nb) {
+        absmax[b] = m;
+        if constexpr (DQ) acc += static_cast<double>(m);
+      }
+#pragma unroll
+      for (int rr = 0; rr < RG; ++rr) {
+        const int64_t e = t0 + static_cast<int64_t>((r0 + rr) * 32 + lane) * EPL;
+        if (e < n) chunk_exact<T, QT>(ch[rr], m, e, n, codes, lut_lane);
+      }
+    }
   }
 
   if constexpr (DQ) {
@@ -310,11 +376,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }
 
 // Double quantization of the absmax array: one warp per group of 256 blocks
-// (grid-strided over the groups), no CTA-wide synchronization.  Every warp
-// reduces the per-CTA partial sums of the quantize kernel in the same fixed
-// order (lane-strided fp64 sums, then a fixed xor tree), so all agree on the
-// offset; the sum is exact whenever the absmax values span few enough
-// binades, and then equals the oracle's sequential sum.
+// (grid-strided over the groups).  Every CTA first reduces the per-CTA
+// partial sums of the quantize kernel in the same fixed order -- thread i
+// adds partials i, i + 256, ... (independent loads, one round trip), then a
+// fixed xor tree per warp and the 8 warp sums in order -- so all CTAs agree
+// on the offset; the sum is exact whenever the absmax values span few
+// enough binades, and then equals the oracle's sequential sum.
 constexpr int kDqThreads = 256;
 
 __global__ void __launch_bounds__(kDqThreads)
@@ -322,13 +389,19 @@ __global__ void __launch_bounds__(kDqThreads)
                      const double* __restrict__ partials, int n_partials,
                      uint8_t* __restrict__ absmax_q, float* __restrict__ scale2,
                      float* __restrict__ offset) {
+  __shared__ double red[kDqThreads / 32];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   pdl_wait();  // the quantize kernel's absmax and partial sums are complete
   double sum = 0.0;
-  for (int i = lane; i < n_partials; i += 32) sum += partials[i];
+  for (int i = threadIdx.x; i < n_partials; i += kDqThreads) sum += partials[i];
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) red[warp] = sum;
+  __syncthreads();
+  sum = 0.0;
+#pragma unroll
+  for (int w = 0; w < kDqThreads / 32; ++w) sum += red[w];
   const float off = static_cast<float>(sum / static_cast<double>(nb));
   if (blockIdx.x == 0 && threadIdx.x == 0) offset[0] = off;
 
@@ -357,6 +430,41 @@ __global__ void __launch_bounds__(kDqThreads)
         absmax_q[b] = static_cast<uint8_t>(static_cast<int>(q) + 128);
       }
     }
+  }
+}
+
+// Every fp32 input of rcp_rn_normal's range against __frcp_rn.
+constexpr uint32_t kRcpFirst = 0x00800000u;              // 2^-126
+constexpr uint32_t kRcpCount = 0x7e800000u - kRcpFirst;  // up to 2^126
+
+__global__ void check_rcp_init(unsigned long long* res) {
+  res[0] = 0ull;
+  res[1] = 0xffffffffull;
+}
+
+__global__ void __launch_bounds__(256) check_rcp_kernel(unsigned long long* res) {
+  unsigned long long bad = 0;
+  uint32_t first = 0xffffffffu;
+  const uint32_t stride = gridDim.x * blockDim.x;
+  for (uint32_t i = blockIdx.x * blockDim.x + threadIdx.x; i < kRcpCount; i += stride) {
+    const uint32_t bits = kRcpFirst + i;
+    const float a = __uint_as_float(bits);
+    if (__float_as_uint(rcp_rn_normal(a)) != __float_as_uint(__frcp_rn(a))) {
+      ++bad;
+      first = min(first, bits);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    bad += __shfl_xor_sync(0xffffffffu, bad, o);
+    first = min(first, __shfl_xor_sync(0xffffffffu, first, o));
+  }
+  if ((threadIdx.x & 31) == 0 && bad != 0) {
+    atomicAdd(res, bad);
+    // the low word of res[1] holds the smallest mismatching pattern; the
+    // high word stays 0
+    atomicMin(reinterpret_cast<unsigned long long*>(res + 1),
+              static_cast<unsigned long long>(first));
   }
 }
 
@@ -393,6 +501,17 @@ cudaError_t dispatch_q(int qt, bool dq, int bs, const void* x, int64_t n,
 }
 
 }  // namespace
+
+cudaError_t launch_check_rcp(void* result, cudaStream_t s) {
+  auto* res = static_cast<unsigned long long*>(result);
+  cudaError_t e = launch_kernel(check_rcp_init, dim3(1), dim3(1), 0, s, false, res);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return e;
+  return launch_kernel(check_rcp_kernel, dim3(sms * 8), dim3(256), 0, s, false, res);
+}
 
 int quant_grid(int64_t n, int x_dtype, int num_sms) {
   const int64_t epl = x_dtype == BNB4_F32 ? 4 : 8;

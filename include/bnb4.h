@@ -235,6 +235,20 @@ BNB4_API int bnb4_debug_gemm_withhold(const void* X, int64_t M, int64_t K,
                                       const bnb4_qstate* W, int64_t N, void* Y,
                                       int32_t wait_limit_us, void* stream);
 
+/*
+ * Self-check of the quantize kernel's reciprocal (no counterpart on the
+ * pages).  bnb_quantize_4bit computes r = RN(1/absmax) for an absmax in
+ * [2^-126, 2^126) with an approximate reciprocal refined by Newton-Raphson
+ * and Markstein's correction; this call compares that value, bit for bit,
+ * with CUDA's round-to-nearest reciprocal for every fp32 input of the range
+ * (2,113,929,216 values, a few milliseconds).
+ *  result   device, 16 bytes, 8-byte aligned: receives {uint64 number of
+ *           mismatching inputs, uint32 smallest mismatching bit pattern
+ *           (0xffffffff when none), uint32 0}.  Overwritten, never read.
+ * Errors: INVALID_ARG, ALIGNMENT, CUDA.
+ */
+BNB4_API int bnb4_debug_check_rcp(void* result, void* stream);
+
 /* Static description of a status code; never NULL. */
 BNB4_API const char* bnb4_strerror(int status);
 

@@ -45,6 +45,15 @@ def test_small_ragged(qtype, bs, dq, N, K, B):
     case(N, K, B, bs, qtype, dq, seed=N * 31 + K)
 
 
+@pytest.mark.parametrize("N,K,B", [(4099, 4096, 1), (1030, 2112, 2), (517, 11008, 4),
+                                   (30001, 256, 8), (4096, 64, 1), (22, 1344, 2)])
+def test_row_groups_and_warp_splits(N, K, B):
+    """Every row-group shape (4 rows x 4 K-slices for B <= 2, 8 x 2 for B <=
+    4, 16 x 1 above), warps per CTA from 1 to 8, ragged N in every group
+    size and K that leaves slices and segments of the last step empty."""
+    case(N, K, B, 64, bnb4.NF4, True, seed=N + 3 * K + B)
+
+
 def test_gpu_quantized_weight_end_to_end():
     """GPU quantize then GEMV on the GPU state (the codes equal the oracle's,
     so the same fp64 reference applies)."""

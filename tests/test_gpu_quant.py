@@ -102,3 +102,61 @@ def test_codes_are_deterministic_and_independent_of_dq():
     assert torch.equal(a.codes, b.codes) and torch.equal(a.absmax, b.absmax)
     for k in ("codes", "absmax", "absmax_q", "scale2", "offset"):
         assert torch.equal(getattr(a, k), getattr(c, k))
+
+
+def _special_blocks(bs, n_blocks, rng):
+    """n_blocks blocks of N(0, 0.02^2) with special blocks spread through
+    them: every absmax class the kernel treats apart (zero, subnormal,
+    either side of 2^-126 and 2^126, near the fp32 maximum, infinite) and
+    NaN elements in otherwise normal blocks."""
+    x = (rng.standard_normal(bs * n_blocks) * 0.02).astype(np.float32)
+    f = lambda bits: np.array([bits], np.uint32).view(np.float32)[0]
+    specials = [
+        lambda b: b * 0.0,                                   # all zero
+        lambda b: np.full_like(b, -0.0),                     # all -0
+        lambda b: b * np.float32(1e-37),                     # subnormal and tiny
+        lambda b: np.where(np.arange(b.size) == 3, f(0x00800000), b * 1e-38),  # max 2^-126
+        lambda b: np.where(np.arange(b.size) == 5, f(0x007fffff), b * 1e-39),  # max just below
+        lambda b: np.where(np.arange(b.size) == 1, f(0x7e7fffff), b * 1e36),   # max just below 2^126
+        lambda b: np.where(np.arange(b.size) == 2, f(0x7e800000), b * 1e36),   # max 2^126
+        lambda b: np.where(np.arange(b.size) == 0, f(0x7f7fffff), b * 1e37),   # near FLT_MAX
+        lambda b: np.where(np.arange(b.size) == 7, np.float32(np.inf), b),     # +inf
+        lambda b: np.where(np.arange(b.size) == 9, np.float32(-np.inf), b),    # -inf
+        lambda b: np.where(np.arange(b.size) % 5 == 0, np.float32(np.nan), b), # NaNs, finite max
+    ]
+    for i, blk in enumerate(range(3, n_blocks, 7)):
+        sl = slice(blk * bs, (blk + 1) * bs)
+        x[sl] = specials[i % len(specials)](x[sl]).astype(np.float32)
+    return x
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("qtype", [bnb4.NF4, bnb4.FP4])
+@pytest.mark.parametrize("bs", [32, 64, 256])
+def test_special_values_in_full_tiles(dtype, qtype, bs):
+    """Zero, subnormal, boundary, huge and infinite block maxima and NaN
+    elements, placed inside full tiles (so the streaming loop's warp-uniform
+    choice between the fast and the exact path is exercised) and in the
+    ragged tail: codes and absmax equal the oracle's bit for bit."""
+    rng = np.random.default_rng(bs + (7 if dtype == "bf16" else 0) + 3 * qtype)
+    n = 16384 * 3 + 77 * bs // 32 + 5
+    nb = -(-n // bs)
+    x = _special_blocks(bs, nb, rng)[:n]
+    xt = torch.from_numpy(x)
+    if dtype == "bf16":
+        xt = xt.to(torch.bfloat16)
+    gpu, orc = run_both(xt, bs, qtype, False)
+    assert_state_equal(gpu, orc, False)
+
+
+def test_fast_reciprocal_exhaustive():
+    """The quantize kernel's reciprocal (approximation + Newton-Raphson +
+    Markstein correction) equals CUDA's round-to-nearest reciprocal for every
+    fp32 input in [2^-126, 2^126)."""
+    res = torch.zeros(2, dtype=torch.int64, device="cuda")
+    rc = bnb4.bnb4_debug_check_rcp(res.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert rc == 0, bnb4.bnb4_strerror(rc)
+    torch.cuda.synchronize()
+    mismatches, first = res.cpu().tolist()
+    assert mismatches == 0, "first mismatching input bits 0x%08x" % (first & 0xffffffff)
+    assert first & 0xffffffff == 0xffffffff
