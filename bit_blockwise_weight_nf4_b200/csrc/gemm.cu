@@ -57,6 +57,7 @@ constexpr int A_STAGE = MSUB * A_BYTES;  // 32 KB
 constexpr int B_BYTES = BNC * BK * 2;    // 16 KB
 constexpr int WP_BYTES = BNC * BK / 2;   // 4 KB packed codes
 constexpr int SCALE_FLOATS = 2 * BNC;    // 2 per row for blocksize 32
+constexpr int Y_BOX_BYTES = BM * 64 * 2;  // 16 KB output box (128 rows x 64 bf16)
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + SA * A_STAGE;
 constexpr int OFF_W = OFF_B + SB * B_BYTES;
@@ -74,6 +75,7 @@ static_assert(OFF_B % 1024 == 0 && OFF_W % 1024 == 0, "swizzled tiles need 1024-
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(kDeqWarps * 32 == NGROUPS * kGroupThreads, "groups");
 static_assert(SB == NGROUPS && SW % NGROUPS == 0, "group ownership of slots");
+static_assert(4 * MSUB * Y_BOX_BYTES <= OFF_W, "output boxes fit in the X and B rings");
 
 struct Bars {
   uint64_t afull[SA], aempty[SA];  // X tiles of both CTAs landed (leader) / consumed
@@ -207,6 +209,18 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       : "memory");
 }
 
+// TMA 2D store from this CTA's smem (a 128-byte swizzled box) to global
+// memory, tracked in the thread's bulk group; elements past the tensor's
+// edge are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x,
+                                             int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(x), "r"(y)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
 // 1024 bytes apart (stride byte offset), sm100 descriptor version 1.
 __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
@@ -304,12 +318,13 @@ __device__ __forceinline__ uint4 dq8(const Lut& l, uint32_t w) {
 template <int BS, int QT, bool DQ>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm4_kernel(const __grid_constant__ CUtensorMap map_x,
-                 const __grid_constant__ CUtensorMap map_w, int M, int N, int K,
+                 const __grid_constant__ CUtensorMap map_w,
+                 const __grid_constant__ CUtensorMap map_y, int M, int N, int K,
                  int n_pair_cols, const float* __restrict__ absmax,
                  const uint8_t* __restrict__ absmax_q,
                  const float* __restrict__ scale2,
-                 const float* __restrict__ offset, uint16_t* __restrict__ Y,
-                 int* err, uint64_t wait_limit_ns, int withhold_first_x) {
+                 const float* __restrict__ offset, int* err, uint64_t wait_limit_ns,
+                 int withhold_first_x) {
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the shared array by pointer
   // arithmetic (not an integer cast) so every access stays a shared-memory
@@ -533,27 +548,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive_cluster(map_to(bar(bars->bfull[sb]), 0));
     }
     // epilogue: accumulator j, TMEM lanes 32 q .. 32 q + 31 (rows of this
-    // CTA), a 64-column quarter h.  tcgen05.ld is warp-collective, so the
-    // go / no-go decision is uniform across the warp.
+    // CTA), a 64-column quarter h.  The tile goes through shared memory --
+    // the X and dequantized-weight rings are idle once every MMA has
+    // completed -- as 4 * MSUB boxes of 128 rows x 64 columns in the 128-byte
+    // swizzled layout of the TMA store, then leaves in 4 * MSUB tensor
+    // stores: whole 128-byte row segments instead of one 16-byte piece per
+    // row per store instruction.  tcgen05.ld is warp-collective, so the go /
+    // no-go decision is uniform across the warp; every epilogue warp reaches
+    // the named barrier, go or not.
     bool go = __all_sync(0xffffffffu, ok);
     if (go) {
       bool w = true;
       if (lane == 0) w = wait_bounded(bar(bars->accum), 0, bars, err);
       go = __shfl_sync(0xffffffffu, w ? 1 : 0, 0) != 0;
     }
+    uint8_t* ybuf = smem + OFF_A;  // 4 * MSUB boxes of 16 KB
     if (go) {
       asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
       const int q = warp & 3;                     // TMEM lane quarter
       const int h = (warp - kFirstDeqWarp) >> 2;  // 64-column quarter
+      const int r = q * 32 + lane;                // row of the CTA's 128
 #pragma unroll 1
       for (int j = 0; j < MSUB; ++j) {
-        const int row = m_pair + j * 2 * BM + static_cast<int>(rank) * BM + q * 32 + lane;
+        uint8_t* box = ybuf + (j * 4 + h) * Y_BOX_BYTES + r * 128;
 #pragma unroll 1
         for (int c = 0; c < 2; ++c) {
-          const int col = h * 64 + c * 32;
           uint32_t v[32];
           const uint32_t taddr =
-              tmem + (static_cast<uint32_t>(q * 32) << 16) + j * BNP + col;
+              tmem + (static_cast<uint32_t>(q * 32) << 16) + j * BNP + h * 64 + c * 32;
           asm volatile(
               "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
               "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -567,22 +589,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                 "=r"(v[30]), "=r"(v[31])
               : "r"(taddr));
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-          if (row < M && n_pair + col < N) {
-            uint16_t* dst = Y + static_cast<int64_t>(row) * N + n_pair + col;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              if (n_pair + col + 8 * i < N) {
-                const uint4 o = make_uint4(
-                    pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1])),
-                    pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
-                    pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
-                    pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
-                *reinterpret_cast<uint4*>(dst + 8 * i) = o;
-              }
-            }
+          for (int i = 0; i < 4; ++i) {  // 16-byte chunk c * 4 + i of the row
+            const uint4 o = make_uint4(
+                pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1])),
+                pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
+                pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
+                pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+            *reinterpret_cast<uint4*>(box + (((c * 4 + i) ^ (r & 7)) << 4)) = o;
           }
         }
       }
+      // the stores become visible to the TMA (async proxy)
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kDeqWarps * 32) : "memory");
+    if (threadIdx.x == kFirstDeqWarp * 32 && !*reinterpret_cast<volatile int*>(&bars->abort)) {
+      // boxes past the M or N edge are skipped; a box that straddles an edge
+      // is clipped by the TMA
+#pragma unroll 1
+      for (int bx = 0; bx < 4 * MSUB; ++bx) {
+        const int x = n_pair + (bx & 3) * 64;
+        const int y = m_pair + (bx >> 2) * 2 * BM + static_cast<int>(rank) * BM;
+        if (x < N && y < M) tma_store_2d(&map_y, smem_u32(ybuf + bx * Y_BOX_BYTES), x, y);
+      }
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // written before exit
     }
   }
 
@@ -644,12 +676,15 @@ cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W,
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  CUtensorMap mx, mw;
+  CUtensorMap mx, mw, my;
   if (!make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, BK, BM,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (!make_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.codes, K / 2, N, K / 2,
                    BK / 2, BNC, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return cudaErrorInvalidValue;
+  if (!make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, N * 2, 64, BM,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const int n_pair_cols = static_cast<int>((N + BNP - 1) / BNP);
   const int m_pairs = static_cast<int>((M + 2 * MSUB * BM - 1) / (2 * MSUB * BM));
@@ -665,10 +700,9 @@ cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W,
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, mx, mw, static_cast<int>(M), static_cast<int>(N),
+  return cudaLaunchKernelEx(&cfg, kern, mx, mw, my, static_cast<int>(M), static_cast<int>(N),
                             static_cast<int>(K), n_pair_cols, W.absmax, W.absmax_q,
-                            W.scale2, W.offset, static_cast<uint16_t*>(Y), err,
-                            wait_limit_ns, withhold);
+                            W.scale2, W.offset, err, wait_limit_ns, withhold);
 }
 
 template <int QT, bool DQ>

@@ -59,3 +59,12 @@ def test_small_ragged(qtype, bs, dq, M, N, K):
     if K % bs:
         pytest.skip("K must be a multiple of the blocksize")
     case(M, N, K, bs, qtype, dq, seed=M + N + K)
+
+
+@pytest.mark.parametrize("M,N,K", [(1500, 4104, 512),   # several M tiles, ragged M and N
+                                   (700, 2056, 320),    # ragged M, N and K steps
+                                   (2048, 11008, 256)]) # more tiles than SM pairs
+def test_tiles_ragged(M, N, K):
+    """Partial pair tiles at the M and N edges, and more tiles than SM pairs
+    (several waves)."""
+    case(M, N, K, 64, bnb4.NF4, True, seed=M + 7 * N + K, n_rows=64)
