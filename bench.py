@@ -72,6 +72,9 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=32,
                     help="decoder layers in the stack (32 = the Llama-7B workload)")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch the timed steps one call at a time instead of "
+                         "replaying them as one CUDA graph")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -237,8 +240,10 @@ class Step:
         self.launches_per_step = 5 * len(lins)  # quantize is 2 kernels
 
     def new_events(self):
+        """Timing events of one step; `external` makes a record captured in a
+        CUDA graph a timed event-record node."""
         import torch
-        return [[torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        return [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]
                 for _ in self.lins]
 
     def run(self, events=None):
@@ -390,6 +395,20 @@ def run_ours(args):
         raise RuntimeError("device error word set during warm-up")
 
     events = [step.new_events() for _ in range(args.steps)]
+    graph = None
+    if not args.eager:
+        # the K timed steps (every launch and the per-row events) as one CUDA
+        # graph: the same kernels on the same buffers, without per-call host
+        # launch overhead between them
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.graph(graph, stream=cap):
+            for k in range(args.steps):
+                step.run(events[k])
+        torch.cuda.current_stream().wait_stream(cap)
+        graph.replay()  # untimed: the graph's first launch
+        torch.cuda.synchronize()
     clocks = ClockSampler(physical_gpu_index(local))
     clocks.start()
     barrier(world)
@@ -397,8 +416,11 @@ def run_ours(args):
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record()
-    for k in range(args.steps):
-        step.run(events[k])
+    if graph is not None:
+        graph.replay()
+    else:
+        for k in range(args.steps):
+            step.run(events[k])
     t_end.record()
     torch.cuda.synchronize()
     barrier(world)
@@ -442,7 +464,9 @@ def run_ours(args):
                    "gemm_m": GEMM_M, "gemv_batch": 1,
                    "l2": "inputs larger than L2 (%.2f GB of bf16 weights), no flush"
                          % (sum(w.numel() * 2 for w in W) / 1e9),
-                   "parallelism": "replicas x%d" % world},
+                   "parallelism": "replicas x%d" % world,
+                   "launch": "eager, one call per kernel" if args.eager
+                             else "the timed steps replayed as one CUDA graph"},
         "roofline": {"bound": "tensor", "kernel": "gemm4 (fused dequant + tcgen05)",
                      "achieved": gemm_tflops, "peak": tf_sus, "unit": "TFLOP/s",
                      "frac": gemm_tflops / tf_sus, "traffic": gemm_traffic(),
@@ -456,6 +480,7 @@ def run_ours(args):
         "peaks": {"hbm_gbs": hbm, "bf16_tflops": tf_burst,
                   "bf16_tflops_sustained": tf_sus, "source": peak_src},
     }
+    del graph
     if not args.no_e2e:
         line["e2e"] = run_e2e(step, W, X, x, lins, world, args)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
