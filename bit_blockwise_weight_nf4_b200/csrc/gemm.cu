@@ -49,8 +49,12 @@ constexpr int BNP = 256;     // weight rows per pair (N of one MMA)
 constexpr int BNC = 128;     // weight rows per CTA
 constexpr int BK = 64;       // K per stage (one 128-byte swizzle row of bf16)
 constexpr int SA = 3;        // X stages
-constexpr int SB = 4;        // dequantized weight stages (one per group)
-constexpr int SW = 8;        // packed weight + scale stages
+// Dequantized weight stages: K step kt uses stage kt % SB, so the group that
+// dequantizes step kt + 4 (4 groups take every 4th step) refills the stage
+// the MMA of step kt + 4 - SB used; 6 stages give the groups 2 more MMA
+// steps of slack than 4 (measured: 4% faster on all three Llama shapes).
+constexpr int SB = 6;
+constexpr int SW = 4;        // packed weight + scale stages (one per group)
 constexpr int NGROUPS = 4;   // dequant groups (one K step each in flight)
 constexpr int A_BYTES = BM * BK * 2;     // 16 KB
 constexpr int A_STAGE = MSUB * A_BYTES;  // 32 KB
@@ -74,7 +78,7 @@ constexpr uint32_t kSuspendHintNs = 1000000;       // 1 ms per try_wait
 static_assert(OFF_B % 1024 == 0 && OFF_W % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(kDeqWarps * 32 == NGROUPS * kGroupThreads, "groups");
-static_assert(SB == NGROUPS && SW % NGROUPS == 0, "group ownership of slots");
+static_assert(SW == NGROUPS, "each group owns one packed-weight stage");
 static_assert(4 * MSUB * Y_BOX_BYTES <= OFF_W, "output boxes fit in the X and B rings");
 
 struct Bars {
@@ -518,6 +522,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float* sc = scales(sw);
       const float s0 = sc[r];
       const float s1 = BS == 32 ? sc[BNC + r] : s0;
+      // the next TMA load into this stage (async proxy) must not overtake
+      // these shared-memory reads (generic proxy): order them before the
+      // release
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(bars->wempty[sw]));
       if (!wait_bounded(bar(bars->bempty[sb]), ((kt / SB) & 1) ^ 1, bars, err)) {

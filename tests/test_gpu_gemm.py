@@ -68,3 +68,20 @@ def test_tiles_ragged(M, N, K):
     """Partial pair tiles at the M and N edges, and more tiles than SM pairs
     (several waves)."""
     case(M, N, K, 64, bnb4.NF4, True, seed=M + 7 * N + K, n_rows=64)
+
+
+@pytest.mark.parametrize("qtype,bs", [(bnb4.FP4, 64), (bnb4.NF4, 64), (bnb4.NF4, 32)])
+def test_repeated_launches_bit_identical(qtype, bs):
+    """The kernel's accumulation order is fixed, so repeated launches on the
+    same inputs must agree bit for bit; a race between the shared-memory
+    rings (a stage refilled while it is still being read) shows up here as
+    run-to-run differences long before it breaks the tolerance."""
+    W = synth.weight_bf16(4096, 4096, seed=bs + 11 * qtype).cuda().view(-1)
+    st = bnb4.quantize_4bit(W, bs, qtype, True)
+    X = synth.activations_bf16(2048, 4096, seed=bs + 11 * qtype + 1).cuda()
+    outs = [bnb4.gemm_4bit(X, st, 4096) for _ in range(16)]
+    torch.cuda.synchronize()
+    assert bnb4.bnb4_device_status(torch.cuda.current_stream().cuda_stream) == 0
+    ref = outs[0].view(torch.int16)
+    differing = [i for i in range(1, len(outs)) if not torch.equal(outs[i].view(torch.int16), ref)]
+    assert not differing, "launches %s differ from the first" % differing
