@@ -182,7 +182,7 @@ int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstate* W,
   if (!x || !y) return BNB4_ERR_INVALID_ARG;
   int rc = check_weight(W, N, K);
   if (rc != BNB4_OK) return rc;
-  if (B < 1 || B > 8) return BNB4_ERR_SHAPE;
+  if (B < 1 || B > 64) return BNB4_ERR_SHAPE;
   if (!aligned(x, 16) || !aligned(y, 2)) return BNB4_ERR_ALIGNMENT;
   int sms;
   if ((rc = num_sms(&sms)) != BNB4_OK) return rc;

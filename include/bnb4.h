@@ -194,7 +194,9 @@ BNB4_API int bnb_dequantize_4bit(const bnb4_qstate* st, void* out, int32_t out_d
  * exact, fp32 accumulation (order unspecified), one final rounding to bf16.
  *  x  device bf16 [B, K], 16-byte aligned;   y  device bf16 [B, N].
  *  W  quantization state of the weight [N, K] (W->n == N*K).
- * Constraints: 1 <= B <= 8; K % 64 == 0; K % W->blocksize == 0.
+ * Constraints: 1 <= B <= 64; K % 64 == 0; K % W->blocksize == 0.
+ * Batches above 8 run in groups of 8 columns over one dequantization of
+ * each weight fragment (the small-batch tier between decode and prefill).
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, SHAPE, CUDA.
  */
 BNB4_API int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstate* W,

@@ -48,10 +48,28 @@ def test_small_ragged(qtype, bs, dq, N, K, B):
 @pytest.mark.parametrize("N,K,B", [(4099, 4096, 1), (1030, 2112, 2), (517, 11008, 4),
                                    (30001, 256, 8), (4096, 64, 1), (22, 1344, 2)])
 def test_row_groups_and_warp_splits(N, K, B):
-    """Every row-group shape (4 rows x 4 K-slices for B <= 2, 8 x 2 for B <=
-    4, 16 x 1 above), warps per CTA from 1 to 8, ragged N in every group
-    size and K that leaves slices and segments of the last step empty."""
+    """16-row groups with ragged N, 1 to 8 warps holding K steps (K from 64
+    to 11008: a warp with no step, a last step with empty segments)."""
     case(N, K, B, 64, bnb4.NF4, True, seed=N + 3 * K + B)
+
+
+@pytest.mark.parametrize("B", [9, 16, 17, 24, 32, 33, 40, 63, 64])
+@pytest.mark.parametrize("N,K", [(1030, 2112), (4096, 4096)])
+def test_batch_column_groups(N, K, B):
+    """Small-batch tier: 2, 4 or 8 groups of 8 batch columns share one
+    dequantization of each weight fragment; groups wholly past B are
+    skipped, a partial last group reads a valid row and stores nothing."""
+    case(N, K, B, 64, bnb4.NF4, True, seed=N + 7 * K + B)
+
+
+@pytest.mark.parametrize("qtype", [bnb4.NF4, bnb4.FP4])
+@pytest.mark.parametrize("bs", [32, 64, 128, 256])
+@pytest.mark.parametrize("dq", [True, False])
+@pytest.mark.parametrize("B", [12, 30, 64])
+def test_batch_groups_every_format(qtype, bs, dq, B):
+    """Every blocksize / code table / scale format at each column-group
+    count, ragged N and K spanning several warp steps."""
+    case(259, 1280, B, bs, qtype, dq, seed=bs + 11 * B + int(dq))
 
 
 def test_gpu_quantized_weight_end_to_end():
@@ -67,3 +85,23 @@ def test_gpu_quantized_weight_end_to_end():
     g = bnb4.quantize_4bit(W.cuda().view(-1), 64, bnb4.NF4, True)
     y = bnb4.gemv_4bit(x.cuda(), g, N)
     check_linear(cpu_bits(y), y64, xb, What)
+
+
+@pytest.mark.parametrize("B", [17, 64])
+def test_batch_rows_past_B_untouched(B):
+    """The output rows past B (a partial last column group) are never
+    written: a canary row after y [B, N] keeps its bytes."""
+    N, K = 520, 1024
+    W = synth.weight_bf16(N, K, seed=B)
+    x = synth.activations_bf16(B, K, seed=B + 1)
+    st = oracle.quantize(synth.bf16_bits(W.view(-1)), 64, bnb4.NF4, True)
+    What = oracle.dequantize(st, oracle.BF16).reshape(N, K)
+    g = bnb4.state_from_arrays(st)
+    buf = torch.full(((B + 1) * N,), -7.0, dtype=torch.bfloat16, device="cuda")
+    y = buf[:B * N].view(B, N)
+    bnb4.gemv_4bit(x.cuda(), g, N, out=y)
+    torch.cuda.synchronize()
+    assert torch.all(buf[B * N:] == -7.0)
+    check_linear(cpu_bits(y), oracle.linear_ref(synth.bf16_bits(x), What),
+                 synth.bf16_bits(x), What)
+
