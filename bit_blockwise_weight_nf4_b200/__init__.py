@@ -258,7 +258,7 @@ def dequantize_4bit(state, out_dtype=None, out=None):
 
 
 def gemv_4bit(x, state, N, out=None):
-    """y = x @ What^T for bf16 x [B, K], B <= 64; What is the [N, K] weight."""
+    """y = x @ What^T for bf16 x [B, K], B <= 256; What is the [N, K] weight."""
     torch = _torch()
     B, K = x.shape
     if out is None:

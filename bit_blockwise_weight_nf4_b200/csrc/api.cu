@@ -98,6 +98,12 @@ int check_weight(const bnb4_qstate* W, int64_t N, int64_t K) {
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? BNB4_OK : BNB4_ERR_CUDA; }
 
+// Kernel choice by the number of token rows: the mma.sync GEMV up to 8 (one
+// MMA column group), the small-M tcgen05 kernel (weight rows as the MMA's M,
+// K split over a cluster) up to 256, the 2-CTA tcgen05 GEMM above.
+constexpr int64_t kGemvMaxB = 8;
+constexpr int64_t kSmallMaxM = 256;
+
 }  // namespace
 
 extern "C" {
@@ -182,12 +188,17 @@ int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstate* W,
   if (!x || !y) return BNB4_ERR_INVALID_ARG;
   int rc = check_weight(W, N, K);
   if (rc != BNB4_OK) return rc;
-  if (B < 1 || B > 64) return BNB4_ERR_SHAPE;
+  if (B < 1 || B > kSmallMaxM) return BNB4_ERR_SHAPE;
   if (!aligned(x, 16) || !aligned(y, 2)) return BNB4_ERR_ALIGNMENT;
   int sms;
   if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
-  return from_cuda(bnb4::launch_gemv(x, B, K, *W, N, y, sms,
-                                     static_cast<cudaStream_t>(stream)));
+  if (B <= kGemvMaxB)
+    return from_cuda(bnb4::launch_gemv(x, B, K, *W, N, y, sms,
+                                       static_cast<cudaStream_t>(stream)));
+  int* err;
+  if ((rc = error_word(&err)) != BNB4_OK) return rc;
+  return from_cuda(bnb4::launch_gemm_small(x, B, K, *W, N, y, err, sms,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstate* W,
@@ -202,6 +213,9 @@ int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstate* W,
   if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
   int* err;
   if ((rc = error_word(&err)) != BNB4_OK) return rc;
+  if (M <= kSmallMaxM)
+    return from_cuda(bnb4::launch_gemm_small(X, M, K, *W, N, Y, err, sms,
+                                             static_cast<cudaStream_t>(stream)));
   return from_cuda(bnb4::launch_gemm(X, M, K, *W, N, Y, err, sms,
                                      static_cast<cudaStream_t>(stream)));
 }

@@ -39,6 +39,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100.cuh"
 
 namespace bnb4 {
 namespace {
@@ -73,8 +74,6 @@ constexpr int kFirstDeqWarp = 3;
 constexpr int kThreads = (kFirstDeqWarp + kDeqWarps) * 32;
 constexpr int TMEM_COLS = 512;
 constexpr int SMEM_BYTES = OFF_BARS + 256 + 1024 /*align*/;
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s (normal launches)
-constexpr uint32_t kSuspendHintNs = 1000000;       // 1 ms per try_wait
 static_assert(OFF_B % 1024 == 0 && OFF_W % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(kDeqWarps * 32 == NGROUPS * kGroupThreads, "groups");
@@ -90,152 +89,6 @@ struct Bars {
   uint32_t tmem_base;
   int abort;
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ uint32_t cta_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// shared::cluster address of the same smem offset in CTA `rank` of the pair
-__device__ __forceinline__ uint32_t map_to(uint32_t addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
-               "barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
-}
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx_only(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.expect_tx.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-// arrive on a barrier of either CTA of the pair (cluster address), with
-// release at cluster scope
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cbar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cbar)
-               : "memory");
-}
-// try_wait with a suspend-time hint: the thread sleeps until the phase
-// completes or the hint (ns) expires, instead of polling.  CTA-scope acquire
-// for barriers only this CTA (or the MMA commit) arrives on; cluster scope
-// only where the peer CTA arrives (the leader's A and B "full" barriers) --
-// a cluster-scope acquire also invalidates L1, which the producers' scale
-// loads rely on.
-template <bool kCluster>
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  if constexpr (kCluster)
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
-        : "memory");
-  else
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
-        : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-// Bounded wait for the phase of `parity`; false when the CTA is aborting or
-// the time limit expired (then the device error word is set).
-template <bool kCluster = false>
-__device__ bool wait_bounded(uint32_t bar, uint32_t parity, Bars* bars, int* err) {
-  if (mbar_try_wait<kCluster>(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (;;) {
-    if (mbar_try_wait<kCluster>(bar, parity)) return true;
-    if (*reinterpret_cast<volatile int*>(&bars->abort)) return false;
-    if (global_ns() - t0 > bars->wait_limit_ns) {
-      atomicExch(err, 1);
-      *reinterpret_cast<volatile int*>(&bars->abort) = 1;
-      return false;
-    }
-  }
-}
-
-// Wait for operations this CTA started (TMA loads, MMAs) to land before it
-// tears down: unlike wait_bounded it ignores the abort flag -- those
-// operations complete on their own within microseconds -- and gives up after
-// min(limit, 10 ms) when the phase cannot complete because an arrival is
-// missing on the abort path.
-template <bool kCluster = false>
-__device__ void wait_drain(uint32_t bar, uint32_t parity, Bars* bars) {
-  const uint64_t lim = bars->wait_limit_ns < 10000000ull ? bars->wait_limit_ns : 10000000ull;
-  const uint64_t t0 = global_ns();
-  while (!mbar_try_wait<kCluster>(bar, parity))
-    if (global_ns() - t0 > lim) return;
-}
-
-// TMA 2D load into this CTA's smem, completing on this CTA's barrier.
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map,
-                                            int x, int y, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-// TMA 2D load into this CTA's smem, completing on a barrier of either CTA of
-// the pair (`cbar` is a shared::cluster address; no multicast).
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
-                                                 int x, int y, uint32_t cbar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(cbar)
-      : "memory");
-}
-
-// TMA 2D store from this CTA's smem (a 128-byte swizzled box) to global
-// memory, tracked in the thread's bulk group; elements past the tensor's
-// edge are not written.
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x,
-                                             int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.global.shared::cta.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-          reinterpret_cast<uint64_t>(map)),
-      "r"(src), "r"(x), "r"(y)
-      : "memory");
-}
-
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
-// 1024 bytes apart (stride byte offset), sm100 descriptor version 1.
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((addr >> 4) & 0x3fffu);
-  d |= static_cast<uint64_t>(1u) << 16;          // leading byte offset (unused)
-  d |= static_cast<uint64_t>(1024u >> 4) << 32;  // stride byte offset
-  d |= static_cast<uint64_t>(1u) << 46;          // descriptor version
-  d |= static_cast<uint64_t>(2u) << 61;          // SWIZZLE_128B
-  return d;
-}
 
 // Instruction descriptor: kind::f16, D fp32, A and B bf16, both K-major,
 // N = 256, M = 256 (two CTAs).
@@ -261,62 +114,6 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
       "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
       " [%0], m;\n\t}" ::"r"(bar)
       : "memory");
-}
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(s));
-  return d;
-}
-
-struct Lut {
-  uint32_t L[4], H[4];
-};
-
-template <int QT>
-__device__ __forceinline__ Lut make_lut(float ah) {
-  uint32_t P[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int c0 = 2 * j, c1 = 2 * j + 1;
-    const float t0 = QT == kQtNF4 ? nf4_value(c0)
-                                  : ((c0 & 8) ? -fp4_magnitude(c0 & 7) : fp4_magnitude(c0 & 7));
-    const float t1 = QT == kQtNF4 ? nf4_value(c1)
-                                  : ((c1 & 8) ? -fp4_magnitude(c1 & 7) : fp4_magnitude(c1 & 7));
-    P[j] = pack_bf16x2(__fmul_rn(t0, ah), __fmul_rn(t1, ah));
-  }
-  Lut l;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    l.L[q] = prmt(P[2 * q], P[2 * q + 1], 0x6420);
-    l.H[q] = prmt(P[2 * q], P[2 * q + 1], 0x7531);
-  }
-  return l;
-}
-
-// 8 codes of one packed 32-bit word (natural order k0..k7) -> 8 bf16 in k
-// order as 4 words.  The low 3 bits of each code select from the two
-// 8-entry halves of the table, bit 3 picks the half; one mask / shift of the
-// whole word serves both 4-code halves (prmt reads the low 16 selector bits).
-__device__ __forceinline__ uint4 dq8(const Lut& l, uint32_t w) {
-  const uint32_t sel = w & 0x77777777u;
-  const uint32_t mix = ((w >> 1) & 0x44444444u) | 0x32103210u;
-  uint4 o;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const uint32_t s = h ? sel >> 16 : sel;
-    const uint32_t m = h ? mix >> 16 : mix;
-    const uint32_t lo = prmt(prmt(l.L[0], l.L[1], s), prmt(l.L[2], l.L[3], s), m);
-    const uint32_t hi = prmt(prmt(l.H[0], l.H[1], s), prmt(l.H[2], l.H[3], s), m);
-    if (h == 0) {
-      o.x = prmt(lo, hi, 0x4051);
-      o.y = prmt(lo, hi, 0x6273);
-    } else {
-      o.z = prmt(lo, hi, 0x4051);
-      o.w = prmt(lo, hi, 0x6273);
-    }
-  }
-  return o;
 }
 
 template <int BS, int QT, bool DQ>
@@ -639,34 +436,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                  "r"(TMEM_COLS));
   }
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base,
-                 uint64_t inner, uint64_t outer, uint64_t row_bytes,
-                 uint32_t box_inner, uint32_t box_outer,
-                 CUtensorMapSwizzle swizzle) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int BS, int QT, bool DQ>

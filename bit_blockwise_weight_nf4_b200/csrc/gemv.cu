@@ -141,8 +141,8 @@ struct StepBuf {
   RawScale a[2][2];    // [row][block within the segment (blocksize 32)]
 };
 
-template <int BS, int QT, bool DQ, int kDepth, int NB>
-__global__ void __launch_bounds__(kThreads, NB >= 8 ? 1 : 2)
+template <int BS, int QT, bool DQ, int kDepth>
+__global__ void __launch_bounds__(kThreads, 2)
     gemv4_kernel(const uint16_t* __restrict__ x, int B, int64_t K,
                  const uint8_t* __restrict__ codes,
                  const float* __restrict__ absmax,
@@ -150,10 +150,7 @@ __global__ void __launch_bounds__(kThreads, NB >= 8 ? 1 : 2)
                  const float* __restrict__ scale2,
                  const float* __restrict__ offset, int64_t N,
                  uint16_t* __restrict__ y) {
-  // NB groups of 8 batch columns; each dequantized weight fragment feeds
-  // the MMAs of all NB groups
-  constexpr int CH = NB == 1 ? kChains : 1;  // accumulator chains per group
-  __shared__ float red[kWarps][32][4 * NB];
+  __shared__ float red[kWarps][32][4];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int g = lane >> 2;  // rows g and g + 8 of the group; batch column g of x
@@ -167,10 +164,7 @@ __global__ void __launch_bounds__(kThreads, NB >= 8 ? 1 : 2)
       warp < steps ? static_cast<int>((steps - warp + kWarps - 1) / kWarps) : 0;
   // batch columns beyond B read row B-1 (valid memory); their outputs are
   // never stored
-  const uint16_t* xrow[NB];
-#pragma unroll
-  for (int j = 0; j < NB; ++j)
-    xrow[j] = x + static_cast<int64_t>(8 * j + g < B ? 8 * j + g : B - 1) * K;
+  const uint16_t* xrow = x + static_cast<int64_t>(g < B ? g : B - 1) * K;
 
   auto issue = [&](int i, StepBuf& b) {
     const int64_t k0 = (static_cast<int64_t>(i) * kWarps + warp) * kKStep + 64 * t;
@@ -192,7 +186,7 @@ __global__ void __launch_bounds__(kThreads, NB >= 8 ? 1 : 2)
     }
   };
 
-  float acc[NB][CH][4] = {};
+  float acc[kChains][4] = {};
   StepBuf buf[kDepth];
 #pragma unroll
   for (int d = 0; d < kDepth; ++d)
@@ -218,6 +212,7 @@ __global__ void __launch_bounds__(kThreads, NB >= 8 ? 1 : 2)
         const int64_t kx = seg ? k0 : 0;  // x stays in bounds on a ragged edge
 #pragma unroll
         for (int p = 0; p < 8; ++p) {  // codes k0 + 8p .. +7 of both rows: two MMAs
+          const uint4 xb = __ldg(reinterpret_cast<const uint4*>(xrow + kx + 8 * p));
           const int h = p >> 2, wi = p & 3;
           const uint32_t w0 = wi == 0 ? buf[d].c[0][h].x : wi == 1 ? buf[d].c[0][h].y
                             : wi == 2 ? buf[d].c[0][h].z : buf[d].c[0][h].w;
@@ -226,85 +221,64 @@ __global__ void __launch_bounds__(kThreads, NB >= 8 ? 1 : 2)
           uint32_t o0[4], o1[4];
           dq8(lut[0][BS == 32 ? h : 0], w0, o0);
           dq8(lut[1][BS == 32 ? h : 0], w1, o1);
-#pragma unroll
-          for (int j = 0; j < NB; ++j) {
-            if (j > 0 && 8 * j >= B) break;  // warp-uniform: no columns left
-            const uint4 xb = __ldg(reinterpret_cast<const uint4*>(xrow[j] + kx + 8 * p));
-            mma_bf16(acc[j][(2 * p) % CH], o0[0], o1[0], o0[1], o1[1], xb.x, xb.y);
-            mma_bf16(acc[j][(2 * p + 1) % CH], o0[2], o1[2], o0[3], o1[3], xb.z, xb.w);
-          }
+          mma_bf16(acc[(2 * p) % kChains], o0[0], o1[0], o0[1], o1[1], xb.x, xb.y);
+          mma_bf16(acc[(2 * p + 1) % kChains], o0[2], o1[2], o0[3], o1[3], xb.z, xb.w);
         }
         if (i + kDepth < my_steps) issue(i + kDepth, buf[d]);
       }
     }
   }
 
-  // acc[j][.][v]: rows g (v = 0, 1) and g + 8 (v = 2, 3) of the group,
-  // batch columns 8 j + 2t and 8 j + 2t + 1
+  // acc[.]: rows g (0, 1) and g + 8 (2, 3) of the group, batch columns 2t and
+  // 2t + 1
 #pragma unroll
-  for (int j = 0; j < NB; ++j) {
+  for (int v = 0; v < 4; ++v) {
+    float sum = 0.f;
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      float sum = 0.f;
-#pragma unroll
-      for (int c = 0; c < CH; ++c) sum += acc[j][c][v];
-      red[warp][lane][4 * j + v] = sum;
-    }
+    for (int c = 0; c < kChains; ++c) sum += acc[c][v];
+    red[warp][lane][v] = sum;
   }
   __syncthreads();
   if (warp == 0) {
+    float s[4];
 #pragma unroll
-    for (int j = 0; j < NB; ++j) {
-      float sv[4];
+    for (int v = 0; v < 4; ++v) {
+      s[v] = 0.f;
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        sv[v] = 0.f;
+      for (int w = 0; w < kWarps; ++w) s[v] += red[w][lane][v];
+    }
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) sv[v] += red[w][lane][4 * j + v];
-      }
+    for (int r = 0; r < 2; ++r) {
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-#pragma unroll
-        for (int cb = 0; cb < 2; ++cb) {
-          const int bcol = 8 * j + 2 * t + cb;
-          if (ok[r] && bcol < B) {
-            const uint32_t o = pack_bf16x2(sv[2 * r + cb], 0.0f);
-            y[static_cast<int64_t>(bcol) * N + n[r]] = static_cast<uint16_t>(o);
-          }
+      for (int cb = 0; cb < 2; ++cb) {
+        const int bcol = 2 * t + cb;
+        if (ok[r] && bcol < B) {
+          const uint32_t o = pack_bf16x2(s[2 * r + cb], 0.0f);
+          y[static_cast<int64_t>(bcol) * N + n[r]] = static_cast<uint16_t>(o);
         }
       }
     }
   }
 }
 
-template <int BS, int QT, bool DQ, int kDepth, int NB>
+template <int BS, int QT, bool DQ, int kDepth>
 cudaError_t launch_t(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
                      int64_t N, void* y, cudaStream_t s) {
   const int64_t grid = (N + kRowsPerCta - 1) / kRowsPerCta;
-  return launch_kernel(gemv4_kernel<BS, QT, DQ, kDepth, NB>, dim3(static_cast<unsigned>(grid)),
+  return launch_kernel(gemv4_kernel<BS, QT, DQ, kDepth>, dim3(static_cast<unsigned>(grid)),
              dim3(kThreads), 0, s, false, static_cast<const uint16_t*>(x), static_cast<int>(B), K,
              static_cast<const uint8_t*>(W.codes), static_cast<const float*>(W.absmax),
              static_cast<const uint8_t*>(W.absmax_q), static_cast<const float*>(W.scale2),
              static_cast<const float*>(W.offset), N, static_cast<uint16_t*>(y));
 }
 
-template <int BS, int QT, bool DQ>
-cudaError_t launch_nb(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
-                      int64_t N, void* y, cudaStream_t s) {
-  // two K steps of loads in flight per lane (for K <= 4096 that is all of a
-  // warp's share), 2 CTAs of 8 warps resident per SM; batches above 8 run
-  // in groups of 8 columns over the same dequantized fragments
-  if (B <= 8) return launch_t<BS, QT, DQ, 2, 1>(x, B, K, W, N, y, s);
-  if (B <= 16) return launch_t<BS, QT, DQ, 2, 2>(x, B, K, W, N, y, s);
-  if (B <= 32) return launch_t<BS, QT, DQ, 2, 4>(x, B, K, W, N, y, s);
-  return launch_t<BS, QT, DQ, 2, 8>(x, B, K, W, N, y, s);
-}
-
 template <int BS, int QT>
 cudaError_t launch_bs(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
                       int64_t N, void* y, cudaStream_t s) {
-  if (W.double_quant) return launch_nb<BS, QT, true>(x, B, K, W, N, y, s);
-  return launch_nb<BS, QT, false>(x, B, K, W, N, y, s);
+  // two K steps of loads in flight per lane (for K <= 4096 that is all of a
+  // warp's share), 2 CTAs of 8 warps resident per SM
+  if (W.double_quant) return launch_t<BS, QT, true, 2>(x, B, K, W, N, y, s);
+  return launch_t<BS, QT, false, 2>(x, B, K, W, N, y, s);
 }
 
 template <int QT>

@@ -37,4 +37,10 @@ cudaError_t launch_gemm(const void* X, int64_t M, int64_t K,
                         int num_sms, cudaStream_t s, uint64_t wait_limit_ns = 0,
                         int withhold_first_x = 0);
 
+// Linear layer for 1..256 tokens (the small-batch tier): weight rows on the
+// MMA's M side, tokens on its N side, K split over a cluster.
+cudaError_t launch_gemm_small(const void* X, int64_t M, int64_t K,
+                              const bnb4_qstate& W, int64_t N, void* Y, int* err,
+                              int num_sms, cudaStream_t s, uint64_t wait_limit_ns = 0);
+
 }  // namespace bnb4

@@ -194,9 +194,9 @@ BNB4_API int bnb_dequantize_4bit(const bnb4_qstate* st, void* out, int32_t out_d
  * exact, fp32 accumulation (order unspecified), one final rounding to bf16.
  *  x  device bf16 [B, K], 16-byte aligned;   y  device bf16 [B, N].
  *  W  quantization state of the weight [N, K] (W->n == N*K).
- * Constraints: 1 <= B <= 64; K % 64 == 0; K % W->blocksize == 0.
- * Batches above 8 run in groups of 8 columns over one dequantization of
- * each weight fragment (the small-batch tier between decode and prefill).
+ * Constraints: 1 <= B <= 256; K % 64 == 0; K % W->blocksize == 0.
+ * B <= 8 runs the decode kernel (mma.sync, one 8-column group); larger
+ * batches run the small-batch tcgen05 kernel of bnb_gemm_4bit.
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, SHAPE, CUDA.
  */
 BNB4_API int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstate* W,
@@ -210,6 +210,10 @@ BNB4_API int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstat
  *     16-byte aligned.
  *  W  quantization state of the weight [N, K] (W->n == N*K).
  * Constraints: M >= 1; N % 8 == 0; K % 64 == 0; K % W->blocksize == 0.
+ * M <= 256 runs the small-batch kernel (the 128 weight rows of a CTA are
+ * the MMA's M side and the tokens its N; K split over a cluster of up to 8
+ * CTAs whose partial sums are added in rank order), larger M the 2-CTA
+ * prefill kernel (512 x 256 output tiles).  Both are deterministic.
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, SHAPE, CUDA.
  */
 BNB4_API int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstate* W,

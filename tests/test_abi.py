@@ -120,7 +120,7 @@ def test_gemv_argument_errors(lib):
                                   a["y"], None)
     assert call(x=None) == bnb4.ERR_INVALID_ARG
     assert call(B=0) == bnb4.ERR_SHAPE
-    assert call(B=65) == bnb4.ERR_SHAPE
+    assert call(B=257) == bnb4.ERR_SHAPE
     assert call(K=32, N=128) == bnb4.ERR_SHAPE          # K % 64
     assert call(N=65) == bnb4.ERR_SHAPE                 # W.n != N*K
     assert call(W=good_state(n=128 * 64, blocksize=128), N=128) == bnb4.ERR_SHAPE
