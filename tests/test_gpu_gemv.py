@@ -56,9 +56,8 @@ def test_row_groups_and_warp_splits(N, K, B):
 @pytest.mark.parametrize("B", [9, 16, 17, 24, 32, 33, 40, 63, 64])
 @pytest.mark.parametrize("N,K", [(1030, 2112), (4096, 4096)])
 def test_batch_column_groups(N, K, B):
-    """Small-batch tier: 2, 4 or 8 groups of 8 batch columns share one
-    dequantization of each weight fragment; groups wholly past B are
-    skipped, a partial last group reads a valid row and stores nothing."""
+    """bnb_gemv_4bit with 9..64 rows of x (the small-batch kernel: tokens on
+    the MMA's N side, padded to a multiple of 16 with zero rows)."""
     case(N, K, B, 64, bnb4.NF4, True, seed=N + 7 * K + B)
 
 
@@ -67,8 +66,8 @@ def test_batch_column_groups(N, K, B):
 @pytest.mark.parametrize("dq", [True, False])
 @pytest.mark.parametrize("B", [12, 30, 64])
 def test_batch_groups_every_format(qtype, bs, dq, B):
-    """Every blocksize / code table / scale format at each column-group
-    count, ragged N and K spanning several warp steps."""
+    """Every blocksize / code table / scale format through bnb_gemv_4bit
+    above 8 rows, ragged N and K spanning several K steps."""
     case(259, 1280, B, bs, qtype, dq, seed=bs + 11 * B + int(dq))
 
 
@@ -89,8 +88,8 @@ def test_gpu_quantized_weight_end_to_end():
 
 @pytest.mark.parametrize("B", [17, 64])
 def test_batch_rows_past_B_untouched(B):
-    """The output rows past B (a partial last column group) are never
-    written: a canary row after y [B, N] keeps its bytes."""
+    """The output rows past B (inside the last 16-token MMA column block)
+    are never written: a canary row after y [B, N] keeps its bytes."""
     N, K = 520, 1024
     W = synth.weight_bf16(N, K, seed=B)
     x = synth.activations_bf16(B, K, seed=B + 1)
