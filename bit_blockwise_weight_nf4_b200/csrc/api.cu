@@ -213,6 +213,9 @@ int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstate* W,
   if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
   int* err;
   if ((rc = error_word(&err)) != BNB4_OK) return rc;
+  if (M <= kGemvMaxB)
+    return from_cuda(bnb4::launch_gemv(X, M, K, *W, N, Y, sms,
+                                       static_cast<cudaStream_t>(stream)));
   if (M <= kSmallMaxM)
     return from_cuda(bnb4::launch_gemm_small(X, M, K, *W, N, Y, err, sms,
                                              static_cast<cudaStream_t>(stream)));

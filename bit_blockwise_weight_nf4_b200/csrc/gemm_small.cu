@@ -368,16 +368,27 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-constexpr int kOverheadSteps = 2;  // fill + epilogue of a CTA, in K steps
+// Cluster size S (K slices per 128-row tile).  Cost model, in K steps of one
+// CTA alone on an SM: every CTA pays kOverheadSteps (launch, first loads,
+// epilogue and cluster reduction) plus its steps, stretched by
+// kCoResidentStretch per extra CTA sharing the SM; CTAs beyond the resident
+// slots run in further waves.  Fitted to graph-timed sweeps of S = 1..8 on
+// the Llama-7B projection shapes at 16..256 tokens.
+constexpr double kOverheadSteps = 11.0;
+constexpr double kCoResidentStretch = 0.65;
 
-// Cluster size: the number of K slices per 128-row tile that spreads the
-// tiles' K steps most evenly over the SMs, counting a CTA's fixed cost.
-int choose_split(int64_t tiles, int k_tiles, int num_sms) {
+int choose_split(int64_t tiles, int k_tiles, int num_sms, int per_sm) {
   int best = 1;
-  int64_t best_cost = INT64_MAX;
+  double best_cost = 1e300;
+  const int64_t slots = static_cast<int64_t>(num_sms) * per_sm;
   for (int s = 1; s <= kMaxCluster && s <= k_tiles; ++s) {
-    const int64_t per_sm = (tiles * s + num_sms - 1) / num_sms;
-    const int64_t cost = per_sm * ((k_tiles + s - 1) / s + kOverheadSteps);
+    const int64_t ctas = tiles * s;
+    const int64_t waves = (ctas + slots - 1) / slots;
+    const int64_t resident = ctas < slots ? ctas : slots;
+    const int64_t share = (resident + num_sms - 1) / num_sms;  // CTAs per busy SM
+    const double stretch = 1.0 + kCoResidentStretch * static_cast<double>(share - 1);
+    const double cost = static_cast<double>(waves) *
+                        (((k_tiles + s - 1) / s) * stretch + kOverheadSteps);
     if (cost < best_cost) {
       best_cost = cost;
       best = s;
@@ -410,7 +421,10 @@ cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W, 
     return cudaErrorInvalidValue;
   const int64_t tiles = (N + ROWS - 1) / ROWS;
   const int k_tiles = static_cast<int>(K / BK);
-  const int S = choose_split(tiles, k_tiles, num_sms);
+  // CTAs per SM: shared memory allows 2 up to NT = 96, registers 2 at most
+  const int per_sm_smem = 233472 / (smem_bytes(nt) + 1024);
+  const int per_sm = per_sm_smem < 2 ? (per_sm_smem < 1 ? 1 : per_sm_smem) : 2;
+  const int S = choose_split(tiles, k_tiles, num_sms, per_sm);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(tiles * S));
   cfg.blockDim = dim3(kThreads);

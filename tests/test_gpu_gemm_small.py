@@ -2,7 +2,8 @@
 weight rows on the MMA's M side and K split over a cluster of 1..8 CTAs)
 against the fp64 oracle over the dequantized bf16 weight, with the tolerance
 of the method's brief.  Reached through both linear entry points: the GEMM
-for M <= 256 and the GEMV for 8 < B <= 256."""
+for 8 < M <= 256 (M <= 8 runs the decode kernel) and the GEMV for
+8 < B <= 256."""
 import numpy as np
 import pytest
 import torch
@@ -39,17 +40,18 @@ def case(M, N, K, bs=64, qtype=bnb4.NF4, dq=True, seed=0, entry="gemm"):
 @pytest.mark.parametrize("M", [1, 2, 8, 9, 15, 16, 17, 31, 33, 48, 63, 64, 65,
                                100, 128, 129, 200, 255, 256])
 def test_token_counts(M):
-    """Every token count class: NT = M rounded up to 16 (16..256), rows past
-    M read as zeros by the TMA and never stored; 9 weight-row tiles (the
+    """Every token count class: M <= 8 through the decode kernel, above it
+    NT = M rounded up to 16 (16..256), rows past M read as zeros by the TMA
+    and never stored; 9 weight-row tiles (the
     last ragged) with 33 K steps split over a 7-CTA cluster (5 or 4 steps
     per rank)."""
     case(M, 1032, 2112, seed=M)
 
 
-@pytest.mark.parametrize("N,K", [(16384, 256),   # cluster of 1
-                                 (8192, 512),    # 2
-                                 (6144, 960),    # 3
-                                 (4104, 512),    # 4, ragged N
+@pytest.mark.parametrize("N,K", [(16384, 256),   # cluster of 2 / 1 (24 / 160 tokens)
+                                 (8192, 512),    # 4 / 2
+                                 (6144, 960),    # 5 / 3
+                                 (4104, 512),    # 8 / 4, ragged N
                                  (2056, 320),    # 5: one K step per rank
                                  (512, 704),     # 6: ranks of 2 and 1 steps
                                  (264, 1280),    # 7, ragged N
@@ -58,8 +60,9 @@ def test_token_counts(M):
 @pytest.mark.parametrize("M", [24, 160])
 def test_cluster_splits(N, K, M):
     """The K split over clusters of every size the launcher picks (noted per
-    shape for 148 SMs), uneven step counts per rank, and the rank-order
-    reduction of the partial sums through distributed shared memory."""
+    shape for 148 SMs: 2 CTAs per SM at 24 tokens, 1 at 160), uneven step
+    counts per rank, and the rank-order reduction of the partial sums
+    through distributed shared memory."""
     case(M, N, K, seed=N + K + M)
 
 
