@@ -118,29 +118,46 @@ __device__ __forceinline__ uint32_t code_of(float v, const uint2* lut_lane) {
   }
 }
 
-__device__ __forceinline__ uint2 lds_v2(uint32_t addr) {
-  uint2 r;
-  asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
-  return r;
-}
-
-// Nearest code for |v| <= 1 + 2^-23 (finite block, absmax in the normal
-// range) or NaN: the bucket index is then 0..64 (or 127 for NaN) without
-// clamping; the 7-bit mask only keeps the address inside the table.
-// lut_addr = shared address of this lane's slot of bucket 0.
+// One Horner step of the fast path, p * 16 + code(v), for |v| <= 1 + 2^-23
+// (finite block, absmax in the normal range) or NaN: the bucket index is then
+// 0..64 (127 for the canonical NaN) without clamping, the 7-bit mask only
+// keeps the address inside the table, and code = base + (v > cand) as in
+// code_of.  lut_addr = shared address of this lane's slot of bucket 0.
+// Written out in PTX so that a step is 7 instructions (NF4; 11 for FP4):
+// bucket FMA, mask, table address, 64-bit table read, compare to the
+// candidate midpoint as a 0 / -1 mask, multiply-add of the base count,
+// subtract the mask.
 template <int QT>
-__device__ __forceinline__ uint32_t code_fast(float v, uint32_t lut_addr) {
+__device__ __forceinline__ uint32_t horner_code(uint32_t p, float v, uint32_t lut_addr) {
+  uint32_t out;
   if constexpr (QT == kQtNF4) {
-    const float f = __fmaf_rn(v, 32.0f, kMagic + 32.0f);
-    const uint2 e = lds_v2(lut_addr + ((__float_as_uint(f) & 0x7fu) << 8));
-    return e.y + (v > __uint_as_float(e.x) ? 1u : 0u);
+    asm("{\n\t.reg .b32 f, j, a, c, b, m, t;\n\t"
+        "fma.rn.f32 f, %1, 0f42000000, 0f4B400020;\n\t"  // v * 32 + 1.5 * 2^23 + 32
+        "and.b32 j, f, 127;\n\t"
+        "mad.lo.u32 a, j, 256, %2;\n\t"
+        "ld.shared.v2.u32 {c, b}, [a];\n\t"
+        "set.gt.u32.f32 m, %1, c;\n\t"
+        "mad.lo.u32 t, %3, 16, b;\n\t"
+        "sub.u32 %0, t, m;\n\t}"
+        : "=r"(out)
+        : "f"(v), "r"(lut_addr), "r"(p));
   } else {
-    const float a = fabsf(v);
-    const float f = __fmaf_rn(a, 32.0f, kMagic);
-    const uint2 e = lds_v2(lut_addr + ((__float_as_uint(f) & 0x7fu) << 8));
-    const uint32_t m = e.y + (a > __uint_as_float(e.x) ? 1u : 0u);
-    return m + (v < -kFp4Mid0 ? 8u : 0u);
+    asm("{\n\t.reg .b32 av, f, j, a, c, b, m, s, t;\n\t"
+        "abs.f32 av, %1;\n\t"
+        "fma.rn.f32 f, av, 0f42000000, 0f4B400000;\n\t"  // |v| * 32 + 1.5 * 2^23
+        "and.b32 j, f, 127;\n\t"
+        "mad.lo.u32 a, j, 256, %2;\n\t"
+        "ld.shared.v2.u32 {c, b}, [a];\n\t"
+        "set.gt.u32.f32 m, av, c;\n\t"
+        "set.lt.u32.f32 s, %1, 0fBD2AAAAB;\n\t"  // v < -kFp4Mid0: sign bit
+        "and.b32 s, s, 8;\n\t"
+        "mad.lo.u32 t, %3, 16, b;\n\t"
+        "sub.u32 t, t, m;\n\t"
+        "add.u32 %0, t, s;\n\t}"
+        : "=r"(out)
+        : "f"(v), "r"(lut_addr), "r"(p));
   }
+  return out;
 }
 
 // Correctly rounded 1/a for a in [2^-126, 2^126): the hardware approximate
@@ -317,10 +334,8 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             uint32_t p = 0;
 #pragma unroll
             for (int q = EPL / 2 - 1; q >= 0; --q) {
-              p = p * 16u +
-                  code_fast<QT>(__fmul_rn(Elem<T>::get(c[r], 2 * q), inv), lut_addr);
-              p = p * 16u +
-                  code_fast<QT>(__fmul_rn(Elem<T>::get(c[r], 2 * q + 1), inv), lut_addr);
+              p = horner_code<QT>(p, __fmul_rn(Elem<T>::get(c[r], 2 * q), inv), lut_addr);
+              p = horner_code<QT>(p, __fmul_rn(Elem<T>::get(c[r], 2 * q + 1), inv), lut_addr);
             }
             if constexpr (EPL == 8)
               *reinterpret_cast<uint32_t*>(cp + r * ROW / 2) = p;
