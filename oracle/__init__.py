@@ -7,7 +7,8 @@ import this package; the product library never does, and the two share no
 code.  The method, the page citations and every reading taken where the pages
 are silent are written out in the header comment of ``bnb4_oracle.c``.
 
-Arrays are numpy.  bf16 data travels as ``np.uint16`` bit patterns.
+Arrays are numpy.  bf16 data travels as ``np.uint16`` bit patterns, fp16
+data as ``np.float16`` (or its ``np.uint16`` bit patterns where stated).
 """
 import ctypes
 import os
@@ -20,6 +21,7 @@ NF4 = 0
 FP4 = 1
 F32 = 0
 BF16 = 1
+F16 = 2
 
 _lib = None
 
@@ -35,12 +37,17 @@ def _load():
         lib.orc_codebook.argtypes = [i32, p]
         lib.orc_bf16_rne.argtypes = [ctypes.c_float]
         lib.orc_bf16_rne.restype = ctypes.c_uint16
+        lib.orc_f16_rne.argtypes = [ctypes.c_float]
+        lib.orc_f16_rne.restype = ctypes.c_uint16
+        lib.orc_f16_to_float.argtypes = [ctypes.c_uint16]
+        lib.orc_f16_to_float.restype = ctypes.c_float
         lib.orc_nearest_code.argtypes = [i32, ctypes.c_float]
         lib.orc_quantize_4bit.argtypes = [p, i32, i64, i32, i32, i32,
                                           p, p, p, p, p, p]
         lib.orc_dequantize_4bit.argtypes = [p, i64, i32, i32, i32,
                                             p, p, p, p, p, i32]
-        lib.orc_linear_ref.argtypes = [p, i64, i64, p, i64, p, i64, p, i64, p]
+        lib.orc_linear_ref.argtypes = [p, i32, i64, i64, p, i64, p, i64, p, i64,
+                                       p, p]
         _lib = lib
     return _lib
 
@@ -66,6 +73,16 @@ def bf16_rne(f):
     return int(_load().orc_bf16_rne(ctypes.c_float(f)))
 
 
+def f16_rne(f):
+    """IEEE binary16 bit pattern of fp32 value ``f`` (round to nearest even)."""
+    return int(_load().orc_f16_rne(ctypes.c_float(f)))
+
+
+def f16_to_float(h):
+    """Exact fp32 value of binary16 bit pattern ``h``."""
+    return float(_load().orc_f16_to_float(ctypes.c_uint16(h)))
+
+
 def nearest_code(qtype, v):
     """Code of one normalised fp32 value."""
     return int(_load().orc_nearest_code(qtype, ctypes.c_float(v)))
@@ -76,7 +93,8 @@ def n_blocks(n, blocksize):
 
 
 def quantize(x, blocksize=64, qtype=NF4, double_quant=True):
-    """Quantize a flat fp32 array or bf16 bit-pattern (uint16) array.
+    """Quantize a flat fp32 array, bf16 bit-pattern (uint16) array or fp16
+    (float16) array.
 
     Returns a dict with ``codes`` (uint8, ceil(n/2)), ``absmax`` (fp32, nb),
     and for double quant ``absmax_q`` (uint8, nb), ``scale2`` (fp32,
@@ -88,8 +106,11 @@ def quantize(x, blocksize=64, qtype=NF4, double_quant=True):
         xd = F32
     elif x.dtype == np.uint16:
         xd = BF16
+    elif x.dtype == np.float16:
+        xd = F16
+        x = x.view(np.uint16)
     else:
-        raise TypeError("oracle quantize takes float32 or uint16 (bf16 bits)")
+        raise TypeError("oracle quantize takes float32, uint16 (bf16 bits) or float16")
     n = x.size
     nb = n_blocks(n, blocksize)
     st = {"n": n, "blocksize": blocksize, "qtype": qtype,
@@ -112,7 +133,7 @@ def quantize(x, blocksize=64, qtype=NF4, double_quant=True):
 
 def dequantize(st, out_dtype=F32):
     """Dequantize a state from :func:`quantize` (or one built from GPU
-    outputs) to fp32, or to bf16 bit patterns (uint16)."""
+    outputs) to fp32, or to bf16 / fp16 bit patterns (uint16)."""
     n = st["n"]
     out = np.zeros(n, np.float32 if out_dtype == F32 else np.uint16)
     dq = bool(st["double_quant"])
@@ -128,25 +149,29 @@ def dequantize(st, out_dtype=F32):
     return out
 
 
-def linear_ref(x_bits, W_bits, rows=None, cols=None):
-    """fp64 y = x . W^T for bf16 bit-pattern x [M, K] and W [N, K].
+def linear_ref(x_bits, W_bits, rows=None, cols=None, dtype=BF16, bias_bits=None):
+    """fp64 y = x . W^T (+ bias) for bit-pattern x [M, K], W [N, K] and bias
+    [N] in bf16 (``dtype`` BF16) or fp16 (F16).
 
     ``rows`` / ``cols`` optionally select a subset of x rows / W rows; the
     result is [len(rows), len(cols)].
     """
-    x_bits = np.ascontiguousarray(x_bits, np.uint16)
-    W_bits = np.ascontiguousarray(W_bits, np.uint16)
+    x_bits = np.ascontiguousarray(x_bits).view(np.uint16)
+    W_bits = np.ascontiguousarray(W_bits).view(np.uint16)
     M, K = x_bits.shape
     N, K2 = W_bits.shape
     if K != K2:
         raise ValueError("inner dimensions differ")
+    b = None if bias_bits is None else np.ascontiguousarray(bias_bits).view(np.uint16)
+    if b is not None and b.size != N:
+        raise ValueError("bias must have N entries")
     r = None if rows is None else np.ascontiguousarray(rows, np.int64)
     c = None if cols is None else np.ascontiguousarray(cols, np.int64)
     nr = M if r is None else r.size
     nc = N if c is None else c.size
     y = np.zeros((nr, nc), np.float64)
-    rc = _load().orc_linear_ref(_ptr(x_bits), M, K, _ptr(r), nr, _ptr(W_bits),
-                                N, _ptr(c), nc, _ptr(y))
+    rc = _load().orc_linear_ref(_ptr(x_bits), dtype, M, K, _ptr(r), nr, _ptr(W_bits),
+                                N, _ptr(c), nc, _ptr(b), _ptr(y))
     _check(rc, "linear_ref")
     return y
 
@@ -155,3 +180,8 @@ def bf16_bits_to_f64(bits):
     """Exact float64 values of bf16 bit patterns."""
     b = np.ascontiguousarray(bits, np.uint16).astype(np.uint32) << 16
     return b.view(np.float32).astype(np.float64)
+
+
+def f16_bits_to_f64(bits):
+    """Exact float64 values of fp16 bit patterns."""
+    return np.ascontiguousarray(bits, np.uint16).view(np.float16).astype(np.float64)

@@ -52,6 +52,15 @@
  *      nearest even of w.
  *  R10 Linear layer reference: y = x . What^T summed in fp64, What being the
  *      bf16 dequantized weight (the operand the tensor cores consume).
+ *  R11 fp16 compute type (the CSDN article's configuration section sets a
+ *      compute dtype beside the quant type and the double-quant flag; the
+ *      ossradar release notes' fused 4-bit GEMM takes fp16 or bf16
+ *      activations): an fp16 input is decoded exactly to fp32 before the
+ *      absmax; an fp16 dequantized weight is the IEEE binary16
+ *      round-to-nearest-even of w (overflow to infinity); the fp16 linear
+ *      layer uses fp16 x and What in R10.
+ *  R12 Bias (the release notes fuse the bias into the 4-bit GEMM): y = x .
+ *      What^T + bias[n], the bias in the compute type, added to the fp64 sum.
  */
 #include <math.h>
 #include <stddef.h>
@@ -97,6 +106,57 @@ static float bf16_bits_to_float(uint16_t b) {
   float f;
   memcpy(&f, &u, 4);
   return f;
+}
+
+/* R11: exact value of an IEEE binary16 bit pattern (1 sign bit, 5 exponent
+ * bits with bias 15, 10 fraction bits; exponent field 0 = zero or subnormal
+ * m * 2^-24, 31 = infinity or NaN). */
+static float f16_bits_to_float(uint16_t h) {
+  uint32_t sign = (uint32_t)(h >> 15) << 31;
+  uint32_t e = (h >> 10) & 31u, m = h & 1023u, u;
+  float f;
+  if (e == 0) {
+    f = (float)m * 0x1p-24f; /* exact: m < 2^10 */
+    return sign ? -f : f;
+  }
+  if (e == 31)
+    u = sign | 0x7f800000u | (m << 13);
+  else
+    u = sign | ((e + 112u) << 23) | (m << 13); /* rebias 15 -> 127 */
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+float orc_f16_to_float(uint16_t h) { return f16_bits_to_float(h); }
+
+/* R11: IEEE round-to-nearest-even of an fp32 value to binary16.  Values of
+ * magnitude 65520 or more (the midpoint past the largest finite 65504) become
+ * infinity; below 2^-14 the result is the subnormal RNE(|f| * 2^24) * 2^-24
+ * (the scaling by 2^24 is exact and rintf rounds half to even); NaN stays NaN
+ * with the quiet bit set. */
+uint16_t orc_f16_rne(float f) {
+  uint32_t u, sign, a;
+  memcpy(&u, &f, 4);
+  sign = (u >> 16) & 0x8000u;
+  a = u & 0x7fffffffu;
+  if (a > 0x7f800000u) return (uint16_t)(sign | 0x7e00u | ((a >> 13) & 0x3ffu));
+  if (a >= 0x477ff000u) return (uint16_t)(sign | 0x7c00u); /* >= 65520 or inf */
+  if (a >= 0x38800000u) {                                   /* >= 2^-14: normal */
+    uint32_t r = a - 0x38000000u;                           /* exponent - 112 */
+    r += 0x0fffu + ((r >> 13) & 1u);                        /* to nearest, ties even */
+    return (uint16_t)(sign | (r >> 13));
+  } else {
+    float mag;
+    memcpy(&mag, &a, 4);
+    return (uint16_t)(sign | (uint32_t)rintf(mag * 0x1p24f));
+  }
+}
+
+/* the element of an fp32 (0), bf16 (1) or fp16 (2) array as fp32 (exact) */
+static float elem_f32(const void* x, int dtype, int64_t i) {
+  if (dtype == 0) return ((const float*)x)[i];
+  if (dtype == 1) return bf16_bits_to_float(((const uint16_t*)x)[i]);
+  return f16_bits_to_float(((const uint16_t*)x)[i]);
 }
 
 /* R9: IEEE round-to-nearest-even of an fp32 value to bf16, from the bit
@@ -153,7 +213,7 @@ int orc_quantize_4bit(const void* x, int x_dtype, int64_t n, int blocksize,
                       float* offset, int* sum_exact) {
   int64_t nb, b, i;
   if (n <= 0 || !x || !codes || !absmax) return ORC_EINVAL;
-  if (x_dtype != 0 && x_dtype != 1) return ORC_EINVAL;
+  if (x_dtype != 0 && x_dtype != 1 && x_dtype != 2) return ORC_EINVAL;
   if (qtype != 0 && qtype != 1) return ORC_EINVAL;
   if (!valid_blocksize(blocksize)) return ORC_EINVAL;
   if (double_quant && (!absmax_q || !scale2 || !offset)) return ORC_EINVAL;
@@ -167,16 +227,14 @@ int orc_quantize_4bit(const void* x, int x_dtype, int64_t n, int blocksize,
     float a = 0.0f, r;
     /* R2 */
     for (i = lo; i < hi; ++i) {
-      float xi = x_dtype == 0 ? ((const float*)x)[i]
-                              : bf16_bits_to_float(((const uint16_t*)x)[i]);
+      float xi = elem_f32(x, x_dtype, i);
       if (fabsf(xi) > a) a = fabsf(xi);
     }
     absmax[b] = a;
     /* R5 */
     r = a == 0.0f ? 0.0f : 1.0f / a;
     for (i = lo; i < hi; ++i) {
-      float xi = x_dtype == 0 ? ((const float*)x)[i]
-                              : bf16_bits_to_float(((const uint16_t*)x)[i]);
+      float xi = elem_f32(x, x_dtype, i);
       float v = xi * r;
       int c = nearest_code(qtype, v);
       /* R7 */
@@ -254,7 +312,7 @@ static float decoded_absmax(int64_t b, int double_quant, const float* absmax,
 
 /*
  * Dequantize n elements.  out_dtype 0 writes fp32 w, 1 writes bf16 bit
- * patterns (uint16).  Uses absmax when !double_quant, else absmax_q, scale2
+ * patterns (uint16), 2 fp16 bit patterns (R11).  Uses absmax when !double_quant, else absmax_q, scale2
  * and offset.
  */
 int orc_dequantize_4bit(const uint8_t* codes, int64_t n, int blocksize,
@@ -266,7 +324,7 @@ int orc_dequantize_4bit(const uint8_t* codes, int64_t n, int blocksize,
   if (n <= 0 || !codes || !out) return ORC_EINVAL;
   if (qtype != 0 && qtype != 1) return ORC_EINVAL;
   if (!valid_blocksize(blocksize)) return ORC_EINVAL;
-  if (out_dtype != 0 && out_dtype != 1) return ORC_EINVAL;
+  if (out_dtype != 0 && out_dtype != 1 && out_dtype != 2) return ORC_EINVAL;
   if (double_quant ? (!absmax_q || !scale2 || !offset) : !absmax)
     return ORC_EINVAL;
   codebook(qtype, t);
@@ -277,22 +335,28 @@ int orc_dequantize_4bit(const uint8_t* codes, int64_t n, int blocksize,
     float w = t[c] * ah;
     if (out_dtype == 0)
       ((float*)out)[i] = w;
-    else
+    else if (out_dtype == 1)
       ((uint16_t*)out)[i] = orc_bf16_rne(w);
+    else
+      ((uint16_t*)out)[i] = orc_f16_rne(w);
   }
   return ORC_OK;
 }
 
 /*
- * R10: y[i][c] = sum_k x[rows[i]][k] * W[cols[c]][k] in fp64, for bf16 x
- * [M, K] and bf16 W [N, K] (both row-major bit patterns).  rows / cols may be
- * NULL to mean all rows (n_rows = M) / all columns (n_cols = N).
+ * R10, R11, R12: y[i][c] = sum_k x[rows[i]][k] * W[cols[c]][k] in fp64 (+
+ * bias[cols[c]] when bias is not NULL), for x [M, K], W [N, K] and bias [N]
+ * given as bf16 (dtype 1) or fp16 (dtype 2) bit patterns, row-major.
+ * rows / cols may be NULL to mean all rows (n_rows = M) / all columns
+ * (n_cols = N).
  */
-int orc_linear_ref(const uint16_t* x, int64_t M, int64_t K, const int64_t* rows,
-                   int64_t n_rows, const uint16_t* W, int64_t N,
-                   const int64_t* cols, int64_t n_cols, double* y) {
+int orc_linear_ref(const uint16_t* x, int dtype, int64_t M, int64_t K,
+                   const int64_t* rows, int64_t n_rows, const uint16_t* W,
+                   int64_t N, const int64_t* cols, int64_t n_cols,
+                   const uint16_t* bias, double* y) {
   int64_t i, c, k;
   if (!x || !W || !y || M <= 0 || K <= 0 || N <= 0) return ORC_EINVAL;
+  if (dtype != 1 && dtype != 2) return ORC_EINVAL;
   if (!rows) n_rows = M;
   if (!cols) n_cols = N;
   for (i = 0; i < n_rows; ++i) {
@@ -303,8 +367,9 @@ int orc_linear_ref(const uint16_t* x, int64_t M, int64_t K, const int64_t* rows,
       double acc = 0.0;
       if (nn < 0 || nn >= N) return ORC_EINVAL;
       for (k = 0; k < K; ++k)
-        acc += (double)bf16_bits_to_float(x[r * K + k]) *
-               (double)bf16_bits_to_float(W[nn * K + k]);
+        acc += (double)elem_f32(x, dtype, r * K + k) *
+               (double)elem_f32(W, dtype, nn * K + k);
+      if (bias) acc += (double)elem_f32(bias, dtype, nn);
       y[i * n_cols + c] = acc;
     }
   }

@@ -1,7 +1,8 @@
 """Pins for the CPU oracle: each test checks it against something other than
 itself -- the closed form through a library quantile function, the values the
 NF4 article prints, exact rational arithmetic, torch's bf16 cast, numpy's
-matmul, or brute force on tiny inputs.  No GPU is needed."""
+IEEE binary16 conversion, numpy's matmul, or brute force on tiny inputs.  No
+GPU is needed."""
 import os
 from fractions import Fraction
 from statistics import NormalDist
@@ -409,3 +410,91 @@ def test_nf4_beats_int4_on_normal_weights():
     q = np.clip(np.rint(blk / a * 7), -7, 7)
     mse_int4 = np.mean((q * a / 7 - blk) ** 2)
     assert mse_nf4 < mse_int4
+
+
+# ---- fp16 compute type and bias ---------------------------------------------
+
+def test_f16_rne_matches_numpy_cast():
+    """The oracle's binary16 rounding against numpy's IEEE float32 -> float16
+    conversion (round to nearest even): random values over every exponent,
+    exact ties, the subnormal range, the overflow boundary and specials."""
+    rng = np.random.default_rng(21)
+    vals = np.concatenate([
+        rng.standard_normal(4000).astype(np.float32),
+        (rng.standard_normal(2000) * 1e-5).astype(np.float32),   # subnormal f16
+        (rng.standard_normal(2000) * 1e-7).astype(np.float32),   # below 2^-24
+        (rng.standard_normal(2000) * 3e4).astype(np.float32),    # near overflow
+        rng.integers(0, 2 ** 31, 4000, dtype=np.uint32).view(np.float32),
+        np.array([0.0, -0.0, np.inf, -np.inf, 65504.0, 65519.99, 65520.0,
+                  -65520.0, 2 ** -14, 2 ** -24, 2 ** -25, 3 * 2 ** -26,
+                  2 ** -25 * 1.0000001, 1.0 + 2 ** -11, 1.0 + 3 * 2 ** -11,
+                  6.1e-5], np.float32)])
+    # exact ties at normal and subnormal spacing
+    ties = (rng.integers(0x38800000 >> 13, 0x477fe000 >> 13, 500).astype(np.uint32) << 13
+            | 0x1000).view(np.float32)
+    sub_ties = ((rng.integers(0, 1024, 200) * 2 + 1) * 2.0 ** -25).astype(np.float32)
+    vals = np.concatenate([vals, ties, sub_ties])
+    vals = vals[~np.isnan(vals)]
+    with np.errstate(over="ignore"):  # values past 65520 become infinity
+        want = vals.astype(np.float16).view(np.uint16)
+    got = np.array([oracle.f16_rne(float(v)) for v in vals], np.uint16)
+    assert np.array_equal(got, want), np.nonzero(got != want)[0][:8]
+    nan = oracle.f16_rne(float("nan"))
+    assert nan & 0x7c00 == 0x7c00 and nan & 0x3ff
+
+
+def test_f16_decode_is_exact_for_every_pattern():
+    """All 65536 binary16 patterns decode to the value numpy assigns them."""
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    want = pats.view(np.float16).astype(np.float32)
+    got = np.array([oracle.f16_to_float(int(h)) for h in pats], np.float32)
+    fin = ~np.isnan(want)
+    assert np.array_equal(got[fin].view(np.uint32), want[fin].view(np.uint32))
+    assert np.all(np.isnan(got[~fin]))
+
+
+@pytest.mark.parametrize("qtype", [oracle.NF4, oracle.FP4])
+def test_f16_input_is_exact_widening(qtype):
+    """Quantizing fp16 data equals quantizing the same values as fp32."""
+    rng = np.random.default_rng(22)
+    x = (rng.standard_normal(64 * 33 + 5) * 0.02).astype(np.float16)
+    x[::97] *= np.float16(20.0)
+    a = oracle.quantize(x, 64, qtype, True)
+    b = oracle.quantize(x.astype(np.float32), 64, qtype, True)
+    for k in ("codes", "absmax", "absmax_q", "scale2", "offset"):
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_dequant_f16_is_rne_of_fp32():
+    """The fp16 dequantized weight is numpy's fp16 rounding of the fp32 one."""
+    rng = np.random.default_rng(23)
+    x = (rng.standard_normal(64 * 40 + 3) * 0.02).astype(np.float32)
+    for qtype in (oracle.NF4, oracle.FP4):
+        st = oracle.quantize(x, 64, qtype, double_quant=True)
+        w32 = oracle.dequantize(st, oracle.F32)
+        w16 = oracle.dequantize(st, oracle.F16)
+        assert np.array_equal(w16, w32.astype(np.float16).view(np.uint16))
+
+
+def test_linear_ref_f16_and_bias_match_numpy_matmul():
+    """fp16 operands and a bias: the fp64 reference equals numpy's float64
+    matmul of the exact values plus the bias (summation order aside)."""
+    rng = np.random.default_rng(24)
+    x = rng.standard_normal((5, 96)).astype(np.float16)
+    W = (rng.standard_normal((7, 96)) * 0.05).astype(np.float16)
+    bias = rng.standard_normal(7).astype(np.float16)
+    y = oracle.linear_ref(x.view(np.uint16), W.view(np.uint16), dtype=oracle.F16,
+                          bias_bits=bias.view(np.uint16))
+    want = x.astype(np.float64) @ W.astype(np.float64).T + bias.astype(np.float64)
+    np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-12)
+    yb = oracle.linear_ref(x.view(np.uint16), W.view(np.uint16), dtype=oracle.F16)
+    np.testing.assert_allclose(y - yb, np.broadcast_to(bias.astype(np.float64), y.shape),
+                               rtol=1e-12, atol=1e-12)
+    # a bf16 bias is decoded as bf16
+    xb = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16)
+    Wb = torch.from_numpy(W.astype(np.float32)).to(torch.bfloat16)
+    bb = torch.from_numpy(bias.astype(np.float32)).to(torch.bfloat16)
+    bits = lambda t: t.view(torch.int16).numpy().view(np.uint16)
+    y2 = oracle.linear_ref(bits(xb), bits(Wb), bias_bits=bits(bb))
+    want2 = xb.double().numpy() @ Wb.double().numpy().T + bb.double().numpy()
+    np.testing.assert_allclose(y2, want2, rtol=1e-12, atol=1e-12)
