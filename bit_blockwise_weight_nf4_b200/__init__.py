@@ -5,12 +5,12 @@ quantize / dequantize / GEMV / GEMM path runs in the CUDA library:
 
 * raw ctypes entry points with the C names (``bnb_quantize_4bit``,
   ``bnb_quantize_4bit_noalloc``, ``bnb_dequantize_4bit``, ``bnb_gemv_4bit``, ``bnb_gemm_4bit``,
-  ``bnb4_query_sizes``, ``bnb4_device_status``, ``bnb4_strerror``,
-  ``bnb4_abi_version``), returning the C status;
+  ``bnb_linear_4bit``, ``bnb4_query_sizes``, ``bnb4_device_status``,
+  ``bnb4_strerror``, ``bnb4_abi_version``), returning the C status;
 * torch helpers (``QuantState``, ``quantize_4bit``, ``dequantize_4bit``,
-  ``gemv_4bit``, ``gemm_4bit``) that allocate device buffers with torch, call
-  the entry points on torch's current stream and raise ``Bnb4Error`` on a
-  non-zero status.
+  ``gemv_4bit``, ``gemm_4bit``, ``linear_4bit``) that allocate device buffers
+  with torch, call the entry points on torch's current stream and raise
+  ``Bnb4Error`` on a non-zero status.
 
 There is no CPU fallback: if ``libbnb4.so`` is missing, ``load()`` raises.
 Build it with ``python -m bit_blockwise_weight_nf4_b200.build``.
@@ -37,8 +37,9 @@ NF4 = 0
 FP4 = 1
 F32 = 0
 BF16 = 1
+F16 = 2
 
-ABI_VERSION = 1
+ABI_VERSION = 2
 
 
 class QState(ctypes.Structure):
@@ -86,6 +87,7 @@ def load():
         "bnb_dequantize_4bit": ([QP, p, i32, p], ctypes.c_int),
         "bnb_gemv_4bit": ([p, i64, i64, QP, i64, p, p], ctypes.c_int),
         "bnb_gemm_4bit": ([p, i64, i64, QP, i64, p, p], ctypes.c_int),
+        "bnb_linear_4bit": ([p, i32, i64, i64, QP, i64, p, p, p], ctypes.c_int),
         "bnb4_device_status": ([p, i32], ctypes.c_int),
         "bnb4_debug_gemm_withhold": ([p, i64, i64, QP, i64, p, i32, p], ctypes.c_int),
         "bnb4_debug_check_rcp": ([p, p], ctypes.c_int),
@@ -140,6 +142,10 @@ def bnb_gemv_4bit(x, B, K, W, N, y, stream):
 
 def bnb_gemm_4bit(X, M, K, W, N, Y, stream):
     return load().bnb_gemm_4bit(X, M, K, ctypes.byref(W), N, Y, stream)
+
+
+def bnb_linear_4bit(x, dtype, M, K, W, N, bias, y, stream):
+    return load().bnb_linear_4bit(x, dtype, M, K, ctypes.byref(W), N, bias, y, stream)
 
 
 def bnb4_debug_gemm_withhold(X, M, K, W, N, Y, wait_limit_us, stream):
@@ -213,7 +219,7 @@ class QuantState:
                                         self.absmax.numel() * 4)
 
 
-_DT = {"torch.float32": F32, "torch.bfloat16": BF16}
+_DT = {"torch.float32": F32, "torch.bfloat16": BF16, "torch.float16": F16}
 
 
 def workspace_for(state):
@@ -226,12 +232,12 @@ def workspace_for(state):
 
 def quantize_4bit(x, blocksize=64, qtype=NF4, double_quant=True, state=None,
                   workspace=None):
-    """Quantize a contiguous fp32 / bf16 CUDA tensor (flattened)."""
+    """Quantize a contiguous fp32 / bf16 / fp16 CUDA tensor (flattened)."""
     if not x.is_contiguous():
         raise ValueError("quantize_4bit takes a contiguous tensor")
     dt = _DT.get(str(x.dtype))
     if dt is None:
-        raise TypeError("quantize_4bit takes float32 or bfloat16")
+        raise TypeError("quantize_4bit takes float32, bfloat16 or float16")
     if state is None:
         state = QuantState(x.numel(), blocksize, qtype, double_quant, x.device)
     if workspace is None:
@@ -246,7 +252,7 @@ def quantize_4bit(x, blocksize=64, qtype=NF4, double_quant=True, state=None,
 
 
 def dequantize_4bit(state, out_dtype=None, out=None):
-    """Dequantize to a flat fp32 (default) or bf16 CUDA tensor."""
+    """Dequantize to a flat fp32 (default), bf16 or fp16 CUDA tensor."""
     torch = _torch()
     out_dtype = out_dtype or torch.float32
     if out is None:
@@ -278,6 +284,26 @@ def gemm_4bit(X, state, N, out=None):
     rc = bnb_gemm_4bit(X.data_ptr(), M, K, state.cstruct(), N, out.data_ptr(),
                        _stream())
     _check(rc, "bnb_gemm_4bit")
+    return out
+
+
+def linear_4bit(x, state, N, bias=None, out=None):
+    """y = x @ What^T (+ bias) for x [M, K] in bf16 or fp16 (the compute
+    type; What is the [N, K] weight dequantized in it, bias [N] of the same
+    dtype or None)."""
+    torch = _torch()
+    M, K = x.shape
+    dt = {"torch.bfloat16": BF16, "torch.float16": F16}.get(str(x.dtype))
+    if dt is None:
+        raise TypeError("linear_4bit takes bfloat16 or float16 activations")
+    if bias is not None and bias.dtype != x.dtype:
+        raise TypeError("bias must have the dtype of x")
+    if out is None:
+        out = torch.empty(M, N, dtype=x.dtype, device=x.device)
+    rc = bnb_linear_4bit(x.data_ptr(), dt, M, K, state.cstruct(), N,
+                         None if bias is None else bias.data_ptr(), out.data_ptr(),
+                         _stream())
+    _check(rc, "bnb_linear_4bit")
     return out
 
 

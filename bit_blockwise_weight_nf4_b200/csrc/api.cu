@@ -146,7 +146,8 @@ int bnb4_query_sizes(int64_t n, int32_t blocksize, int32_t double_quant,
 int bnb_quantize_4bit(const void* x, int32_t x_dtype, const bnb4_qstate* st,
                       void* workspace, size_t workspace_bytes, void* stream) {
   if (!x) return BNB4_ERR_INVALID_ARG;
-  if (x_dtype != BNB4_F32 && x_dtype != BNB4_BF16) return BNB4_ERR_UNSUPPORTED;
+  if (x_dtype != BNB4_F32 && x_dtype != BNB4_BF16 && x_dtype != BNB4_F16)
+    return BNB4_ERR_UNSUPPORTED;
   int rc = check_state_common(st);
   if (rc != BNB4_OK) return rc;
   if (!st->absmax) return BNB4_ERR_INVALID_ARG;
@@ -172,7 +173,8 @@ int bnb_quantize_4bit(const void* x, int32_t x_dtype, const bnb4_qstate* st,
 int bnb_dequantize_4bit(const bnb4_qstate* st, void* out, int32_t out_dtype,
                         void* stream) {
   if (!out) return BNB4_ERR_INVALID_ARG;
-  if (out_dtype != BNB4_F32 && out_dtype != BNB4_BF16) return BNB4_ERR_UNSUPPORTED;
+  if (out_dtype != BNB4_F32 && out_dtype != BNB4_BF16 && out_dtype != BNB4_F16)
+    return BNB4_ERR_UNSUPPORTED;
   int rc = check_state_read(st);
   if (rc != BNB4_OK) return rc;
   if (!aligned(out, 16)) return BNB4_ERR_ALIGNMENT;
@@ -193,11 +195,11 @@ int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstate* W,
   int sms;
   if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
   if (B <= kGemvMaxB)
-    return from_cuda(bnb4::launch_gemv(x, B, K, *W, N, y, sms,
+    return from_cuda(bnb4::launch_gemv(x, B, K, *W, N, y, nullptr, BNB4_BF16, sms,
                                        static_cast<cudaStream_t>(stream)));
   int* err;
   if ((rc = error_word(&err)) != BNB4_OK) return rc;
-  return from_cuda(bnb4::launch_gemm_small(x, B, K, *W, N, y, err, sms,
+  return from_cuda(bnb4::launch_gemm_small(x, B, K, *W, N, y, nullptr, BNB4_BF16, err, sms,
                                            static_cast<cudaStream_t>(stream)));
 }
 
@@ -214,13 +216,35 @@ int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstate* W,
   int* err;
   if ((rc = error_word(&err)) != BNB4_OK) return rc;
   if (M <= kGemvMaxB)
-    return from_cuda(bnb4::launch_gemv(X, M, K, *W, N, Y, sms,
+    return from_cuda(bnb4::launch_gemv(X, M, K, *W, N, Y, nullptr, BNB4_BF16, sms,
                                        static_cast<cudaStream_t>(stream)));
   if (M <= kSmallMaxM)
-    return from_cuda(bnb4::launch_gemm_small(X, M, K, *W, N, Y, err, sms,
-                                             static_cast<cudaStream_t>(stream)));
-  return from_cuda(bnb4::launch_gemm(X, M, K, *W, N, Y, err, sms,
+    return from_cuda(bnb4::launch_gemm_small(X, M, K, *W, N, Y, nullptr, BNB4_BF16, err,
+                                             sms, static_cast<cudaStream_t>(stream)));
+  return from_cuda(bnb4::launch_gemm(X, M, K, *W, N, Y, nullptr, BNB4_BF16, err, sms,
                                      static_cast<cudaStream_t>(stream)));
+}
+
+int bnb_linear_4bit(const void* x, int32_t dtype, int64_t M, int64_t K, const bnb4_qstate* W,
+                    int64_t N, const void* bias, void* y, void* stream) {
+  if (!x || !y) return BNB4_ERR_INVALID_ARG;
+  if (dtype != BNB4_BF16 && dtype != BNB4_F16) return BNB4_ERR_UNSUPPORTED;
+  int rc = check_weight(W, N, K);
+  if (rc != BNB4_OK) return rc;
+  if (M < 1 || M > (int64_t(1) << 31) || N > (int64_t(1) << 31)) return BNB4_ERR_SHAPE;
+  if (M > kSmallMaxM && N % 8 != 0) return BNB4_ERR_SHAPE;
+  if (!aligned(x, 16) || !aligned(y, M > kSmallMaxM ? 16 : 2) || !aligned(bias, 16))
+    return BNB4_ERR_ALIGNMENT;
+  int sms;
+  if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M <= kGemvMaxB)
+    return from_cuda(bnb4::launch_gemv(x, M, K, *W, N, y, bias, dtype, sms, s));
+  int* err;
+  if ((rc = error_word(&err)) != BNB4_OK) return rc;
+  if (M <= kSmallMaxM)
+    return from_cuda(bnb4::launch_gemm_small(x, M, K, *W, N, y, bias, dtype, err, sms, s));
+  return from_cuda(bnb4::launch_gemm(x, M, K, *W, N, y, bias, dtype, err, sms, s));
 }
 
 int bnb4_debug_gemm_withhold(const void* X, int64_t M, int64_t K,
@@ -237,7 +261,7 @@ int bnb4_debug_gemm_withhold(const void* X, int64_t M, int64_t K,
   if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
   int* err;
   if ((rc = error_word(&err)) != BNB4_OK) return rc;
-  return from_cuda(bnb4::launch_gemm(X, M, K, *W, N, Y, err, sms,
+  return from_cuda(bnb4::launch_gemm(X, M, K, *W, N, Y, nullptr, BNB4_BF16, err, sms,
                                      static_cast<cudaStream_t>(stream),
                                      static_cast<uint64_t>(wait_limit_us) * 1000u, 1));
 }

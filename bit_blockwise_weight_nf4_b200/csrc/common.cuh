@@ -83,6 +83,36 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Two fp32 -> packed fp16x2 (lo in bits 0..15), IEEE round to nearest even
+// (infinity past the largest finite value, subnormals kept).
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// The 16-bit compute formats (F = BNB4_BF16 or BNB4_F16): a packed pair from
+// two fp32 values, and the exact fp32 value of a 16-bit pattern.
+template <int F>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (F == BNB4_F16)
+    return pack_f16x2(lo, hi);
+  else
+    return pack_bf16x2(lo, hi);
+}
+template <int F>
+__device__ __forceinline__ float half_to_f32(uint32_t bits16) {
+  if constexpr (F == BNB4_F16) {
+    float f;
+    asm("{\n\t.reg .b16 h, u;\n\tmov.b32 {h, u}, %1;\n\tcvt.f32.f16 %0, h;\n\t}"
+        : "=f"(f)
+        : "r"(bits16));
+    return f;
+  } else {
+    return __uint_as_float(bits16 << 16);
+  }
+}
+
 // Programmatic dependent launch, used only inside one API call: a kernel
 // whose predecessor on the stream is the library's own previous kernel of the
 // same call (the double-quant kernel after the quantize kernel) is launched

@@ -28,15 +28,17 @@ constexpr int kThreads = 256;
 constexpr int kRows = 8;
 constexpr int kCtasPerSm = 4;  // resident CTAs per SM (64 registers)
 
-template <typename TO>
-struct Out;
-template <>
-struct Out<float> {
-  static constexpr int kPerChunk = 4;
+// Output element type per format: fp32 (4 per 16-byte chunk) or a 16-bit
+// pattern, bf16 or fp16 (8 per chunk).
+template <int OF>
+struct Out {
+  using T = uint16_t;
+  static constexpr int kPerChunk = 8;
 };
 template <>
-struct Out<uint16_t> {
-  static constexpr int kPerChunk = 8;
+struct Out<BNB4_F32> {
+  using T = float;
+  static constexpr int kPerChunk = 4;
 };
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
@@ -86,14 +88,14 @@ __device__ __forceinline__ void chunk_values(uint32_t cw, float ah, const float*
   }
 }
 
-template <typename TO, int EPL>
-__device__ __forceinline__ void store_chunk(TO* dst, const float (&w)[EPL]) {
+template <int OF, int EPL>
+__device__ __forceinline__ void store_chunk(typename Out<OF>::T* dst, const float (&w)[EPL]) {
   if constexpr (EPL == 4) {
     *reinterpret_cast<float4*>(dst) = make_float4(w[0], w[1], w[2], w[3]);
   } else {
     *reinterpret_cast<uint4*>(dst) =
-        make_uint4(pack_bf16x2(w[0], w[1]), pack_bf16x2(w[2], w[3]),
-                   pack_bf16x2(w[4], w[5]), pack_bf16x2(w[6], w[7]));
+        make_uint4(pack2<OF>(w[0], w[1]), pack2<OF>(w[2], w[3]),
+                   pack2<OF>(w[4], w[5]), pack2<OF>(w[6], w[7]));
   }
 }
 
@@ -105,14 +107,16 @@ __device__ __forceinline__ uint32_t load_codes(const uint8_t* p) {
     return __ldg(reinterpret_cast<const uint16_t*>(p));
 }
 
-template <typename TO, bool DQ, int BS>
+template <int OF, bool DQ, int BS>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     dequant4_kernel(const uint8_t* __restrict__ codes, int64_t n, int qtype,
                     const float* __restrict__ absmax,
                     const uint8_t* __restrict__ absmax_q,
                     const float* __restrict__ scale2,
-                    const float* __restrict__ offset, TO* __restrict__ out) {
-  constexpr int EPL = Out<TO>::kPerChunk;
+                    const float* __restrict__ offset,
+                    typename Out<OF>::T* __restrict__ out) {
+  using TO = typename Out<OF>::T;
+  constexpr int EPL = Out<OF>::kPerChunk;
   constexpr int ROW = 32 * EPL;
   constexpr int TILE = kRows * ROW;
   static_assert(TILE % BS == 0, "tile must hold whole blocks");
@@ -154,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         chunk_values<EPL>(cw[r], decode<DQ>(raw[r], off), table, w);
         cw[r] = load_codes<EPL>(cn + r * ROW / 2);
         raw[r] = load_raw<DQ>(bn + rb(r), absmax, absmax_q, scale2);
-        store_chunk<TO, EPL>(op + r * ROW, w);
+        store_chunk<OF, EPL>(op + r * ROW, w);
       }
       cp = cn;
       b0 = bn;
@@ -178,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       chunk_values<EPL>(cwp, decode<DQ>(load_raw<DQ>(e / BS, absmax, absmax_q, scale2), off),
                         table, w);
       if (e + EPL <= n) {
-        store_chunk<TO, EPL>(out + e, w);
+        store_chunk<OF, EPL>(out + e, w);
       } else {
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
@@ -186,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
             if constexpr (EPL == 4)
               out[e + i] = w[i];
             else
-              out[e + i] = static_cast<uint16_t>(pack_bf16x2(w[i], 0.0f) & 0xffffu);
+              out[e + i] = static_cast<uint16_t>(pack2<OF>(w[i], 0.0f) & 0xffffu);
           }
         }
       }
@@ -194,9 +198,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   }
 }
 
-template <typename TO, bool DQ, int BS>
+template <int OF, bool DQ, int BS>
 cudaError_t launch(const bnb4_qstate& st, void* out, int grid, cudaStream_t s) {
-  return launch_kernel(dequant4_kernel<TO, DQ, BS>, dim3(grid), dim3(kThreads), 0, s, false,
+  using TO = typename Out<OF>::T;
+  return launch_kernel(dequant4_kernel<OF, DQ, BS>, dim3(grid), dim3(kThreads), 0, s, false,
                        static_cast<const uint8_t*>(st.codes), st.n,
                        static_cast<int>(st.qtype), static_cast<const float*>(st.absmax),
                        static_cast<const uint8_t*>(st.absmax_q),
@@ -204,13 +209,13 @@ cudaError_t launch(const bnb4_qstate& st, void* out, int grid, cudaStream_t s) {
                        static_cast<const float*>(st.offset), static_cast<TO*>(out));
 }
 
-template <typename TO, bool DQ>
+template <int OF, bool DQ>
 cudaError_t launch_bs(const bnb4_qstate& st, void* out, int grid, cudaStream_t s) {
   switch (st.blocksize) {
-    case 32: return launch<TO, DQ, 32>(st, out, grid, s);
-    case 64: return launch<TO, DQ, 64>(st, out, grid, s);
-    case 128: return launch<TO, DQ, 128>(st, out, grid, s);
-    default: return launch<TO, DQ, 256>(st, out, grid, s);
+    case 32: return launch<OF, DQ, 32>(st, out, grid, s);
+    case 64: return launch<OF, DQ, 64>(st, out, grid, s);
+    case 128: return launch<OF, DQ, 128>(st, out, grid, s);
+    default: return launch<OF, DQ, 256>(st, out, grid, s);
   }
 }
 
@@ -230,10 +235,13 @@ cudaError_t launch_dequantize(const bnb4_qstate& st, void* out, int out_dtype,
                               int grid, cudaStream_t s) {
   const bool dq = st.double_quant != 0;
   if (out_dtype == BNB4_F32)
-    return dq ? launch_bs<float, true>(st, out, grid, s)
-              : launch_bs<float, false>(st, out, grid, s);
-  return dq ? launch_bs<uint16_t, true>(st, out, grid, s)
-            : launch_bs<uint16_t, false>(st, out, grid, s);
+    return dq ? launch_bs<BNB4_F32, true>(st, out, grid, s)
+              : launch_bs<BNB4_F32, false>(st, out, grid, s);
+  if (out_dtype == BNB4_F16)
+    return dq ? launch_bs<BNB4_F16, true>(st, out, grid, s)
+              : launch_bs<BNB4_F16, false>(st, out, grid, s);
+  return dq ? launch_bs<BNB4_BF16, true>(st, out, grid, s)
+            : launch_bs<BNB4_BF16, false>(st, out, grid, s);
 }
 
 }  // namespace bnb4

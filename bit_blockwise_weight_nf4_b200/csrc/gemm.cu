@@ -1,7 +1,9 @@
 // gemm.cu -- prefill GEMM with fused 4-bit weight dequantization, sm_100a:
-//   Y[m, n] = bf16( sum_k X[m, k] * What[n, k] ),
-//   What[n, k] = bf16(RN(t[code] * a_hat))  (exact dequantized weight),
-// fp32 accumulation in tensor memory by tcgen05.mma (kind::f16, bf16 inputs).
+//   Y[m, n] = h( sum_k X[m, k] * What[n, k] + bias[n] ),
+//   What[n, k] = h(RN(t[code] * a_hat))  (exact dequantized weight),
+// h = round to the 16-bit compute format (bf16 or fp16, nearest even), bias
+// optional; fp32 accumulation in tensor memory by tcgen05.mma (kind::f16,
+// bf16 or fp16 inputs).
 //
 // Method: the fused 4-bit dequantize + GEMM of bitsandbytes' release notes
 // 0.50.0 (ossradar page), nested quantization decoded inside, over the NF4 /
@@ -90,19 +92,21 @@ struct Bars {
   int abort;
 };
 
-// Instruction descriptor: kind::f16, D fp32, A and B bf16, both K-major,
-// N = 256, M = 256 (two CTAs).
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+// Instruction descriptor: kind::f16, D fp32, A and B both bf16 (format code
+// 1) or both fp16 (0), K-major, N = 256, M = 256 (two CTAs).
+template <int F>
+constexpr uint32_t kIdesc = (1u << 4) | (F == BNB4_F16 ? 0u : (1u << 7) | (1u << 10)) |
                             (static_cast<uint32_t>(BNP >> 3) << 17) |
                             (static_cast<uint32_t>((2 * BM) >> 4) << 24);
 
-__device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc,
-                                               uint64_t bdesc, uint32_t accumulate) {
+template <int F>
+__device__ __forceinline__ void umma16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate));
+      "l"(adesc), "l"(bdesc), "r"(kIdesc<F>), "r"(accumulate));
 }
 
 // Arrive on the barrier at `bar`'s offset in both CTAs of the pair once all
@@ -116,7 +120,7 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
       : "memory");
 }
 
-template <int BS, int QT, bool DQ>
+template <int BS, int QT, bool DQ, int F>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm4_kernel(const __grid_constant__ CUtensorMap map_x,
                  const __grid_constant__ CUtensorMap map_w,
@@ -124,8 +128,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                  int n_pair_cols, const float* __restrict__ absmax,
                  const uint8_t* __restrict__ absmax_q,
                  const float* __restrict__ scale2,
-                 const float* __restrict__ offset, int* err, uint64_t wait_limit_ns,
-                 int withhold_first_x) {
+                 const float* __restrict__ offset, const uint16_t* __restrict__ bias,
+                 int* err, uint64_t wait_limit_ns, int withhold_first_x) {
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the shared array by pointer
   // arithmetic (not an integer cast) so every access stays a shared-memory
@@ -291,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t a_addr = smem_u32(a_tile(sa, j));
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
-            umma_bf16_pair(tmem + j * BNP, sw128_desc(a_addr + 32 * k),
+            umma16_pair<F>(tmem + j * BNP, sw128_desc(a_addr + 32 * k),
                            sw128_desc(b_addr + 32 * k), (kt > 0 || k > 0) ? 1u : 0u);
         }
         umma_commit_pair(bar(bars->aempty[sa]));
@@ -332,9 +336,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* brow = b_tile(sb) + r * 128;
       const int swz = r & 7;
       if (row_ok) {
-        const Lut l0 = make_lut<QT>(s0);
+        const Lut l0 = make_lut<QT, F>(s0);
         Lut l1 = l0;
-        if constexpr (BS == 32) l1 = make_lut<QT>(s1);
+        if constexpr (BS == 32) l1 = make_lut<QT, F>(s1);
         const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
         for (int p = 0; p < 8; ++p) {
@@ -396,11 +400,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
           for (int i = 0; i < 4; ++i) {  // 16-byte chunk c * 4 + i of the row
-            const uint4 o = make_uint4(
-                pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1])),
-                pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3])),
-                pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5])),
-                pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7])));
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(v[8 * i + e]);
+            // bias of the chunk's 8 columns (N % 8 == 0: a chunk is wholly
+            // inside or outside the N edge)
+            const int col0 = n_pair + h * 64 + c * 32 + 8 * i;
+            if (bias && col0 < N) {
+              const uint4 bb = __ldg(reinterpret_cast<const uint4*>(bias + col0));
+              const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                f[e] = __fadd_rn(f[e], half_to_f32<F>(e & 1 ? bw[e >> 1] >> 16 : bw[e >> 1]));
+            }
+            const uint4 o = make_uint4(pack2<F>(f[0], f[1]), pack2<F>(f[2], f[3]),
+                                       pack2<F>(f[4], f[5]), pack2<F>(f[6], f[7]));
             *reinterpret_cast<uint4*>(box + (((c * 4 + i) ^ (r & 7)) << 4)) = o;
           }
         }
@@ -438,12 +452,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int BS, int QT, bool DQ>
+template <int BS, int QT, bool DQ, int F>
 cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W,
-                     int64_t N, void* Y, int* err, uint64_t wait_limit_ns, int withhold,
-                     cudaStream_t s) {
+                     int64_t N, void* Y, const void* bias, int* err, uint64_t wait_limit_ns,
+                     int withhold, cudaStream_t s) {
   static bool attr_set[64] = {};  // per device
-  auto kern = gemm4_kernel<BS, QT, DQ>;
+  auto kern = gemm4_kernel<BS, QT, DQ, F>;
+  constexpr CUtensorMapDataType kT16 =
+      F == BNB4_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -454,13 +470,13 @@ cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W,
     attr_set[dev] = true;
   }
   CUtensorMap mx, mw, my;
-  if (!make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, BK, BM,
+  if (!make_map_2d(&mx, kT16, X, K, M, K * 2, BK, BM,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   if (!make_map_2d(&mw, CU_TENSOR_MAP_DATA_TYPE_UINT8, W.codes, K / 2, N, K / 2,
                    BK / 2, BNC, CU_TENSOR_MAP_SWIZZLE_NONE))
     return cudaErrorInvalidValue;
-  if (!make_map_2d(&my, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, N * 2, 64, BM,
+  if (!make_map_2d(&my, kT16, Y, N, M, N * 2, 64, BM,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const int n_pair_cols = static_cast<int>((N + BNP - 1) / BNP);
@@ -479,35 +495,44 @@ cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W,
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, mx, mw, my, static_cast<int>(M), static_cast<int>(N),
                             static_cast<int>(K), n_pair_cols, W.absmax, W.absmax_q,
-                            W.scale2, W.offset, err, wait_limit_ns, withhold);
+                            W.scale2, W.offset, static_cast<const uint16_t*>(bias), err,
+                            wait_limit_ns, withhold);
 }
 
-template <int QT, bool DQ>
+template <int QT, bool DQ, int F>
 cudaError_t launch_bs(const void* X, int64_t M, int64_t K, const bnb4_qstate& W,
-                      int64_t N, void* Y, int* err, uint64_t lim, int withhold,
-                      cudaStream_t s) {
+                      int64_t N, void* Y, const void* bias, int* err, uint64_t lim,
+                      int withhold, cudaStream_t s) {
   switch (W.blocksize) {
-    case 32: return launch_t<32, QT, DQ>(X, M, K, W, N, Y, err, lim, withhold, s);
-    case 64: return launch_t<64, QT, DQ>(X, M, K, W, N, Y, err, lim, withhold, s);
-    case 128: return launch_t<128, QT, DQ>(X, M, K, W, N, Y, err, lim, withhold, s);
-    default: return launch_t<256, QT, DQ>(X, M, K, W, N, Y, err, lim, withhold, s);
+    case 32: return launch_t<32, QT, DQ, F>(X, M, K, W, N, Y, bias, err, lim, withhold, s);
+    case 64: return launch_t<64, QT, DQ, F>(X, M, K, W, N, Y, bias, err, lim, withhold, s);
+    case 128: return launch_t<128, QT, DQ, F>(X, M, K, W, N, Y, bias, err, lim, withhold, s);
+    default: return launch_t<256, QT, DQ, F>(X, M, K, W, N, Y, bias, err, lim, withhold, s);
   }
+}
+
+template <int F>
+cudaError_t launch_f(const void* X, int64_t M, int64_t K, const bnb4_qstate& W, int64_t N,
+                     void* Y, const void* bias, int* err, uint64_t lim, int wh,
+                     cudaStream_t s) {
+  if (W.qtype == kQtNF4)
+    return W.double_quant ? launch_bs<kQtNF4, true, F>(X, M, K, W, N, Y, bias, err, lim, wh, s)
+                          : launch_bs<kQtNF4, false, F>(X, M, K, W, N, Y, bias, err, lim, wh, s);
+  return W.double_quant ? launch_bs<kQtFP4, true, F>(X, M, K, W, N, Y, bias, err, lim, wh, s)
+                        : launch_bs<kQtFP4, false, F>(X, M, K, W, N, Y, bias, err, lim, wh, s);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm(const void* X, int64_t M, int64_t K,
-                        const bnb4_qstate& W, int64_t N, void* Y, int* err,
-                        int num_sms, cudaStream_t s, uint64_t wait_limit_ns,
-                        int withhold_first_x) {
+                        const bnb4_qstate& W, int64_t N, void* Y, const void* bias,
+                        int fmt, int* err, int num_sms, cudaStream_t s,
+                        uint64_t wait_limit_ns, int withhold_first_x) {
   (void)num_sms;
   const uint64_t lim = wait_limit_ns ? wait_limit_ns : kWaitLimitNs;
   const int wh = withhold_first_x;
-  if (W.qtype == kQtNF4)
-    return W.double_quant ? launch_bs<kQtNF4, true>(X, M, K, W, N, Y, err, lim, wh, s)
-                          : launch_bs<kQtNF4, false>(X, M, K, W, N, Y, err, lim, wh, s);
-  return W.double_quant ? launch_bs<kQtFP4, true>(X, M, K, W, N, Y, err, lim, wh, s)
-                        : launch_bs<kQtFP4, false>(X, M, K, W, N, Y, err, lim, wh, s);
+  return fmt == BNB4_F16 ? launch_f<BNB4_F16>(X, M, K, W, N, Y, bias, err, lim, wh, s)
+                         : launch_f<BNB4_BF16>(X, M, K, W, N, Y, bias, err, lim, wh, s);
 }
 
 }  // namespace bnb4

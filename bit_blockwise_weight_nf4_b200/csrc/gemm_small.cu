@@ -1,8 +1,10 @@
 // gemm_small.cu -- small-M linear with fused 4-bit weight dequantization on
 // sm_100a (the batch tier between the decode GEMV and the prefill GEMM):
-//   Y[m, n] = bf16( sum_k X[m, k] * What[n, k] ),  1 <= M <= 256,
-//   What[n, k] = bf16(RN(t[code] * a_hat))  (exact dequantized weight),
-// fp32 accumulation in tensor memory by tcgen05.mma (kind::f16, bf16 inputs).
+//   Y[m, n] = h( sum_k X[m, k] * What[n, k] + bias[n] ),  1 <= M <= 256,
+//   What[n, k] = h(RN(t[code] * a_hat))  (exact dequantized weight),
+// h = round to the 16-bit compute format (bf16 or fp16, nearest even), bias
+// optional; fp32 accumulation in tensor memory by tcgen05.mma (kind::f16,
+// bf16 or fp16 inputs).
 //
 // Method: the fused 4-bit dequantize + matmul of bitsandbytes' release notes
 // 0.50.0 (ossradar page) for few tokens, over the NF4 / FP4 blockwise format
@@ -76,11 +78,11 @@ struct Bars {
   int abort;
 };
 
-// Instruction descriptor: kind::f16, D fp32, A and B bf16, both K-major,
-// M = 128 (one CTA), N = nt.
-__host__ __device__ constexpr uint32_t idesc_for(int nt) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(nt >> 3) << 17) |
-         (static_cast<uint32_t>(ROWS >> 4) << 24);
+// Instruction descriptor: kind::f16, D fp32, A and B both bf16 (format code
+// 1) or both fp16 (0), K-major, M = 128 (one CTA), N = nt.
+__host__ __device__ constexpr uint32_t idesc_for(int nt, int fmt) {
+  return (1u << 4) | (fmt == BNB4_F16 ? 0u : (1u << 7) | (1u << 10)) |
+         (static_cast<uint32_t>(nt >> 3) << 17) | (static_cast<uint32_t>(ROWS >> 4) << 24);
 }
 
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
@@ -113,13 +115,14 @@ struct RowStep {
   float g[2];       // scale2 of the block's group (double quant)
 };
 
-template <int BS, int QT, bool DQ>
+template <int BS, int QT, bool DQ, int F>
 __global__ void __launch_bounds__(kThreads, 2)
     gemm_small_kernel(const __grid_constant__ CUtensorMap map_x, int M, int N, int K, int nt,
                       uint32_t idesc, uint32_t tmem_cols, const uint8_t* __restrict__ codes,
                       const float* __restrict__ absmax, const uint8_t* __restrict__ absmax_q,
                       const float* __restrict__ scale2, const float* __restrict__ offset,
-                      uint16_t* __restrict__ Y, int* err, uint64_t wait_limit_ns) {
+                      const uint16_t* __restrict__ bias, uint16_t* __restrict__ Y, int* err,
+                      uint64_t wait_limit_ns) {
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base, derived from the shared array by pointer
   // arithmetic so every access stays a shared-memory access
@@ -260,9 +263,9 @@ __global__ void __launch_bounds__(kThreads, 2)
           a0 = __uint_as_float(b.u[0]);
           a1 = __uint_as_float(b.u[1]);
         }
-        const Lut l0 = make_lut<QT>(a0);
+        const Lut l0 = make_lut<QT, F>(a0);
         Lut l1 = l0;
-        if constexpr (BS == 32) l1 = make_lut<QT>(a1);
+        if constexpr (BS == 32) l1 = make_lut<QT, F>(a1);
         const uint32_t cw[8] = {b.c0.x, b.c0.y, b.c0.z, b.c0.w, b.c1.x, b.c1.y, b.c1.z, b.c1.w};
 #pragma unroll
         for (int p = 0; p < 8; ++p)
@@ -315,11 +318,13 @@ __global__ void __launch_bounds__(kThreads, 2)
             : "r"(tmem + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(c)));
         asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
         if (S == 1) {
+          const float b = bias && nr < N ? half_to_f32<F>(bias[nr]) : 0.0f;
 #pragma unroll
           for (int j = 0; j < 8; ++j)
             if (c + j < M && nr < N)
-              Y[static_cast<int64_t>(c + j) * N + nr] =
-                  static_cast<uint16_t>(pack_bf16x2(__uint_as_float(v[j]), 0.0f));
+              Y[static_cast<int64_t>(c + j) * N + nr] = static_cast<uint16_t>(
+                  pack2<F>(bias ? __fadd_rn(__uint_as_float(v[j]), b) : __uint_as_float(v[j]),
+                           0.0f));
         } else {
 #pragma unroll
           for (int j = 0; j < 8; ++j) red[(c + j) * ROWS + row] = __uint_as_float(v[j]);
@@ -344,6 +349,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int t1 = t0 + per < M ? t0 + per : M;
     const uint32_t red0 = smem_u32(smem);
     if (nr < N) {
+      const float b = bias ? half_to_f32<F>(bias[nr]) : 0.0f;
 #pragma unroll 1
       for (int c = t0 + c0; c < t1; c += 2) {
         const uint32_t off = red0 + static_cast<uint32_t>((c * ROWS + r) * 4);
@@ -355,7 +361,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int s = 1; s < kMaxCluster; ++s)
           if (s < S) sum += part[s];
-        Y[static_cast<int64_t>(c) * N + nr] = static_cast<uint16_t>(pack_bf16x2(sum, 0.0f));
+        if (bias) sum = __fadd_rn(sum, b);
+        Y[static_cast<int64_t>(c) * N + nr] = static_cast<uint16_t>(pack2<F>(sum, 0.0f));
       }
     }
   }
@@ -397,11 +404,12 @@ int choose_split(int64_t tiles, int k_tiles, int num_sms, int per_sm) {
   return best;
 }
 
-template <int BS, int QT, bool DQ>
+template <int BS, int QT, bool DQ, int F>
 cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W, int64_t N,
-                     void* Y, int* err, int num_sms, uint64_t wait_limit_ns, cudaStream_t s) {
+                     void* Y, const void* bias, int* err, int num_sms, uint64_t wait_limit_ns,
+                     cudaStream_t s) {
   static bool attr_set[64] = {};  // per device
-  auto kern = gemm_small_kernel<BS, QT, DQ>;
+  auto kern = gemm_small_kernel<BS, QT, DQ, F>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -416,7 +424,9 @@ cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W, 
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(nt)) cols <<= 1;
   CUtensorMap mx;
-  if (!make_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, K * 2, BK, nt,
+  if (!make_map_2d(&mx, F == BNB4_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                      : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                   X, K, M, K * 2, BK, nt,
                    CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const int64_t tiles = (N + ROWS - 1) / ROWS;
@@ -438,38 +448,48 @@ cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W, 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, mx, static_cast<int>(M), static_cast<int>(N),
-                            static_cast<int>(K), nt, idesc_for(nt), cols,
+                            static_cast<int>(K), nt, idesc_for(nt, F), cols,
                             static_cast<const uint8_t*>(W.codes),
                             static_cast<const float*>(W.absmax),
                             static_cast<const uint8_t*>(W.absmax_q),
                             static_cast<const float*>(W.scale2),
-                            static_cast<const float*>(W.offset), static_cast<uint16_t*>(Y), err,
+                            static_cast<const float*>(W.offset),
+                            static_cast<const uint16_t*>(bias), static_cast<uint16_t*>(Y), err,
                             wait_limit_ns);
 }
 
-template <int QT, bool DQ>
+template <int QT, bool DQ, int F>
 cudaError_t launch_bs(const void* X, int64_t M, int64_t K, const bnb4_qstate& W, int64_t N,
-                      void* Y, int* err, int sms, uint64_t lim, cudaStream_t s) {
+                      void* Y, const void* bias, int* err, int sms, uint64_t lim,
+                      cudaStream_t s) {
   switch (W.blocksize) {
-    case 32: return launch_t<32, QT, DQ>(X, M, K, W, N, Y, err, sms, lim, s);
-    case 64: return launch_t<64, QT, DQ>(X, M, K, W, N, Y, err, sms, lim, s);
-    case 128: return launch_t<128, QT, DQ>(X, M, K, W, N, Y, err, sms, lim, s);
-    default: return launch_t<256, QT, DQ>(X, M, K, W, N, Y, err, sms, lim, s);
+    case 32: return launch_t<32, QT, DQ, F>(X, M, K, W, N, Y, bias, err, sms, lim, s);
+    case 64: return launch_t<64, QT, DQ, F>(X, M, K, W, N, Y, bias, err, sms, lim, s);
+    case 128: return launch_t<128, QT, DQ, F>(X, M, K, W, N, Y, bias, err, sms, lim, s);
+    default: return launch_t<256, QT, DQ, F>(X, M, K, W, N, Y, bias, err, sms, lim, s);
   }
+}
+
+template <int F>
+cudaError_t launch_f(const void* X, int64_t M, int64_t K, const bnb4_qstate& W, int64_t N,
+                     void* Y, const void* bias, int* err, int sms, uint64_t lim,
+                     cudaStream_t s) {
+  if (W.qtype == kQtNF4)
+    return W.double_quant ? launch_bs<kQtNF4, true, F>(X, M, K, W, N, Y, bias, err, sms, lim, s)
+                          : launch_bs<kQtNF4, false, F>(X, M, K, W, N, Y, bias, err, sms, lim, s);
+  return W.double_quant ? launch_bs<kQtFP4, true, F>(X, M, K, W, N, Y, bias, err, sms, lim, s)
+                        : launch_bs<kQtFP4, false, F>(X, M, K, W, N, Y, bias, err, sms, lim, s);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm_small(const void* X, int64_t M, int64_t K, const bnb4_qstate& W,
-                              int64_t N, void* Y, int* err, int num_sms, cudaStream_t s,
-                              uint64_t wait_limit_ns) {
+                              int64_t N, void* Y, const void* bias, int fmt, int* err,
+                              int num_sms, cudaStream_t s, uint64_t wait_limit_ns) {
   if (M < 1 || M > kMaxNT) return cudaErrorInvalidValue;
   const uint64_t lim = wait_limit_ns ? wait_limit_ns : kWaitLimitNs;
-  if (W.qtype == kQtNF4)
-    return W.double_quant ? launch_bs<kQtNF4, true>(X, M, K, W, N, Y, err, num_sms, lim, s)
-                          : launch_bs<kQtNF4, false>(X, M, K, W, N, Y, err, num_sms, lim, s);
-  return W.double_quant ? launch_bs<kQtFP4, true>(X, M, K, W, N, Y, err, num_sms, lim, s)
-                        : launch_bs<kQtFP4, false>(X, M, K, W, N, Y, err, num_sms, lim, s);
+  return fmt == BNB4_F16 ? launch_f<BNB4_F16>(X, M, K, W, N, Y, bias, err, num_sms, lim, s)
+                         : launch_f<BNB4_BF16>(X, M, K, W, N, Y, bias, err, num_sms, lim, s);
 }
 
 }  // namespace bnb4

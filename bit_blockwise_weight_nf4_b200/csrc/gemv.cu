@@ -1,6 +1,8 @@
 // gemv.cu -- decode GEMV with 4-bit weights on sm_100a:
-//   y[b, n] = bf16( sum_k x[b, k] * What[n, k] ),  1 <= B <= 8,
-//   What[n, k] = bf16(RN(t[code] * a_hat))   (dequantized weight, exact).
+//   y[b, n] = h( sum_k x[b, k] * What[n, k] + bias[n] ),  1 <= B <= 8,
+//   What[n, k] = h(RN(t[code] * a_hat))   (dequantized weight, exact),
+// h = round to the 16-bit compute format, bf16 or fp16 (nearest even); the
+// bias is optional.
 //
 // Method: bitsandbytes' gemv_4bit op (ossradar page, release notes 0.50.0)
 // over the blockwise NF4 / FP4 format of the CSDN article (section
@@ -49,7 +51,7 @@ struct Lut {
   uint32_t L[4], H[4];
 };
 
-template <int QT>
+template <int QT, int F>
 __device__ __forceinline__ Lut make_lut(float ah) {
   uint32_t P[8];
 #pragma unroll
@@ -60,7 +62,7 @@ __device__ __forceinline__ Lut make_lut(float ah) {
     const float t1 = QT == kQtNF4 ? nf4_value(2 * j + 1)
                                   : ((2 * j + 1) & 8 ? -fp4_magnitude((2 * j + 1) & 7)
                                                      : fp4_magnitude((2 * j + 1) & 7));
-    P[j] = pack_bf16x2(__fmul_rn(t0, ah), __fmul_rn(t1, ah));
+    P[j] = pack2<F>(__fmul_rn(t0, ah), __fmul_rn(t1, ah));
   }
   Lut l;
 #pragma unroll
@@ -93,15 +95,21 @@ __device__ __forceinline__ void dq8(const Lut& l, uint32_t w, uint32_t (&o)[4]) 
   dq4(l, sel >> 16, mix >> 16, o[2], o[3]);
 }
 
-// D[16 x 8] += A[16 x 16] (weight rows) * B[16 x 8] (x columns), bf16 in,
-// fp32 accumulate.
-__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1,
-                                         uint32_t a2, uint32_t a3, uint32_t b0,
-                                         uint32_t b1) {
-  asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+// D[16 x 8] += A[16 x 16] (weight rows) * B[16 x 8] (x columns), bf16 or
+// fp16 in (format F), fp32 accumulate.
+template <int F>
+__device__ __forceinline__ void mma16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                      uint32_t a3, uint32_t b0, uint32_t b1) {
+  if constexpr (F == BNB4_F16)
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  else
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 // Raw scale inputs of one quant block, loaded ahead and decoded when used
@@ -141,7 +149,7 @@ struct StepBuf {
   RawScale a[2][2];    // [row][block within the segment (blocksize 32)]
 };
 
-template <int BS, int QT, bool DQ, int kDepth>
+template <int BS, int QT, bool DQ, int kDepth, int F>
 __global__ void __launch_bounds__(kThreads, 2)
     gemv4_kernel(const uint16_t* __restrict__ x, int B, int64_t K,
                  const uint8_t* __restrict__ codes,
@@ -149,7 +157,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                  const uint8_t* __restrict__ absmax_q,
                  const float* __restrict__ scale2,
                  const float* __restrict__ offset, int64_t N,
-                 uint16_t* __restrict__ y) {
+                 const uint16_t* __restrict__ bias, uint16_t* __restrict__ y) {
   __shared__ float red[kWarps][32][4];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -204,9 +212,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         Lut lut[2][2];
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
-          lut[r][0] = make_lut<QT>(ok[r] && seg ? decode<DQ>(buf[d].a[r][0], off) : 0.0f);
+          lut[r][0] = make_lut<QT, F>(ok[r] && seg ? decode<DQ>(buf[d].a[r][0], off) : 0.0f);
           lut[r][1] = BS == 32
-                          ? make_lut<QT>(ok[r] && seg ? decode<DQ>(buf[d].a[r][1], off) : 0.0f)
+                          ? make_lut<QT, F>(ok[r] && seg ? decode<DQ>(buf[d].a[r][1], off) : 0.0f)
                           : lut[r][0];
         }
         const int64_t kx = seg ? k0 : 0;  // x stays in bounds on a ragged edge
@@ -221,8 +229,8 @@ __global__ void __launch_bounds__(kThreads, 2)
           uint32_t o0[4], o1[4];
           dq8(lut[0][BS == 32 ? h : 0], w0, o0);
           dq8(lut[1][BS == 32 ? h : 0], w1, o1);
-          mma_bf16(acc[(2 * p) % kChains], o0[0], o1[0], o0[1], o1[1], xb.x, xb.y);
-          mma_bf16(acc[(2 * p + 1) % kChains], o0[2], o1[2], o0[3], o1[3], xb.z, xb.w);
+          mma16<F>(acc[(2 * p) % kChains], o0[0], o1[0], o0[1], o1[1], xb.x, xb.y);
+          mma16<F>(acc[(2 * p + 1) % kChains], o0[2], o1[2], o0[3], o1[3], xb.z, xb.w);
         }
         if (i + kDepth < my_steps) issue(i + kDepth, buf[d]);
       }
@@ -253,7 +261,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int cb = 0; cb < 2; ++cb) {
         const int bcol = 2 * t + cb;
         if (ok[r] && bcol < B) {
-          const uint32_t o = pack_bf16x2(s[2 * r + cb], 0.0f);
+          float v = s[2 * r + cb];
+          if (bias) v = __fadd_rn(v, half_to_f32<F>(bias[n[r]]));
+          const uint32_t o = pack2<F>(v, 0.0f);
           y[static_cast<int64_t>(bcol) * N + n[r]] = static_cast<uint16_t>(o);
         }
       }
@@ -261,45 +271,53 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-template <int BS, int QT, bool DQ, int kDepth>
+template <int BS, int QT, bool DQ, int kDepth, int F>
 cudaError_t launch_t(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
-                     int64_t N, void* y, cudaStream_t s) {
+                     int64_t N, const void* bias, void* y, cudaStream_t s) {
   const int64_t grid = (N + kRowsPerCta - 1) / kRowsPerCta;
-  return launch_kernel(gemv4_kernel<BS, QT, DQ, kDepth>, dim3(static_cast<unsigned>(grid)),
+  return launch_kernel(gemv4_kernel<BS, QT, DQ, kDepth, F>, dim3(static_cast<unsigned>(grid)),
              dim3(kThreads), 0, s, false, static_cast<const uint16_t*>(x), static_cast<int>(B), K,
              static_cast<const uint8_t*>(W.codes), static_cast<const float*>(W.absmax),
              static_cast<const uint8_t*>(W.absmax_q), static_cast<const float*>(W.scale2),
-             static_cast<const float*>(W.offset), N, static_cast<uint16_t*>(y));
+             static_cast<const float*>(W.offset), N, static_cast<const uint16_t*>(bias),
+             static_cast<uint16_t*>(y));
 }
 
-template <int BS, int QT>
+template <int BS, int QT, int F>
 cudaError_t launch_bs(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
-                      int64_t N, void* y, cudaStream_t s) {
+                      int64_t N, const void* bias, void* y, cudaStream_t s) {
   // two K steps of loads in flight per lane (for K <= 4096 that is all of a
   // warp's share), 2 CTAs of 8 warps resident per SM
-  if (W.double_quant) return launch_t<BS, QT, true, 2>(x, B, K, W, N, y, s);
-  return launch_t<BS, QT, false, 2>(x, B, K, W, N, y, s);
+  if (W.double_quant) return launch_t<BS, QT, true, 2, F>(x, B, K, W, N, bias, y, s);
+  return launch_t<BS, QT, false, 2, F>(x, B, K, W, N, bias, y, s);
 }
 
-template <int QT>
+template <int QT, int F>
 cudaError_t launch_q(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
-                     int64_t N, void* y, cudaStream_t s) {
+                     int64_t N, const void* bias, void* y, cudaStream_t s) {
   switch (W.blocksize) {
-    case 32: return launch_bs<32, QT>(x, B, K, W, N, y, s);
-    case 64: return launch_bs<64, QT>(x, B, K, W, N, y, s);
-    case 128: return launch_bs<128, QT>(x, B, K, W, N, y, s);
-    default: return launch_bs<256, QT>(x, B, K, W, N, y, s);
+    case 32: return launch_bs<32, QT, F>(x, B, K, W, N, bias, y, s);
+    case 64: return launch_bs<64, QT, F>(x, B, K, W, N, bias, y, s);
+    case 128: return launch_bs<128, QT, F>(x, B, K, W, N, bias, y, s);
+    default: return launch_bs<256, QT, F>(x, B, K, W, N, bias, y, s);
   }
+}
+
+template <int F>
+cudaError_t launch_f(const void* x, int64_t B, int64_t K, const bnb4_qstate& W, int64_t N,
+                     const void* bias, void* y, cudaStream_t s) {
+  return W.qtype == kQtNF4 ? launch_q<kQtNF4, F>(x, B, K, W, N, bias, y, s)
+                           : launch_q<kQtFP4, F>(x, B, K, W, N, bias, y, s);
 }
 
 }  // namespace
 
-cudaError_t launch_gemv(const void* x, int64_t B, int64_t K,
-                        const bnb4_qstate& W, int64_t N, void* y, int num_sms,
+cudaError_t launch_gemv(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
+                        int64_t N, void* y, const void* bias, int fmt, int num_sms,
                         cudaStream_t s) {
   (void)num_sms;
-  return W.qtype == kQtNF4 ? launch_q<kQtNF4>(x, B, K, W, N, y, s)
-                           : launch_q<kQtFP4>(x, B, K, W, N, y, s);
+  return fmt == BNB4_F16 ? launch_f<BNB4_F16>(x, B, K, W, N, bias, y, s)
+                         : launch_f<BNB4_BF16>(x, B, K, W, N, bias, y, s);
 }
 
 }  // namespace bnb4

@@ -25,22 +25,25 @@ cudaError_t launch_dequantize(const bnb4_qstate& st, void* out, int out_dtype,
 // over its whole input range; result = {u64 mismatches, u32 first, u32 0}.
 cudaError_t launch_check_rcp(void* result, cudaStream_t s);
 
+// The linear kernels take the 16-bit compute format `fmt` (BNB4_BF16 or
+// BNB4_F16) of x, y and bias; bias (N elements) may be null.
 cudaError_t launch_gemv(const void* x, int64_t B, int64_t K,
-                        const bnb4_qstate& W, int64_t N, void* y, int num_sms,
-                        cudaStream_t s);
+                        const bnb4_qstate& W, int64_t N, void* y, const void* bias,
+                        int fmt, int num_sms, cudaStream_t s);
 
 // wait_limit_ns = 0 selects the normal bound of every mbarrier wait (2 s);
 // withhold_first_x != 0 is the failure-detection diagnostic (the first X
 // stage is never loaded, so the kernel's waits run out).
 cudaError_t launch_gemm(const void* X, int64_t M, int64_t K,
-                        const bnb4_qstate& W, int64_t N, void* Y, int* err,
-                        int num_sms, cudaStream_t s, uint64_t wait_limit_ns = 0,
-                        int withhold_first_x = 0);
+                        const bnb4_qstate& W, int64_t N, void* Y, const void* bias,
+                        int fmt, int* err, int num_sms, cudaStream_t s,
+                        uint64_t wait_limit_ns = 0, int withhold_first_x = 0);
 
 // Linear layer for 1..256 tokens (the small-batch tier): weight rows on the
 // MMA's M side, tokens on its N side, K split over a cluster.
 cudaError_t launch_gemm_small(const void* X, int64_t M, int64_t K,
-                              const bnb4_qstate& W, int64_t N, void* Y, int* err,
-                              int num_sms, cudaStream_t s, uint64_t wait_limit_ns = 0);
+                              const bnb4_qstate& W, int64_t N, void* Y, const void* bias,
+                              int fmt, int* err, int num_sms, cudaStream_t s,
+                              uint64_t wait_limit_ns = 0);
 
 }  // namespace bnb4

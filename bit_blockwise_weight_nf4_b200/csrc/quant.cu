@@ -221,6 +221,23 @@ struct Elem<uint16_t> {  // bf16 bit patterns
   }
 };
 
+// fp16 input: IEEE binary16 patterns, decoded exactly to fp32.
+struct Half16 {
+  uint16_t bits;
+};
+template <>
+struct Elem<Half16> {
+  static constexpr int kPerChunk = 8;
+  __device__ static float get(const uint4& c, int i) {
+    const uint32_t w = (i >> 1) == 0 ? c.x : (i >> 1) == 1 ? c.y
+                       : (i >> 1) == 2 ? c.z : c.w;
+    return half_to_f32<BNB4_F16>((i & 1) ? w >> 16 : w);
+  }
+  __device__ static uint4 load_partial(const Half16* x, int64_t e, int64_t n) {
+    return Elem<uint16_t>::load_partial(reinterpret_cast<const uint16_t*>(x), e, n);
+  }
+};
+
 // Block absmax of a row group: the lane's chunk(s), then an xor-shuffle
 // reduction over the lanes holding the block (for LPB = 64 the two rows of
 // the group hold one block across the whole warp).
@@ -546,6 +563,9 @@ cudaError_t launch_quantize(const void* x, int x_dtype, const bnb4_qstate& st,
       x_dtype == BNB4_F32
           ? dispatch_q<float>(st.qtype, dq, st.blocksize, x, st.n, st.codes,
                               st.absmax, partials, grid, s)
+      : x_dtype == BNB4_F16
+          ? dispatch_q<Half16>(st.qtype, dq, st.blocksize, x, st.n, st.codes,
+                               st.absmax, partials, grid, s)
           : dispatch_q<uint16_t>(st.qtype, dq, st.blocksize, x, st.n, st.codes,
                                  st.absmax, partials, grid, s);
   if (e != cudaSuccess || !dq) return e;

@@ -74,7 +74,8 @@ extern "C" BNB4_API int bnb_quantize_4bit_noalloc(const void* x, int32_t x_dtype
                                                   const bnb4_qstate* st,
                                                   void* stream) {
   if (!x || !st) return BNB4_ERR_INVALID_ARG;
-  if (x_dtype != BNB4_F32 && x_dtype != BNB4_BF16) return BNB4_ERR_UNSUPPORTED;
+  if (x_dtype != BNB4_F32 && x_dtype != BNB4_BF16 && x_dtype != BNB4_F16)
+    return BNB4_ERR_UNSUPPORTED;
   if (!st->codes || st->n <= 0 || st->reserved != 0) return BNB4_ERR_INVALID_ARG;
   if (st->qtype != BNB4_NF4 && st->qtype != BNB4_FP4) return BNB4_ERR_INVALID_ARG;
   if (st->double_quant != 1) return BNB4_ERR_INVALID_ARG;

@@ -174,7 +174,10 @@ struct Lut {
   uint32_t L[4], H[4];
 };
 
-template <int QT>
+// Per-block table of the 16 dequantized values in the 16-bit compute format F
+// (BNB4_BF16 or BNB4_F16), split by byte: L[q] holds the low bytes of
+// entries 4q..4q+3, H[q] the high bytes.
+template <int QT, int F>
 __device__ __forceinline__ Lut make_lut(float ah) {
   uint32_t P[8];
 #pragma unroll
@@ -184,7 +187,7 @@ __device__ __forceinline__ Lut make_lut(float ah) {
                                   : ((c0 & 8) ? -fp4_magnitude(c0 & 7) : fp4_magnitude(c0 & 7));
     const float t1 = QT == kQtNF4 ? nf4_value(c1)
                                   : ((c1 & 8) ? -fp4_magnitude(c1 & 7) : fp4_magnitude(c1 & 7));
-    P[j] = pack_bf16x2(__fmul_rn(t0, ah), __fmul_rn(t1, ah));
+    P[j] = pack2<F>(__fmul_rn(t0, ah), __fmul_rn(t1, ah));
   }
   Lut l;
 #pragma unroll

@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define BNB4_ABI_VERSION 1
+#define BNB4_ABI_VERSION 2
 
 /* Every entry point is exported from the shared library (the library is
  * built with hidden visibility by default). */
@@ -72,6 +72,7 @@ extern "C" {
 #define BNB4_FP4 1  /* E2M1 magnitudes / 6, sign-magnitude codes */
 #define BNB4_F32 0  /* fp32 element type */
 #define BNB4_BF16 1 /* bf16 element type (raw 16-bit patterns) */
+#define BNB4_F16 2  /* IEEE fp16 element type (raw 16-bit patterns) */
 
 /*
  * Quantization state of n elements: the packed codes plus the block scales.
@@ -124,7 +125,8 @@ BNB4_API int bnb4_query_sizes(int64_t n, int32_t blocksize, int32_t double_quant
  * scale per block, nearest codebook entry, 16 codes packed two per byte;
  * section "实际性能差异": double quantization of the scales to 8 bits).
  *
- *  x           device, st->n elements of x_dtype (BNB4_F32 or BNB4_BF16),
+ *  x           device, st->n elements of x_dtype (BNB4_F32, BNB4_BF16 or
+ *              BNB4_F16; 16-bit inputs are widened to fp32 exactly),
  *              16-byte aligned.
  *  st          state whose buffers receive the result: codes and absmax
  *              always; absmax_q, scale2 and offset when st->double_quant.
@@ -180,7 +182,8 @@ BNB4_API int bnb_quantize_4bit_noalloc(const void* x, int32_t x_dtype,
 /*
  * Dequantization (NF4 article, section "实际性能差异": the 4-bit codes times
  * the decoded block scale).  w = RN(t[code] * a_hat) in fp32; with out_dtype
- * BNB4_BF16 the output is round-to-nearest-even of w.  out: device, st->n
+ * BNB4_BF16 or BNB4_F16 the output is the round-to-nearest-even of w in that
+ * format (fp16: infinity past 65504, subnormals kept).  out: device, st->n
  * elements, 16-byte aligned.  Bit-exact to the reference definition.
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CUDA.
  */
@@ -218,6 +221,31 @@ BNB4_API int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstat
  */
 BNB4_API int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstate* W,
                   int64_t N, void* Y, void* stream);
+
+/*
+ * The fused 4-bit linear layer in either 16-bit compute type, with an
+ * optional bias (release notes 0.50.0: fused 4-bit GEMM with the nested
+ * quantization and the bias folded in, bf16 or fp16 activations; NF4
+ * article, configuration section: the compute dtype is a setting):
+ *   y[m, n] = h( sum_k x[m, k] * What[n, k] + bias[n] ),  m < M, n < N,
+ * What[n, k] = h(RN(t[code] * a_hat)), h = round to nearest even in the
+ * compute type `dtype` (BNB4_BF16 or BNB4_F16); products exact, fp32
+ * accumulation, the bias added in fp32, one final rounding.
+ *  x     device [M, K] of dtype, 16-byte aligned.
+ *  bias  device [N] of dtype, 16-byte aligned, or NULL for none.
+ *  y     device [M, N] of dtype; 2-byte aligned for M <= 256, 16-byte aligned
+ *        above.
+ *  W     quantization state of the weight [N, K] (W->n == N*K).
+ * Constraints: M >= 1; K % 64 == 0; K % W->blocksize == 0; N % 8 == 0 when
+ * M > 256.  The kernel follows M as in bnb_gemm_4bit (the decode kernel up to
+ * 8 rows, the small-batch kernel up to 256, the prefill kernel above); with
+ * dtype BNB4_BF16 and no bias the result equals that of bnb_gemm_4bit /
+ * bnb_gemv_4bit bit for bit.
+ * Errors: INVALID_ARG, UNSUPPORTED (dtype), ALIGNMENT, SHAPE, CUDA.
+ */
+BNB4_API int bnb_linear_4bit(const void* x, int32_t dtype, int64_t M, int64_t K,
+                             const bnb4_qstate* W, int64_t N, const void* bias, void* y,
+                             void* stream);
 
 /*
  * Synchronizes `stream`, then reads the library's device error word of the

@@ -12,7 +12,11 @@ Tolerance for y = bf16(fp32 sum of x * What) against the fp64 oracle y64:
     tensor cores' accumulation), and the final bf16 rounding by 2^-8 of the
     value: |y - y64| <= 2^-8 (|y64| + gamma S) + gamma S;
   * with at least 1024 outputs, 98% of them equal bf16(y64) exactly (a wrong
-    What, or unrounded weights, would not)."""
+    What, or unrounded weights, would not); 90% for fp16, whose output ulp is
+    8x finer, so that the fp32 tensor-core accumulation over K = 11008 flips
+    a few percent of the roundings (95.8% measured on the prefill kernel),
+    while a wrong fp16 What still fails by far (bf16-rounded weights match
+    ~14%, unrounded fp32 weights ~58%, on 32 x 256 outputs at K = 4096)."""
 import numpy as np
 import torch
 
@@ -20,6 +24,7 @@ import bit_blockwise_weight_nf4_b200 as bnb4
 import oracle
 
 REL_FROB_TOL = 2e-3
+MATCH_MIN = {oracle.BF16: 0.98, oracle.F16: 0.90}
 MAX_ABS_FACTOR = 1e-2
 CANARY = 0xA5
 GUARD = 64  # bytes of canary after every output buffer
@@ -92,32 +97,38 @@ def assert_state_equal(gpu, orc, dq):
 FROB_MIN_ELEMENTS = 1024
 
 
-def check_linear(y_gpu_bits, y64, x_bits, What_bits, rows=None):
-    """Tolerance for y = x What^T (rows of x optionally subsampled; y64 is
-    the fp64 oracle for those rows).  See the module docstring."""
-    y = bits_to_f64(y_gpu_bits).reshape(y64.shape)
+def check_linear(y_gpu_bits, y64, x_bits, What_bits, rows=None, dtype=oracle.BF16):
+    """Tolerance for y = x What^T (+ bias; rows of x optionally subsampled;
+    y64 is the fp64 oracle for those rows) in the compute type ``dtype``
+    (bf16 or fp16 bit patterns).  See the module docstring; for fp16 the
+    final rounding costs 2^-11 instead of 2^-8."""
+    to64 = oracle.f16_bits_to_f64 if dtype == oracle.F16 else bits_to_f64
+    unit = 2.0 ** -11 if dtype == oracle.F16 else 2.0 ** -8
+    y = to64(y_gpu_bits).reshape(y64.shape)
     err = y - y64
     rel = np.linalg.norm(err) / max(np.linalg.norm(y64), 1e-300)
     if y64.size >= FROB_MIN_ELEMENTS:
         assert rel <= REL_FROB_TOL, "relative Frobenius error %.3g" % rel
-    x = bits_to_f64(x_bits)
+    x = to64(x_bits)
     if rows is not None:
         x = x[rows]
-    W = bits_to_f64(What_bits)
+    W = to64(What_bits)
     wmax = np.abs(W).max()
     bound = MAX_ABS_FACTOR * np.linalg.norm(x, axis=1) * wmax
     assert np.all(np.abs(err).max(axis=1) <= bound + 1e-30), "max abs error"
     K = x.shape[1]
     gamma = K * 2.0 ** -22
     S = np.abs(x) @ np.abs(W).T
-    elem = 2.0 ** -8 * (np.abs(y64) + gamma * S) + gamma * S
+    elem = unit * (np.abs(y64) + gamma * S) + gamma * S
     bad = np.abs(err) > elem
     assert not bad.any(), "elementwise bound violated at %d outputs" % bad.sum()
-    # the rounding of the exact fp64 result to bf16 is the dominant error:
-    # almost every output must equal it (a wrong What would not)
-    ref16 = torch.from_numpy(y64).to(torch.bfloat16).view(torch.int16).numpy() \
+    # the rounding of the exact fp64 result to the compute type is the
+    # dominant error: almost every output must equal it (a wrong What would not)
+    t16 = torch.float16 if dtype == oracle.F16 else torch.bfloat16
+    ref16 = torch.from_numpy(y64).to(t16).view(torch.int16).numpy() \
         .view(np.uint16).reshape(-1)
     match = np.mean(ref16 == np.asarray(y_gpu_bits).reshape(-1))
     if y64.size >= FROB_MIN_ELEMENTS:
-        assert match >= 0.98, "only %.4f of outputs equal bf16(fp64 reference)" % match
+        assert match >= MATCH_MIN[dtype], \
+            "only %.4f of outputs equal the rounded fp64 reference" % match
     return rel, match

@@ -141,6 +141,24 @@ def test_gemm_argument_errors(lib):
     assert call(Y=A16 + 8) == bnb4.ERR_ALIGNMENT
 
 
+def test_linear_argument_errors(lib):
+    W = good_state(n=64 * 64)
+
+    def call(x=A16, dtype=bnb4.F16, M=4, K=64, N=64, bias=None, y=A16, W=W):
+        return bnb4.bnb_linear_4bit(x, dtype, M, K, W, N, bias, y, None)
+    assert call(x=None) == bnb4.ERR_INVALID_ARG
+    assert call(y=None) == bnb4.ERR_INVALID_ARG
+    assert call(dtype=bnb4.F32) == bnb4.ERR_UNSUPPORTED
+    assert call(dtype=7) == bnb4.ERR_UNSUPPORTED
+    assert call(M=0) == bnb4.ERR_SHAPE
+    assert call(K=96, W=good_state(n=64 * 96)) == bnb4.ERR_SHAPE          # K % 64
+    assert call(M=300, N=60, W=good_state(n=60 * 64)) == bnb4.ERR_SHAPE   # N % 8 above 256
+    assert call(x=A16 + 2) == bnb4.ERR_ALIGNMENT
+    assert call(bias=A16 + 2) == bnb4.ERR_ALIGNMENT
+    assert call(y=A16 + 1) == bnb4.ERR_ALIGNMENT
+    assert call(M=300, y=A16 + 2) == bnb4.ERR_ALIGNMENT                   # 16 B above 256
+
+
 def test_no_cpu_fallback_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(bnb4, "_lib", None)
     monkeypatch.setattr(bnb4, "LIB_PATH", str(tmp_path / "missing.so"))

@@ -1,5 +1,5 @@
 """GPU parity of bnb_dequantize_4bit against the CPU oracle, bit for bit, in
-fp32 and bf16, on a state the oracle computed (uploaded), and end to end
+fp32, bf16 and fp16, on a state the oracle computed (uploaded), and end to end
 (GPU quantize then GPU dequantize vs oracle quantize then oracle
 dequantize)."""
 import numpy as np
@@ -25,7 +25,7 @@ def gpu_dequant(state, n, out_dtype):
     return host[:n * elt].view(np.float32 if out_dtype == bnb4.F32 else np.uint16)
 
 
-@pytest.mark.parametrize("out_dtype", [bnb4.F32, bnb4.BF16])
+@pytest.mark.parametrize("out_dtype", [bnb4.F32, bnb4.BF16, bnb4.F16])
 @pytest.mark.parametrize("qtype", [bnb4.NF4, bnb4.FP4])
 @pytest.mark.parametrize("bs", [32, 64, 128, 256])
 @pytest.mark.parametrize("dq", [True, False])
@@ -57,4 +57,17 @@ def test_matrix_4096_end_to_end_bf16(qtype):
     want = oracle.dequantize(orc, oracle.BF16)
     st = bnb4.quantize_4bit(W.cuda().view(-1), 64, qtype, True)
     got = cpu_bits(bnb4.dequantize_4bit(st, torch.bfloat16))
+    assert got.tobytes() == want.tobytes()
+
+
+@pytest.mark.parametrize("qtype", [bnb4.NF4, bnb4.FP4])
+def test_matrix_4096_end_to_end_f16(qtype):
+    """The fp16 compute type: an fp16 weight quantized and dequantized to fp16
+    on the GPU equals the oracle doing the same, bit for bit."""
+    W = synth.weight_bf16(4096, 4096, seed=1001, outlier_frac=synth.OUTLIER_FRAC)
+    W = W.to(torch.float16)
+    orc = oracle.quantize(W.view(-1).numpy(), 64, qtype, True)
+    want = oracle.dequantize(orc, oracle.F16)
+    st = bnb4.quantize_4bit(W.cuda().view(-1), 64, qtype, True)
+    got = cpu_bits(bnb4.dequantize_4bit(st, torch.float16))
     assert got.tobytes() == want.tobytes()

@@ -14,9 +14,12 @@ pytestmark = pytest.mark.gpu
 
 
 def run_both(x_cpu, bs, qtype, dq):
-    """x_cpu: fp32 or bf16 CPU tensor. Returns (gpu arrays, oracle state)."""
+    """x_cpu: fp32, bf16 or fp16 CPU tensor. Returns (gpu arrays, oracle
+    state)."""
     if x_cpu.dtype == torch.float32:
         host, dt = x_cpu.contiguous().view(-1).numpy(), bnb4.F32
+    elif x_cpu.dtype == torch.float16:
+        host, dt = x_cpu.contiguous().view(-1).numpy(), bnb4.F16
     else:
         host, dt = synth.bf16_bits(x_cpu.view(-1)), bnb4.BF16
     orc = oracle.quantize(host, bs, qtype, dq)
@@ -25,7 +28,7 @@ def run_both(x_cpu, bs, qtype, dq):
     return g.arrays(), orc
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("qtype", [bnb4.NF4, bnb4.FP4])
 @pytest.mark.parametrize("bs", [32, 64, 128, 256])
 @pytest.mark.parametrize("dq", [True, False])
@@ -34,6 +37,8 @@ def test_quantize_small_ragged(dtype, qtype, bs, dq, n):
     x = synth.normal_f32((n,), seed=n + bs, std=0.02)
     if dtype == "bf16":
         x = x.to(torch.bfloat16)
+    elif dtype == "f16":
+        x = x.to(torch.float16)
     gpu, orc = run_both(x, bs, qtype, dq)
     assert_state_equal(gpu, orc, dq)
 
@@ -48,10 +53,13 @@ def test_roundtrip_vector_1m():
 
 
 @pytest.mark.parametrize("qtype", [bnb4.NF4, bnb4.FP4])
-def test_matrix_4096_with_outliers(qtype):
-    """bf16 4096 x 4096 ~ N(0, 0.02^2), 0.1% of positions x20, blocksize 64,
-    double quant."""
+@pytest.mark.parametrize("f16", [False, True])
+def test_matrix_4096_with_outliers(qtype, f16):
+    """bf16 (or, for the fp16 compute type, the same values in fp16) 4096 x
+    4096 ~ N(0, 0.02^2), 0.1% of positions x20, blocksize 64, double quant."""
     W = synth.weight_bf16(4096, 4096, seed=1000, outlier_frac=synth.OUTLIER_FRAC)
+    if f16:
+        W = W.to(torch.float16)
     gpu, orc = run_both(W, 64, qtype, True)
     assert orc["sum_exact"]
     assert_state_equal(gpu, orc, True)
@@ -130,7 +138,7 @@ def _special_blocks(bs, n_blocks, rng):
     return x
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("qtype", [bnb4.NF4, bnb4.FP4])
 @pytest.mark.parametrize("bs", [32, 64, 256])
 def test_special_values_in_full_tiles(dtype, qtype, bs):
@@ -138,13 +146,15 @@ def test_special_values_in_full_tiles(dtype, qtype, bs):
     elements, placed inside full tiles (so the streaming loop's warp-uniform
     choice between the fast and the exact path is exercised) and in the
     ragged tail: codes and absmax equal the oracle's bit for bit."""
-    rng = np.random.default_rng(bs + (7 if dtype == "bf16" else 0) + 3 * qtype)
+    rng = np.random.default_rng(bs + {"f32": 0, "bf16": 7, "f16": 11}[dtype] + 3 * qtype)
     n = 16384 * 3 + 77 * bs // 32 + 5
     nb = -(-n // bs)
     x = _special_blocks(bs, nb, rng)[:n]
     xt = torch.from_numpy(x)
     if dtype == "bf16":
         xt = xt.to(torch.bfloat16)
+    elif dtype == "f16":  # the fp16 range turns the classes into 0, subnormal, inf
+        xt = xt.to(torch.float16)
     gpu, orc = run_both(xt, bs, qtype, False)
     assert_state_equal(gpu, orc, False)
 
