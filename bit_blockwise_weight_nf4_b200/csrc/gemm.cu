@@ -15,14 +15,14 @@
 // halves -- each CTA dequantizes only its 128 weight rows, so the
 // dequantization work per flop is a quarter of a one-CTA 128 x 256 MMA.
 // Per CTA, 19 warps and three smem rings:
-//  * ring A (3 stages): the CTA's two 128 x 64 bf16 tiles of X per 64-wide K
+//  * ring A (3 stages): the CTA's two 128 x 64 16-bit tiles of X per 64-wide K
 //    step, TMA (128-byte swizzle) completing on the leader CTA's barrier;
 //    warp 0 produces it (the leader also arms the barrier with the bytes of
 //    both CTAs).
-//  * ring W (8 stages): the CTA's 128 x 32-byte packed weight tile (TMA) plus
+//  * ring W (4 stages, one per dequant group): the CTA's 128 x 32-byte packed weight tile (TMA) plus
 //    its 128 decoded block scales (nested quantization decoded by the 32
 //    lanes of warp 2, whose scale loads run two steps ahead).
-//  * ring B (4 stages): the CTA's dequantized 128 x 64 bf16 weight half,
+//  * ring B (6 stages): the CTA's dequantized 128 x 64 16-bit weight half,
 //    written by warps 3..18 in four groups of 4 warps (group g takes the K
 //    steps kt = g mod 4 and owns B slot g; thread r of a group owns weight
 //    row r) in the 128-byte-swizzled K-major layout, then fence.proxy.async
@@ -32,7 +32,7 @@
 //    tcgen05.mma.cta_group::2 (M 256, N 256, K 16), then commits to the
 //    "empty" barriers of both CTAs (multicast commit).
 //  * epilogue: warps 3..18 of each CTA read its accumulator rows with
-//    tcgen05.ld, round to bf16 and store.
+//    tcgen05.ld, add the bias, round to the compute format and store.
 //  * Every mbarrier wait is bounded in time; on expiry the CTA sets the
 //    library's device error word, drains what it started and exits.
 //  No TMA load uses cluster multicast.
@@ -50,7 +50,7 @@ constexpr int BM = 128;      // rows of one accumulator per CTA
 constexpr int MSUB = 2;      // accumulators (M = 256 each across the pair)
 constexpr int BNP = 256;     // weight rows per pair (N of one MMA)
 constexpr int BNC = 128;     // weight rows per CTA
-constexpr int BK = 64;       // K per stage (one 128-byte swizzle row of bf16)
+constexpr int BK = 64;       // K per stage (one 128-byte swizzle row of 16-bit values)
 constexpr int SA = 3;        // X stages
 // Dequantized weight stages: K step kt uses stage kt % SB, so the group that
 // dequantizes step kt + 4 (4 groups take every 4th step) refills the stage
@@ -64,7 +64,7 @@ constexpr int A_STAGE = MSUB * A_BYTES;  // 32 KB
 constexpr int B_BYTES = BNC * BK * 2;    // 16 KB
 constexpr int WP_BYTES = BNC * BK / 2;   // 4 KB packed codes
 constexpr int SCALE_FLOATS = 2 * BNC;    // 2 per row for blocksize 32
-constexpr int Y_BOX_BYTES = BM * 64 * 2;  // 16 KB output box (128 rows x 64 bf16)
+constexpr int Y_BOX_BYTES = BM * 64 * 2;  // 16 KB output box (128 rows x 64 values)
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + SA * A_STAGE;
 constexpr int OFF_W = OFF_B + SB * B_BYTES;

@@ -22,17 +22,17 @@
 //    shared memory, each CTA reducing and storing a share of the tokens --
 //    a fixed order, so results are bit-reproducible.  The host picks S so
 //    that the clusters fill the SMs evenly.
-//  * warp 0: TMA producer of X (NT x 64 bf16 per K step, 128-byte swizzle;
+//  * warp 0: TMA producer of X (NT x 64 16-bit values per K step, 128-byte swizzle;
 //    rows past M read as zeros).  Warp 1: allocates TMEM; one lane issues 4
 //    tcgen05.mma (K 16 each) per step and commits to the stages' "empty"
 //    barriers.  Warps 2..9: two groups of 4 warps (thread r owns weight row
 //    r) alternate K steps; each thread loads its row's 32 code bytes and
 //    block scales two of its steps ahead straight into registers (every code
 //    byte is used by exactly one thread, so no staging), builds the block's
-//    bf16 table, dequantizes with byte permutes into the 128-byte-swizzled
+//    16-bit table, dequantizes with byte permutes into the 128-byte-swizzled
 //    K-major A stage, then fence.proxy.async and one arrive per warp.
 //  * epilogue: the same 8 warps read the accumulator with tcgen05.ld (warp w
-//    sees TMEM lanes 32 (w mod 4) ..), either storing bf16 directly (S = 1)
+//    sees TMEM lanes 32 (w mod 4) ..), either rounding and storing directly (S = 1)
 //    or through the cluster reduction.
 //  * every mbarrier wait is bounded in time; on expiry the CTA sets the
 //    library's device error word, drains what it started and still reaches
@@ -85,7 +85,7 @@ __host__ __device__ constexpr uint32_t idesc_for(int nt, int fmt) {
          (static_cast<uint32_t>(nt >> 3) << 17) | (static_cast<uint32_t>(ROWS >> 4) << 24);
 }
 
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+__device__ __forceinline__ void umma16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
                                           uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -203,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t x_addr = smem_u32(x_tile(sx));
 #pragma unroll
         for (int k = 0; k < BK / 16; ++k)
-          umma_bf16(tmem, sw128_desc(a_addr + 32 * k), sw128_desc(x_addr + 32 * k), idesc,
+          umma16(tmem, sw128_desc(a_addr + 32 * k), sw128_desc(x_addr + 32 * k), idesc,
                     (i > 0 || k > 0) ? 1u : 0u);
         umma_commit(bar(bars->aempty[sa]));
         umma_commit(bar(bars->xempty[sx]));

@@ -13,20 +13,21 @@
 //    steps.  The 4 lanes of a quad own two rows (g and g + 8) and a
 //    contiguous 64-element segment of each per step (2 x 2 128-bit loads);
 //    every lane keeps 2 steps of loads (codes and raw scales) in flight.
-//  * Per (row, quant block) a lane builds the 16-entry bf16 table of
-//    bf16(RN(t[i] * a_hat)) -- bit-identical to dequantizing every element --
+//  * Per (row, quant block) a lane builds the 16-entry table of
+//    h(RN(t[i] * a_hat)) in the compute format h (bf16 or fp16) --
+//    bit-identical to dequantizing every element --
 //    split into low-byte and high-byte tables held in 8 registers.
-//  * 8 packed codes become 4 bf16x2 words with byte permutes (prmt): the low
+//  * 8 packed codes become 4 16-bit pairs with byte permutes (prmt): the low
 //    3 bits of each code select from the two 8-entry halves, bit 3 picks the
 //    half, a last permute interleaves low/high bytes.
-//  * The products run on mma.sync m16n8k16 (bf16 -> fp32) with the weight as
+//  * The products run on mma.sync m16n8k16 (bf16 or fp16 -> fp32) with the weight as
 //    the A operand (16 rows) and x as B (batch columns): one 128-bit load of
 //    x feeds two MMAs straight from its register pairs, and batch columns
 //    beyond B simply read a valid row whose outputs are discarded.  K is
 //    permuted identically in both operands, which leaves the dot products
 //    unchanged; two accumulator chains keep consecutive MMAs independent.
 //  * Partial sums of the 8 warps are reduced in shared memory in a fixed
-//    order and rounded once to bf16.
+//    order, the bias (if any) added in fp32, and rounded once.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -45,7 +46,7 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
   return d;
 }
 
-// bf16 table of one quant block, split by byte: L[q] holds the low bytes of
+// 16-bit table of one quant block, split by byte: L[q] holds the low bytes of
 // entries 4q..4q+3, H[q] the high bytes.
 struct Lut {
   uint32_t L[4], H[4];
@@ -74,7 +75,7 @@ __device__ __forceinline__ Lut make_lut(float ah) {
 }
 
 // Four codes (nibble order k1 k0 k3 k2 in the low 16 bits of the word they
-// came from) -> two bf16x2 words {k0, k1}, {k2, k3}.  `sel` holds the codes'
+// came from) -> two 16-bit pairs {k0, k1}, {k2, k3}.  `sel` holds the codes'
 // low 3 bits (the index into an 8-entry half), `mix` picks, per byte, the
 // half given by bit 3: nibble p of mix = p + 4 * bit3(code p).
 __device__ __forceinline__ void dq4(const Lut& l, uint32_t sel, uint32_t mix,
@@ -85,7 +86,7 @@ __device__ __forceinline__ void dq4(const Lut& l, uint32_t sel, uint32_t mix,
   o23 = prmt(lo, hi, 0x6273);
 }
 
-// 8 packed codes -> 4 bf16x2 words in k order.  The selectors of both halves
+// 8 packed codes -> 4 16-bit pairs in k order.  The selectors of both halves
 // come from one mask / shift of the whole word (prmt reads only the low 16
 // bits of its selector).
 __device__ __forceinline__ void dq8(const Lut& l, uint32_t w, uint32_t (&o)[4]) {

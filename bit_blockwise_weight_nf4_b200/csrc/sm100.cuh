@@ -198,7 +198,7 @@ __device__ __forceinline__ Lut make_lut(float ah) {
   return l;
 }
 
-// 8 codes of one packed 32-bit word (natural order k0..k7) -> 8 bf16 in k
+// 8 codes of one packed 32-bit word (natural order k0..k7) -> 8 16-bit values in k
 // order as 4 words.  The low 3 bits of each code select from the two
 // 8-entry halves of the table, bit 3 picks the half; one mask / shift of the
 // whole word serves both 4-code halves (prmt reads the low 16 selector bits).
