@@ -85,6 +85,8 @@ def load():
         "bnb_quantize_4bit": ([p, i32, QP, p, sz, p], ctypes.c_int),
         "bnb_quantize_4bit_noalloc": ([p, i32, QP, p], ctypes.c_int),
         "bnb_dequantize_4bit": ([QP, p, i32, p], ctypes.c_int),
+        "bnb_quantize_4bit_2d": ([p, i32, i64, i64, i64, QP, p, sz, p], ctypes.c_int),
+        "bnb_dequantize_4bit_2d": ([QP, p, i32, i64, i64, i64, p], ctypes.c_int),
         "bnb_gemv_4bit": ([p, i64, i64, QP, i64, p, p], ctypes.c_int),
         "bnb_gemm_4bit": ([p, i64, i64, QP, i64, p, p], ctypes.c_int),
         "bnb_linear_4bit": ([p, i32, i64, i64, QP, i64, p, p, p], ctypes.c_int),
@@ -134,6 +136,16 @@ def bnb_quantize_4bit_noalloc(x, x_dtype, st, stream):
 
 def bnb_dequantize_4bit(st, out, out_dtype, stream):
     return load().bnb_dequantize_4bit(ctypes.byref(st), out, out_dtype, stream)
+
+
+def bnb_quantize_4bit_2d(x, x_dtype, rows, cols, ld, st, workspace, workspace_bytes, stream):
+    return load().bnb_quantize_4bit_2d(x, x_dtype, rows, cols, ld, ctypes.byref(st),
+                                       workspace, workspace_bytes, stream)
+
+
+def bnb_dequantize_4bit_2d(st, out, out_dtype, rows, cols, ld, stream):
+    return load().bnb_dequantize_4bit_2d(ctypes.byref(st), out, out_dtype, rows, cols, ld,
+                                         stream)
 
 
 def bnb_gemv_4bit(x, B, K, W, N, y, stream):
@@ -230,35 +242,60 @@ def workspace_for(state):
                        device=state.codes.device)
 
 
+def _view_2d(t):
+    """(rows, cols, ld) of a 2-D tensor whose rows are contiguous, else None."""
+    if t.dim() != 2 or t.stride(1) != 1:
+        return None
+    return t.shape[0], t.shape[1], t.stride(0)
+
+
 def quantize_4bit(x, blocksize=64, qtype=NF4, double_quant=True, state=None,
                   workspace=None):
-    """Quantize a contiguous fp32 / bf16 / fp16 CUDA tensor (flattened)."""
-    if not x.is_contiguous():
-        raise ValueError("quantize_4bit takes a contiguous tensor")
+    """Quantize an fp32 / bf16 / fp16 tensor (in its logical row-major order):
+    a CUDA tensor, or a page-locked CPU tensor (``pin_memory()``), which the
+    kernel reads over the bus and quantizes on the way in.  Contiguous
+    tensors of any shape, or 2-D views with contiguous rows (row stride
+    ``x.stride(0)``)."""
     dt = _DT.get(str(x.dtype))
     if dt is None:
         raise TypeError("quantize_4bit takes float32, bfloat16 or float16")
+    if x.device.type == "cpu" and not x.is_pinned():
+        raise ValueError("quantize_4bit reads CPU tensors only from page-locked memory")
+    view = None if x.is_contiguous() else _view_2d(x)
+    if not x.is_contiguous() and view is None:
+        raise ValueError("quantize_4bit takes a contiguous tensor or a 2-D row-strided view")
+    device = x.device if x.device.type == "cuda" else _torch().device("cuda")
     if state is None:
-        state = QuantState(x.numel(), blocksize, qtype, double_quant, x.device)
+        state = QuantState(x.numel(), blocksize, qtype, double_quant, device)
     if workspace is None:
         workspace = workspace_for(state)
     st = state.cstruct()
-    rc = bnb_quantize_4bit(x.data_ptr(), dt, st,
-                           None if workspace is None else workspace.data_ptr(),
-                           0 if workspace is None else workspace.numel(),
-                           _stream())
+    ws = None if workspace is None else workspace.data_ptr()
+    wsb = 0 if workspace is None else workspace.numel()
+    if view is None:
+        rc = bnb_quantize_4bit(x.data_ptr(), dt, st, ws, wsb, _stream())
+    else:
+        rc = bnb_quantize_4bit_2d(x.data_ptr(), dt, *view, st, ws, wsb, _stream())
     _check(rc, "bnb_quantize_4bit")
     return state
 
 
 def dequantize_4bit(state, out_dtype=None, out=None):
-    """Dequantize to a flat fp32 (default), bf16 or fp16 CUDA tensor."""
+    """Dequantize to a flat fp32 (default), bf16 or fp16 CUDA tensor, or into
+    ``out``: a contiguous tensor of state.n elements or a 2-D view with
+    contiguous rows."""
     torch = _torch()
     out_dtype = out_dtype or torch.float32
     if out is None:
         out = torch.empty(state.n, dtype=out_dtype, device=state.codes.device)
-    rc = bnb_dequantize_4bit(state.cstruct(), out.data_ptr(), _DT[str(out.dtype)],
-                             _stream())
+    dt = _DT[str(out.dtype)]
+    if out.is_contiguous():
+        rc = bnb_dequantize_4bit(state.cstruct(), out.data_ptr(), dt, _stream())
+    else:
+        view = _view_2d(out)
+        if view is None:
+            raise ValueError("dequantize_4bit writes a contiguous tensor or a 2-D row-strided view")
+        rc = bnb_dequantize_4bit_2d(state.cstruct(), out.data_ptr(), dt, *view, _stream())
     _check(rc, "bnb_dequantize_4bit")
     return out
 

@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include "bnb4.h"
+#include "common.cuh"
 #include "kernels.h"
 
 namespace {
@@ -98,6 +99,81 @@ int check_weight(const bnb4_qstate* W, int64_t N, int64_t K) {
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? BNB4_OK : BNB4_ERR_CUDA; }
 
+// Input a kernel reads: device or managed memory, or page-locked host memory
+// mapped into the device's address space (read over the bus -- quantize on
+// load).  Pageable host memory is rejected before anything is launched.
+// *dev receives the address the device uses.
+int readable_input(const void* p, const void** dev) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the (non-sticky) error the failed query recorded
+    return BNB4_ERR_INVALID_ARG;
+  }
+  if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) {
+    *dev = p;
+    return BNB4_OK;
+  }
+  if (a.type == cudaMemoryTypeHost && a.devicePointer) {
+    *dev = a.devicePointer;
+    return BNB4_OK;
+  }
+  return BNB4_ERR_INVALID_ARG;
+}
+
+// A row-major [rows, cols] view with row stride ld over a state of n = rows
+// * cols elements: whole 16-byte chunks per row (cols and ld multiples of
+// `epc` elements), ld >= cols, and n < 2^32 (the view's index division).
+int check_view(int64_t rows, int64_t cols, int64_t ld, int64_t n, int64_t epc) {
+  if (rows < 1 || cols < 1 || ld < cols) return BNB4_ERR_SHAPE;
+  if (cols % epc != 0 || ld % epc != 0) return BNB4_ERR_SHAPE;
+  if (rows > INT64_MAX / cols || rows * cols != n) return BNB4_ERR_SHAPE;
+  if (n >= (int64_t(1) << 32)) return BNB4_ERR_SHAPE;
+  return BNB4_OK;
+}
+
+int quantize_impl(const void* x, int32_t x_dtype, const bnb4_qstate* st, void* workspace,
+                  size_t workspace_bytes, void* stream, const bnb4::View2D* view) {
+  if (!x) return BNB4_ERR_INVALID_ARG;
+  if (x_dtype != BNB4_F32 && x_dtype != BNB4_BF16 && x_dtype != BNB4_F16)
+    return BNB4_ERR_UNSUPPORTED;
+  int rc = check_state_common(st);
+  if (rc != BNB4_OK) return rc;
+  if (!st->absmax) return BNB4_ERR_INVALID_ARG;
+  if (!aligned(x, 16)) return BNB4_ERR_ALIGNMENT;
+  if (!aligned(st->absmax, 4)) return BNB4_ERR_ALIGNMENT;
+  if (st->double_quant) {
+    if (!st->absmax_q || !st->scale2 || !st->offset) return BNB4_ERR_INVALID_ARG;
+    if (!aligned(st->scale2, 4) || !aligned(st->offset, 4))
+      return BNB4_ERR_ALIGNMENT;
+    if (!workspace ||
+        workspace_bytes < sizeof(double) * static_cast<size_t>(bnb4::kMaxPartials))
+      return BNB4_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return BNB4_ERR_ALIGNMENT;
+  }
+  int sms;
+  if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
+  const void* xd;
+  if ((rc = readable_input(x, &xd)) != BNB4_OK) return rc;
+  const int grid = bnb4::quant_grid(st->n, x_dtype, sms);
+  return from_cuda(bnb4::launch_quantize(xd, x_dtype, *st, static_cast<double*>(workspace),
+                                         grid, static_cast<cudaStream_t>(stream), view));
+}
+
+int dequantize_impl(const bnb4_qstate* st, void* out, int32_t out_dtype, void* stream,
+                    const bnb4::View2D* view) {
+  if (!out) return BNB4_ERR_INVALID_ARG;
+  if (out_dtype != BNB4_F32 && out_dtype != BNB4_BF16 && out_dtype != BNB4_F16)
+    return BNB4_ERR_UNSUPPORTED;
+  int rc = check_state_read(st);
+  if (rc != BNB4_OK) return rc;
+  if (!aligned(out, 16)) return BNB4_ERR_ALIGNMENT;
+  int sms;
+  if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
+  const int grid = bnb4::dequant_grid(st->n, out_dtype, sms);
+  return from_cuda(bnb4::launch_dequantize(*st, out, out_dtype, grid,
+                                           static_cast<cudaStream_t>(stream), view));
+}
+
 // Kernel choice by the number of token rows: the mma.sync GEMV up to 8 (one
 // MMA column group), the small-M tcgen05 kernel (weight rows as the MMA's M,
 // K split over a cluster) up to 256, the 2-CTA tcgen05 GEMM above.
@@ -145,44 +221,38 @@ int bnb4_query_sizes(int64_t n, int32_t blocksize, int32_t double_quant,
 
 int bnb_quantize_4bit(const void* x, int32_t x_dtype, const bnb4_qstate* st,
                       void* workspace, size_t workspace_bytes, void* stream) {
-  if (!x) return BNB4_ERR_INVALID_ARG;
+  return quantize_impl(x, x_dtype, st, workspace, workspace_bytes, stream, nullptr);
+}
+
+int bnb_quantize_4bit_2d(const void* x, int32_t x_dtype, int64_t rows, int64_t cols,
+                         int64_t ld, const bnb4_qstate* st, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  if (!x || !st) return BNB4_ERR_INVALID_ARG;
   if (x_dtype != BNB4_F32 && x_dtype != BNB4_BF16 && x_dtype != BNB4_F16)
     return BNB4_ERR_UNSUPPORTED;
-  int rc = check_state_common(st);
+  const int rc = check_view(rows, cols, ld, st->n, x_dtype == BNB4_F32 ? 4 : 8);
   if (rc != BNB4_OK) return rc;
-  if (!st->absmax) return BNB4_ERR_INVALID_ARG;
-  if (!aligned(x, 16)) return BNB4_ERR_ALIGNMENT;
-  if (!aligned(st->absmax, 4)) return BNB4_ERR_ALIGNMENT;
-  if (st->double_quant) {
-    if (!st->absmax_q || !st->scale2 || !st->offset) return BNB4_ERR_INVALID_ARG;
-    if (!aligned(st->scale2, 4) || !aligned(st->offset, 4))
-      return BNB4_ERR_ALIGNMENT;
-    if (!workspace ||
-        workspace_bytes < sizeof(double) * static_cast<size_t>(bnb4::kMaxPartials))
-      return BNB4_ERR_WORKSPACE;
-    if (!aligned(workspace, 16)) return BNB4_ERR_ALIGNMENT;
-  }
-  int sms;
-  if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
-  const int grid = bnb4::quant_grid(st->n, x_dtype, sms);
-  return from_cuda(bnb4::launch_quantize(x, x_dtype, *st,
-                                         static_cast<double*>(workspace), grid,
-                                         static_cast<cudaStream_t>(stream)));
+  if (ld == cols)
+    return quantize_impl(x, x_dtype, st, workspace, workspace_bytes, stream, nullptr);
+  const bnb4::View2D v = bnb4::make_view(cols, ld);
+  return quantize_impl(x, x_dtype, st, workspace, workspace_bytes, stream, &v);
 }
 
 int bnb_dequantize_4bit(const bnb4_qstate* st, void* out, int32_t out_dtype,
                         void* stream) {
-  if (!out) return BNB4_ERR_INVALID_ARG;
+  return dequantize_impl(st, out, out_dtype, stream, nullptr);
+}
+
+int bnb_dequantize_4bit_2d(const bnb4_qstate* st, void* out, int32_t out_dtype, int64_t rows,
+                           int64_t cols, int64_t ld, void* stream) {
+  if (!st || !out) return BNB4_ERR_INVALID_ARG;
   if (out_dtype != BNB4_F32 && out_dtype != BNB4_BF16 && out_dtype != BNB4_F16)
     return BNB4_ERR_UNSUPPORTED;
-  int rc = check_state_read(st);
+  const int rc = check_view(rows, cols, ld, st->n, out_dtype == BNB4_F32 ? 4 : 8);
   if (rc != BNB4_OK) return rc;
-  if (!aligned(out, 16)) return BNB4_ERR_ALIGNMENT;
-  int sms;
-  if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
-  const int grid = bnb4::dequant_grid(st->n, out_dtype, sms);
-  return from_cuda(bnb4::launch_dequantize(*st, out, out_dtype, grid,
-                                           static_cast<cudaStream_t>(stream)));
+  if (ld == cols) return dequantize_impl(st, out, out_dtype, stream, nullptr);
+  const bnb4::View2D v = bnb4::make_view(cols, ld);
+  return dequantize_impl(st, out, out_dtype, stream, &v);
 }
 
 int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstate* W,

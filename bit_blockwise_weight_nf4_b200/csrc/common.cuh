@@ -113,6 +113,25 @@ __device__ __forceinline__ float half_to_f32(uint32_t bits16) {
   }
 }
 
+// A row-major [rows, cols] view whose rows start ld elements apart (ld >=
+// cols): flat element e = q * cols + c of the logical tensor lives at offset
+// q * ld + c.  q = floor(e / cols) is the high half of e * magic with magic =
+// ceil(2^64 / cols), exact for e < 2^32 and 2 <= cols < 2^32 (the error of
+// e * magic / 2^64 is below 2^-32 < 1 / cols).
+struct View2D {
+  int64_t cols, ld;
+  uint64_t magic;
+};
+
+__device__ __forceinline__ int64_t view_offset(int64_t e, const View2D& v) {
+  const uint64_t q = __umul64hi(static_cast<uint64_t>(e), v.magic);
+  return e + static_cast<int64_t>(q) * (v.ld - v.cols);
+}
+
+inline View2D make_view(int64_t cols, int64_t ld) {
+  return View2D{cols, ld, ~0ull / static_cast<uint64_t>(cols) + 1ull};
+}
+
 // Programmatic dependent launch, used only inside one API call: a kernel
 // whose predecessor on the stream is the library's own previous kernel of the
 // same call (the double-quant kernel after the quantize kernel) is launched

@@ -107,14 +107,17 @@ __device__ __forceinline__ uint32_t load_codes(const uint8_t* p) {
     return __ldg(reinterpret_cast<const uint16_t*>(p));
 }
 
-template <int OF, bool DQ, int BS>
+// STR: out is a row-major [n / v.cols, v.cols] view with rows v.ld elements
+// apart (16-byte aligned rows, n < 2^32); element e of the logical tensor is
+// written at out + view_offset(e).
+template <int OF, bool DQ, int BS, bool STR>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     dequant4_kernel(const uint8_t* __restrict__ codes, int64_t n, int qtype,
                     const float* __restrict__ absmax,
                     const uint8_t* __restrict__ absmax_q,
                     const float* __restrict__ scale2,
                     const float* __restrict__ offset,
-                    typename Out<OF>::T* __restrict__ out) {
+                    typename Out<OF>::T* __restrict__ out, View2D v) {
   using TO = typename Out<OF>::T;
   constexpr int EPL = Out<OF>::kPerChunk;
   constexpr int ROW = 32 * EPL;
@@ -134,6 +137,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const int64_t e0 = tile * TILE + lane * EPL;
     const uint8_t* cp = codes + e0 / 2;
     TO* op = out + e0;
+    int64_t et = e0;       // logical element of the lane's chunk in row 0
     int64_t b0 = e0 / BS;  // block of the lane's chunk in row 0
     const int64_t stride = n_warps * TILE;
     // block of row r relative to row 0 (ROW may be smaller than BS)
@@ -158,11 +162,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
         chunk_values<EPL>(cw[r], decode<DQ>(raw[r], off), table, w);
         cw[r] = load_codes<EPL>(cn + r * ROW / 2);
         raw[r] = load_raw<DQ>(bn + rb(r), absmax, absmax_q, scale2);
-        store_chunk<OF, EPL>(op + r * ROW, w);
+        store_chunk<OF, EPL>(STR ? out + view_offset(et + r * ROW, v) : op + r * ROW, w);
       }
       cp = cn;
       b0 = bn;
       op += stride;
+      et += stride;
     }
   }
 
@@ -182,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
       chunk_values<EPL>(cwp, decode<DQ>(load_raw<DQ>(e / BS, absmax, absmax_q, scale2), off),
                         table, w);
       if (e + EPL <= n) {
-        store_chunk<OF, EPL>(out + e, w);
+        store_chunk<OF, EPL>(STR ? out + view_offset(e, v) : out + e, w);
       } else {
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
@@ -199,23 +204,32 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 }
 
 template <int OF, bool DQ, int BS>
-cudaError_t launch(const bnb4_qstate& st, void* out, int grid, cudaStream_t s) {
+cudaError_t launch(const bnb4_qstate& st, void* out, int grid, const View2D* view,
+                   cudaStream_t s) {
   using TO = typename Out<OF>::T;
-  return launch_kernel(dequant4_kernel<OF, DQ, BS>, dim3(grid), dim3(kThreads), 0, s, false,
+  if (view)
+    return launch_kernel(dequant4_kernel<OF, DQ, BS, true>, dim3(grid), dim3(kThreads), 0, s,
+                         false, static_cast<const uint8_t*>(st.codes), st.n,
+                         static_cast<int>(st.qtype), static_cast<const float*>(st.absmax),
+                         static_cast<const uint8_t*>(st.absmax_q),
+                         static_cast<const float*>(st.scale2),
+                         static_cast<const float*>(st.offset), static_cast<TO*>(out), *view);
+  return launch_kernel(dequant4_kernel<OF, DQ, BS, false>, dim3(grid), dim3(kThreads), 0, s, false,
                        static_cast<const uint8_t*>(st.codes), st.n,
                        static_cast<int>(st.qtype), static_cast<const float*>(st.absmax),
                        static_cast<const uint8_t*>(st.absmax_q),
                        static_cast<const float*>(st.scale2),
-                       static_cast<const float*>(st.offset), static_cast<TO*>(out));
+                       static_cast<const float*>(st.offset), static_cast<TO*>(out), View2D{});
 }
 
 template <int OF, bool DQ>
-cudaError_t launch_bs(const bnb4_qstate& st, void* out, int grid, cudaStream_t s) {
+cudaError_t launch_bs(const bnb4_qstate& st, void* out, int grid, const View2D* view,
+                      cudaStream_t s) {
   switch (st.blocksize) {
-    case 32: return launch<OF, DQ, 32>(st, out, grid, s);
-    case 64: return launch<OF, DQ, 64>(st, out, grid, s);
-    case 128: return launch<OF, DQ, 128>(st, out, grid, s);
-    default: return launch<OF, DQ, 256>(st, out, grid, s);
+    case 32: return launch<OF, DQ, 32>(st, out, grid, view, s);
+    case 64: return launch<OF, DQ, 64>(st, out, grid, view, s);
+    case 128: return launch<OF, DQ, 128>(st, out, grid, view, s);
+    default: return launch<OF, DQ, 256>(st, out, grid, view, s);
   }
 }
 
@@ -232,16 +246,16 @@ int dequant_grid(int64_t n, int out_dtype, int num_sms) {
 }
 
 cudaError_t launch_dequantize(const bnb4_qstate& st, void* out, int out_dtype,
-                              int grid, cudaStream_t s) {
+                              int grid, cudaStream_t s, const View2D* view) {
   const bool dq = st.double_quant != 0;
   if (out_dtype == BNB4_F32)
-    return dq ? launch_bs<BNB4_F32, true>(st, out, grid, s)
-              : launch_bs<BNB4_F32, false>(st, out, grid, s);
+    return dq ? launch_bs<BNB4_F32, true>(st, out, grid, view, s)
+              : launch_bs<BNB4_F32, false>(st, out, grid, view, s);
   if (out_dtype == BNB4_F16)
-    return dq ? launch_bs<BNB4_F16, true>(st, out, grid, s)
-              : launch_bs<BNB4_F16, false>(st, out, grid, s);
-  return dq ? launch_bs<BNB4_BF16, true>(st, out, grid, s)
-            : launch_bs<BNB4_BF16, false>(st, out, grid, s);
+    return dq ? launch_bs<BNB4_F16, true>(st, out, grid, view, s)
+              : launch_bs<BNB4_F16, false>(st, out, grid, view, s);
+  return dq ? launch_bs<BNB4_BF16, true>(st, out, grid, view, s)
+            : launch_bs<BNB4_BF16, false>(st, out, grid, view, s);
 }
 
 }  // namespace bnb4

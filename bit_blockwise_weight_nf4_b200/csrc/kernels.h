@@ -9,17 +9,22 @@
 
 namespace bnb4 {
 
+struct View2D;  // a strided 2-D view (common.cuh)
+
 // Upper bound on the quantize grid; the double-quant workspace holds one fp64
 // partial sum per CTA.
 constexpr int kMaxPartials = 4096;
 
 int quant_grid(int64_t n, int x_dtype, int num_sms);
+// view: x is a row-major 2-D view with a row stride (see View2D), or null
+// for a contiguous x.
 cudaError_t launch_quantize(const void* x, int x_dtype, const bnb4_qstate& st,
-                            double* partials, int grid, cudaStream_t s);
+                            double* partials, int grid, cudaStream_t s,
+                            const View2D* view = nullptr);
 
 int dequant_grid(int64_t n, int out_dtype, int num_sms);
 cudaError_t launch_dequantize(const bnb4_qstate& st, void* out, int out_dtype,
-                              int grid, cudaStream_t s);
+                              int grid, cudaStream_t s, const View2D* view = nullptr);
 
 // Compares the quantize kernel's reciprocal with the correctly rounded one
 // over its whole input range; result = {u64 mismatches, u32 first, u32 0}.

@@ -290,11 +290,14 @@ __device__ __noinline__ void chunk_exact(uint4 ch, float m, int64_t e, int64_t n
   }
 }
 
-template <typename T, int BS, int QT, bool DQ>
+// STR: x is a row-major [n / v.cols, v.cols] view with rows v.ld elements
+// apart (16-byte aligned rows, n < 2^32); blocks still run over the logical
+// element order, so the results equal those of the contiguous tensor.
+template <typename T, int BS, int QT, bool DQ, bool STR>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     quant4_kernel(const T* __restrict__ x, int64_t n,
                   uint8_t* __restrict__ codes, float* __restrict__ absmax,
-                  double* __restrict__ partials) {
+                  double* __restrict__ partials, View2D v) {
   constexpr int EPL = Elem<T>::kPerChunk;  // elements per 16-byte chunk
   constexpr int LPB = BS / EPL;            // lanes (chunks) per block
   constexpr int ROW = 32 * EPL;            // elements per warp row
@@ -329,10 +332,12 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     const int64_t stride = n_warps * TILE;
     uint4 c[kRows];
 #pragma unroll
-    for (int r = 0; r < kRows; ++r) c[r] = ldg_stream_v4(xp + r * ROW);
+    for (int r = 0; r < kRows; ++r)
+      c[r] = STR ? ldg_stream_v4(x + view_offset(e0 + r * ROW, v)) : ldg_stream_v4(xp + r * ROW);
     for (; tile < n_full; tile += n_warps) {
       // the last tile of the warp refills from itself (the loads are unused)
       const T* xn = tile + n_warps < n_full ? xp + stride : xp;
+      const int64_t en = (tile + n_warps < n_full ? tile + n_warps : tile) * TILE + lane * EPL;
 #pragma unroll
       for (int r0 = 0; r0 < kRows; r0 += RG) {
         const float m = group_absmax<T, LPB, RG>(c + r0);
@@ -361,7 +366,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
           }
         }
 #pragma unroll
-        for (int rr = 0; rr < RG; ++rr) c[r0 + rr] = ldg_stream_v4(xn + (r0 + rr) * ROW);
+        for (int rr = 0; rr < RG; ++rr)
+          c[r0 + rr] = STR ? ldg_stream_v4(x + view_offset(en + (r0 + rr) * ROW, v))
+                           : ldg_stream_v4(xn + (r0 + rr) * ROW);
       }
       xp = xn;
       cp += stride / 2;
@@ -377,8 +384,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     for (int r0 = 0; r0 < kRows; r0 += RG) {
       uint4 ch[RG];
 #pragma unroll
-      for (int rr = 0; rr < RG; ++rr)
-        ch[rr] = Elem<T>::load_partial(x, t0 + static_cast<int64_t>((r0 + rr) * 32 + lane) * EPL, n);
+      for (int rr = 0; rr < RG; ++rr) {
+        const int64_t e = t0 + static_cast<int64_t>((r0 + rr) * 32 + lane) * EPL;
+        if constexpr (STR)  // whole chunks (n and the rows are chunk multiples)
+          ch[rr] = e < n ? ldg_stream_v4(x + view_offset(e, v)) : make_uint4(0, 0, 0, 0);
+        else
+          ch[rr] = Elem<T>::load_partial(x, e, n);
+      }
       const float m = group_absmax<T, LPB, RG>(ch);
       const int64_t b = (t0 + static_cast<int64_t>(r0) * ROW) / BS +
                         (LPB == 64 ? 0 : lane / LPB);
@@ -502,34 +514,37 @@ __global__ void __launch_bounds__(256) check_rcp_kernel(unsigned long long* res)
 
 template <typename T, int BS, int QT, bool DQ>
 cudaError_t launch_quant(const void* x, int64_t n, uint8_t* codes,
-                         float* absmax, double* partials, int grid,
+                         float* absmax, double* partials, int grid, const View2D* view,
                          cudaStream_t s) {
   const size_t smem = kLutEntries * 32 * sizeof(uint2);
-  return launch_kernel(quant4_kernel<T, BS, QT, DQ>, dim3(grid), dim3(kThreads), smem, s,
-                       false, static_cast<const T*>(x), n, codes, absmax, partials);
+  if (view)
+    return launch_kernel(quant4_kernel<T, BS, QT, DQ, true>, dim3(grid), dim3(kThreads), smem,
+                         s, false, static_cast<const T*>(x), n, codes, absmax, partials, *view);
+  return launch_kernel(quant4_kernel<T, BS, QT, DQ, false>, dim3(grid), dim3(kThreads), smem, s,
+                       false, static_cast<const T*>(x), n, codes, absmax, partials, View2D{});
 }
 
 template <typename T, int QT, bool DQ>
 cudaError_t dispatch_bs(int bs, const void* x, int64_t n, uint8_t* codes,
-                        float* absmax, double* partials, int grid,
+                        float* absmax, double* partials, int grid, const View2D* view,
                         cudaStream_t s) {
   switch (bs) {
-    case 32: return launch_quant<T, 32, QT, DQ>(x, n, codes, absmax, partials, grid, s);
-    case 64: return launch_quant<T, 64, QT, DQ>(x, n, codes, absmax, partials, grid, s);
-    case 128: return launch_quant<T, 128, QT, DQ>(x, n, codes, absmax, partials, grid, s);
-    default: return launch_quant<T, 256, QT, DQ>(x, n, codes, absmax, partials, grid, s);
+    case 32: return launch_quant<T, 32, QT, DQ>(x, n, codes, absmax, partials, grid, view, s);
+    case 64: return launch_quant<T, 64, QT, DQ>(x, n, codes, absmax, partials, grid, view, s);
+    case 128: return launch_quant<T, 128, QT, DQ>(x, n, codes, absmax, partials, grid, view, s);
+    default: return launch_quant<T, 256, QT, DQ>(x, n, codes, absmax, partials, grid, view, s);
   }
 }
 
 template <typename T>
 cudaError_t dispatch_q(int qt, bool dq, int bs, const void* x, int64_t n,
                        uint8_t* codes, float* absmax, double* partials,
-                       int grid, cudaStream_t s) {
+                       int grid, const View2D* view, cudaStream_t s) {
   if (qt == kQtNF4)
-    return dq ? dispatch_bs<T, kQtNF4, true>(bs, x, n, codes, absmax, partials, grid, s)
-              : dispatch_bs<T, kQtNF4, false>(bs, x, n, codes, absmax, partials, grid, s);
-  return dq ? dispatch_bs<T, kQtFP4, true>(bs, x, n, codes, absmax, partials, grid, s)
-            : dispatch_bs<T, kQtFP4, false>(bs, x, n, codes, absmax, partials, grid, s);
+    return dq ? dispatch_bs<T, kQtNF4, true>(bs, x, n, codes, absmax, partials, grid, view, s)
+              : dispatch_bs<T, kQtNF4, false>(bs, x, n, codes, absmax, partials, grid, view, s);
+  return dq ? dispatch_bs<T, kQtFP4, true>(bs, x, n, codes, absmax, partials, grid, view, s)
+            : dispatch_bs<T, kQtFP4, false>(bs, x, n, codes, absmax, partials, grid, view, s);
 }
 
 }  // namespace
@@ -557,17 +572,17 @@ int quant_grid(int64_t n, int x_dtype, int num_sms) {
 }
 
 cudaError_t launch_quantize(const void* x, int x_dtype, const bnb4_qstate& st,
-                            double* partials, int grid, cudaStream_t s) {
+                            double* partials, int grid, cudaStream_t s, const View2D* view) {
   const bool dq = st.double_quant != 0;
   cudaError_t e =
       x_dtype == BNB4_F32
           ? dispatch_q<float>(st.qtype, dq, st.blocksize, x, st.n, st.codes,
-                              st.absmax, partials, grid, s)
+                              st.absmax, partials, grid, view, s)
       : x_dtype == BNB4_F16
           ? dispatch_q<Half16>(st.qtype, dq, st.blocksize, x, st.n, st.codes,
-                               st.absmax, partials, grid, s)
+                               st.absmax, partials, grid, view, s)
           : dispatch_q<uint16_t>(st.qtype, dq, st.blocksize, x, st.n, st.codes,
-                                 st.absmax, partials, grid, s);
+                                 st.absmax, partials, grid, view, s);
   if (e != cudaSuccess || !dq) return e;
   const int64_t nb = (st.n + st.blocksize - 1) / st.blocksize;
   const int64_t ng = (nb + 255) / 256;

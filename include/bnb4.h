@@ -125,9 +125,13 @@ BNB4_API int bnb4_query_sizes(int64_t n, int32_t blocksize, int32_t double_quant
  * scale per block, nearest codebook entry, 16 codes packed two per byte;
  * section "实际性能差异": double quantization of the scales to 8 bits).
  *
- *  x           device, st->n elements of x_dtype (BNB4_F32, BNB4_BF16 or
- *              BNB4_F16; 16-bit inputs are widened to fp32 exactly),
- *              16-byte aligned.
+ *  x           st->n elements of x_dtype (BNB4_F32, BNB4_BF16 or BNB4_F16;
+ *              16-bit inputs are widened to fp32 exactly), 16-byte aligned,
+ *              in device memory or in page-locked host memory (the kernel
+ *              then reads the checkpoint over the bus and quantizes it on
+ *              the way in, with no device copy of the unquantized tensor --
+ *              the icman guide's quantize-when-moved-to-the-GPU step).
+ *              Pageable host memory is rejected (INVALID_ARG).
  *  st          state whose buffers receive the result: codes and absmax
  *              always; absmax_q, scale2 and offset when st->double_quant.
  *  workspace   device scratch of at least bnb4_query_sizes(...).workspace
@@ -180,6 +184,22 @@ BNB4_API int bnb_quantize_4bit_noalloc(const void* x, int32_t x_dtype,
                                        const bnb4_qstate* st, void* stream);
 
 /*
+ * Quantization of a non-contiguous 2-D input (release notes 0.49.2:
+ * quantize / dequantize handle non-contiguous tensors): x is a row-major
+ * [rows, cols] view whose rows start ld elements apart.  Blocks run over the
+ * logical row-major element order, so every output equals that of
+ * bnb_quantize_4bit on the contiguous copy of the view, bit for bit.  x may
+ * be device or page-locked host memory as for bnb_quantize_4bit.
+ * Constraints: st->n == rows * cols < 2^32; ld >= cols; cols and ld
+ * multiples of 8 elements (16-bit x_dtype) or 4 (fp32), so every row starts
+ * on a 16-byte boundary.  ld == cols is the contiguous case.
+ * Errors: as bnb_quantize_4bit, SHAPE for the view.
+ */
+BNB4_API int bnb_quantize_4bit_2d(const void* x, int32_t x_dtype, int64_t rows,
+                                  int64_t cols, int64_t ld, const bnb4_qstate* st,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Dequantization (NF4 article, section "实际性能差异": the 4-bit codes times
  * the decoded block scale).  w = RN(t[code] * a_hat) in fp32; with out_dtype
  * BNB4_BF16 or BNB4_F16 the output is the round-to-nearest-even of w in that
@@ -189,6 +209,18 @@ BNB4_API int bnb_quantize_4bit_noalloc(const void* x, int32_t x_dtype,
  */
 BNB4_API int bnb_dequantize_4bit(const bnb4_qstate* st, void* out, int32_t out_dtype,
                         void* stream);
+
+/*
+ * Dequantization into a non-contiguous 2-D output (release notes 0.49.2):
+ * out is a row-major [rows, cols] view, rows ld elements apart, device
+ * memory; element (r, c) receives logical element r * cols + c, bit-equal to
+ * bnb_dequantize_4bit.  Elements between the rows (ld > cols) are not
+ * written.  Constraints: st->n == rows * cols < 2^32; ld >= cols; cols and
+ * ld multiples of 8 (16-bit out_dtype) or 4 (fp32).
+ * Errors: as bnb_dequantize_4bit, SHAPE for the view.
+ */
+BNB4_API int bnb_dequantize_4bit_2d(const bnb4_qstate* st, void* out, int32_t out_dtype,
+                                    int64_t rows, int64_t cols, int64_t ld, void* stream);
 
 /*
  * Decode GEMV (release notes 0.50.0 / gemv_4bit):

@@ -159,6 +159,29 @@ def test_linear_argument_errors(lib):
     assert call(M=300, y=A16 + 2) == bnb4.ERR_ALIGNMENT                   # 16 B above 256
 
 
+def test_view_argument_errors(lib):
+    st = good_state(n=16 * 64)
+
+    def q(rows=16, cols=64, ld=72, dtype=bnb4.BF16, W=st, x=A16):
+        return bnb4.bnb_quantize_4bit_2d(x, dtype, rows, cols, ld, W, A16, 1 << 20, None)
+
+    def d(rows=16, cols=64, ld=72, dtype=bnb4.BF16, W=st, out=A16):
+        return bnb4.bnb_dequantize_4bit_2d(W, out, dtype, rows, cols, ld, None)
+    for call in (q, d):
+        assert call(rows=15) == bnb4.ERR_SHAPE                  # rows * cols != n
+        assert call(ld=60) == bnb4.ERR_SHAPE                    # ld < cols
+        assert call(cols=60, rows=16, W=good_state(n=16 * 60), ld=64) == bnb4.ERR_SHAPE
+        assert call(ld=68) == bnb4.ERR_SHAPE                    # rows not 16-byte aligned
+        assert call(dtype=9) == bnb4.ERR_UNSUPPORTED
+        assert call(rows=1 << 20, cols=1 << 12, ld=1 << 12,
+                    W=good_state(n=1 << 32)) == bnb4.ERR_SHAPE  # n >= 2^32
+        assert call(rows=0) == bnb4.ERR_SHAPE
+    # fp32 rows need only 4-element alignment
+    assert q(cols=68, ld=76, dtype=bnb4.F32, W=good_state(n=16 * 68)) != bnb4.ERR_SHAPE
+    assert q(x=None) == bnb4.ERR_INVALID_ARG
+    assert d(out=None) == bnb4.ERR_INVALID_ARG
+
+
 def test_no_cpu_fallback_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(bnb4, "_lib", None)
     monkeypatch.setattr(bnb4, "LIB_PATH", str(tmp_path / "missing.so"))
