@@ -58,11 +58,11 @@ def quantize_4bit(x: Tensor, blocksize: int, qtype: int,
     else:
         raise ValueError("bnb4::quantize_4bit takes a contiguous tensor or a row-strided 2-D view")
     _check(rc, "bnb4::quantize_4bit")
-    empty_u8 = torch.empty(0, dtype=torch.uint8, device=device)
-    empty_f32 = torch.empty(0, dtype=torch.float32, device=device)
     if double_quant:
         return st.codes, st.absmax, st.absmax_q, st.scale2, st.offset
-    return st.codes, st.absmax, empty_u8, empty_f32, empty_f32
+    # three distinct empty outputs (operator outputs may not alias each other)
+    empty = lambda dt: torch.empty(0, dtype=dt, device=device)
+    return st.codes, st.absmax, empty(torch.uint8), empty(torch.float32), empty(torch.float32)
 
 
 @quantize_4bit.register_fake
