@@ -148,6 +148,48 @@ __global__ void __launch_bounds__(kThreads, 2)
   auto x_tile = [&](int s) { return smem + OFF_X + s * xs_bytes; };
   auto bar = [&](uint64_t& b) { return smem_u32(&b); };
 
+  // Dequantizing threads (warps 2..): thread r of group grp owns weight row
+  // n0 + r and takes K steps i = grp (mod NGROUPS).  The codes and raw block
+  // scales of its first two steps are requested here, before the setup
+  // below, so their memory latency overlaps it (as does the X tensor map's).
+  const bool deq = warp >= kFirstDeqWarp;
+  const int dq = deq ? static_cast<int>(threadIdx.x) - kFirstDeqWarp * 32 : 0;
+  const int grp = dq / kGroupThreads;
+  const int r = dq % kGroupThreads;
+  const int64_t n = static_cast<int64_t>(n0) + r;
+  const bool row_ok = deq && n < N;
+  constexpr int NBLK = BS == 32 ? 2 : 1;
+  auto fetch = [&](int i, RowStep& b) {
+    b.c0 = b.c1 = make_uint4(0, 0, 0, 0);
+    b.u[0] = b.u[1] = 0u;
+    b.g[0] = b.g[1] = 0.0f;
+    if (row_ok && i < steps) {
+      const int64_t k = static_cast<int64_t>(kt0 + i) * BK;
+      const uint8_t* src = codes + n * (K / 2) + k / 2;
+      b.c0 = ldg_stream_v4(src);
+      b.c1 = ldg_stream_v4(src + 16);
+      const int64_t blk = (n * K + k) / BS;
+#pragma unroll
+      for (int j = 0; j < NBLK; ++j) {
+        if constexpr (DQ) {
+          b.u[j] = __ldg(absmax_q + blk + j);
+          b.g[j] = __ldg(scale2 + ((blk + j) >> 8));
+        } else {
+          b.u[j] = __float_as_uint(__ldg(absmax + blk + j));
+        }
+      }
+    }
+  };
+  // two register sets, each refilled two of the group's steps ahead
+  RowStep b0, b1;
+  if (deq) {
+    fetch(grp, b0);
+    fetch(grp + NGROUPS, b1);
+  }
+  if (threadIdx.x == 0)
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_x))
+                 : "memory");
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < SA; ++s) {
       mbar_init(bar(bars->afull[s]), kGroupThreads / 32);
@@ -214,34 +256,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   } else {
     // ------------------------------------------------------ dequantizers
-    const int dq = threadIdx.x - kFirstDeqWarp * 32;
-    const int grp = dq / kGroupThreads;  // takes steps i = grp (mod NGROUPS)
-    const int r = dq % kGroupThreads;    // weight row of the CTA
-    const int64_t n = static_cast<int64_t>(n0) + r;
-    const bool row_ok = n < N;
     const float off = DQ ? __ldg(offset) : 0.0f;
-    constexpr int NBLK = BS == 32 ? 2 : 1;
-    auto fetch = [&](int i, RowStep& b) {
-      b.c0 = b.c1 = make_uint4(0, 0, 0, 0);
-      b.u[0] = b.u[1] = 0u;
-      b.g[0] = b.g[1] = 0.0f;
-      if (row_ok && i < steps) {
-        const int64_t k = static_cast<int64_t>(kt0 + i) * BK;
-        const uint8_t* src = codes + n * (K / 2) + k / 2;
-        b.c0 = ldg_stream_v4(src);
-        b.c1 = ldg_stream_v4(src + 16);
-        const int64_t blk = (n * K + k) / BS;
-#pragma unroll
-        for (int j = 0; j < NBLK; ++j) {
-          if constexpr (DQ) {
-            b.u[j] = __ldg(absmax_q + blk + j);
-            b.g[j] = __ldg(scale2 + ((blk + j) >> 8));
-          } else {
-            b.u[j] = __float_as_uint(__ldg(absmax + blk + j));
-          }
-        }
-      }
-    };
     // one warp-uniform decision per wait: lane 0 waits, the warp follows
     auto warp_wait = [&](uint32_t b, uint32_t parity) {
       bool w = true;
@@ -282,10 +297,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (lane == 0) mbar_arrive(bar(bars->afull[sa]));
       return true;
     };
-    // two register sets, each refilled two of the group's steps ahead
-    RowStep b0, b1;
-    fetch(grp, b0);
-    fetch(grp + NGROUPS, b1);
     for (int i = grp; i < steps && ok; i += 2 * NGROUPS) {
       ok = step(i, b0);
       fetch(i + 2 * NGROUPS, b0);
@@ -341,9 +352,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (S > 1 && warp >= kFirstDeqWarp) {
     // rank s reduces tokens [s * per, (s + 1) * per): thread (r, c0) sums
     // the ranks' partials of weight row r in rank order, tokens c0, c0 + 2, ..
-    const int dq = threadIdx.x - kFirstDeqWarp * 32;
-    const int r = dq % ROWS, c0 = dq / ROWS;
-    const int64_t nr = static_cast<int64_t>(n0) + r;
+    const int c0 = grp;    // thread (r, c0): weight row r, tokens c0, c0 + 2, ..
+    const int64_t nr = n;
     const int per = (M + S - 1) / S;
     const int t0 = r_ * per;
     const int t1 = t0 + per < M ? t0 + per : M;
