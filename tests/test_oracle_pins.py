@@ -231,6 +231,176 @@ def test_bf16_input_is_exact_widening():
         assert np.array_equal(a[k], b[k]), k
 
 
+# ------------------------------------------- normalisation by the reciprocal
+# Reading R5: v = RN(x * RN(1 / absmax)).  The two plausible alternatives --
+# dividing, v = RN(x / absmax), or normalising in fp64 and rounding once to
+# fp32 -- differ from it by at most one fp32 ulp of v, so they give a
+# different code only where that ulp straddles a codebook midpoint.  The
+# search below builds such (x, absmax) pairs in exact rational arithmetic
+# and checks that the oracle takes the reciprocal reading on every one.
+
+def _ulp_step(x, k):
+    """The fp32 value k ulps away from fp32 x (k may be negative)."""
+    v = np.float32(x)
+    toward = np.float32(np.inf) if k > 0 else np.float32(-np.inf)
+    for _ in range(abs(k)):
+        v = np.nextafter(v, toward)
+    return v
+
+
+def _r6_midpoints(qtype):
+    """Reading R6's fp32 midpoints RN(RN(t[i] + t[i+1]) * 0.5), rounded here
+    in exact rational arithmetic (NF4: 15 ascending; FP4: 7 magnitudes).
+    Where t[i] + t[i+1] is not an fp32 number the midpoint sits an ulp off
+    the exact one, so the code can differ from the exact argmin on that
+    single value."""
+    t = [Fraction(float(v)) for v in oracle.codebook(qtype)]
+    k = 15 if qtype == oracle.NF4 else 7
+    return [frac_to_f32(Fraction(float(frac_to_f32(t[i] + t[i + 1]))) / 2)
+            for i in range(k)]
+
+
+def r6_code(qtype, v):
+    """Code of fp32 v under R6: the number of fp32 midpoints strictly below v
+    (FP4: below |v|, sign bit for a negative value with a non-zero
+    magnitude)."""
+    mids = _r6_midpoints(qtype)
+    fv = Fraction(float(v))
+    if qtype == oracle.NF4:
+        return sum(1 for m in mids if fv > Fraction(float(m)))
+    m = sum(1 for mm in mids if abs(fv) > Fraction(float(mm)))
+    return m | 8 if (fv < 0 and m > 0) else m
+
+
+def test_r6_midpoints_equal_nearest_except_on_rounded_midpoints():
+    """R6 against the exact argmin.  An fp32 midpoint lies within half an
+    ulp of the exact one, so the fp32 values on either side of it get the
+    exact nearest code; on the midpoint itself the tie rule gives the lower
+    index, which is the exact nearest entry unless the fp32 midpoint was
+    rounded above the exact one (then the value is strictly closer to the
+    upper entry: a documented consequence of R6)."""
+    rounded_up = 0
+    for qtype in (oracle.NF4, oracle.FP4):
+        t = oracle.codebook(qtype)
+        for i, m in enumerate(_r6_midpoints(qtype)):
+            exact = (Fraction(float(t[i])) + Fraction(float(t[i + 1]))) / 2
+            below = np.nextafter(m, np.float32(-2))
+            above = np.nextafter(m, np.float32(2))
+            assert r6_code(qtype, below) == brute_nearest(qtype, below) == i
+            assert r6_code(qtype, above) == brute_nearest(qtype, above) == i + 1
+            assert r6_code(qtype, m) == oracle.nearest_code(qtype, float(m)) == i
+            if Fraction(float(m)) > exact:
+                rounded_up += 1
+                assert brute_nearest(qtype, m) == i + 1
+            else:
+                assert brute_nearest(qtype, m) == i
+    assert rounded_up > 0
+
+
+def _straddle_cases(qtype, want=24, seed=21):
+    """(a, x, code_reciprocal, code_division) with the two readings on
+    opposite sides of a midpoint; both orientations, positive and negative
+    x."""
+    rng = np.random.default_rng(seed)
+    mids = [Fraction(float(m)) for m in _r6_midpoints(qtype)]
+    if qtype == oracle.FP4:
+        mids = mids + [-m for m in mids]
+    out, seen = [], set()
+    tries = 0
+    while len(out) < want and tries < 4000:
+        tries += 1
+        a = np.float32(rng.uniform(0.01, 0.09))
+        fa = Fraction(float(a))
+        r = frac_to_f32(1 / fa)
+        # a reciprocal with a large relative error makes straddles likely
+        if abs(Fraction(float(r)) * fa - 1) < Fraction(1, 2 ** 26):
+            continue
+        for m in mids:
+            x0 = frac_to_f32(m * fa)
+            for k in range(-3, 4):
+                x = _ulp_step(x0, k)
+                if not (abs(float(x)) < float(a)):
+                    continue
+                fx = Fraction(float(x))
+                v_rcp = frac_to_f32(fx * Fraction(float(r)))
+                v_div = frac_to_f32(fx / fa)
+                c_rcp = r6_code(qtype, v_rcp)
+                c_div = r6_code(qtype, v_div)
+                if c_rcp != c_div:
+                    key = (int(c_rcp > c_div), bool(x < 0))
+                    seen.add(key)
+                    out.append((a, x, c_rcp, c_div))
+    return out, seen
+
+
+@pytest.mark.parametrize("qtype", [oracle.NF4, oracle.FP4])
+def test_normalisation_multiplies_by_rounded_reciprocal(qtype):
+    cases, seen = _straddle_cases(qtype)
+    assert len(cases) >= 24
+    # both directions of the disagreement, and (NF4) both signs of x
+    assert {k[0] for k in seen} == {0, 1}
+    if qtype == oracle.NF4:
+        assert {k[1] for k in seen} == {False, True}
+    bs = 32
+    x = np.zeros(len(cases) * bs, np.float32)
+    for j, (a, xv, _, _) in enumerate(cases):
+        x[j * bs] = a          # the block max, code +-1
+        x[j * bs + 1] = xv     # the straddling element
+    st = oracle.quantize(x, bs, qtype, double_quant=False)
+    hi = st["codes"] >> 4
+    lo = st["codes"] & 15
+    for j, (a, xv, c_rcp, c_div) in enumerate(cases):
+        assert st["absmax"][j] == a
+        got = int(lo[j * bs // 2])  # element 1 of the block: low nibble of byte 0
+        assert got == c_rcp, (float(a), float(xv))
+        assert got != c_div
+        # normalising in fp64 and rounding once lands on the division's side
+        v64 = np.float32(np.float64(xv) / np.float64(a))
+        assert r6_code(qtype, v64) == c_div
+        assert int(hi[j * bs // 2]) == (15 if qtype == oracle.NF4 else 7)
+
+
+def _r6_vectorised(qtype, v):
+    """r6_code over an fp32 array (fp32 comparisons are exact)."""
+    mids = np.array(_r6_midpoints(qtype), np.float32)
+    if qtype == oracle.NF4:
+        return (v[:, None] > mids[None, :]).sum(axis=1)
+    m = (np.abs(v)[:, None] > mids[None, :]).sum(axis=1)
+    return np.where((v < 0) & (m > 0), m | 8, m)
+
+
+@pytest.mark.parametrize("qtype", [oracle.NF4, oracle.FP4])
+def test_quantize_codes_match_reciprocal_restatement(qtype):
+    """10^5 N(0, 0.02^2) elements: every code equals R6's code of
+    RN(x * RN(1/a)), computed here with IEEE fp32 arithmetic (itself checked
+    against exact rational rounding on a sample)."""
+    rng = np.random.default_rng(23)
+    n, bs = 100_000, 64
+    x = (rng.standard_normal(n) * 0.02).astype(np.float32)
+    st = oracle.quantize(x, bs, qtype, double_quant=False)
+    codes = np.zeros(n, np.uint8)
+    codes[0::2] = st["codes"] >> 4
+    codes[1::2] = st["codes"] & 15
+    nb = (n + bs - 1) // bs
+    pad = np.zeros(nb * bs, np.float32)
+    pad[:n] = x
+    a = np.abs(pad.reshape(nb, bs)).max(axis=1).astype(np.float32)
+    assert np.array_equal(a, st["absmax"])
+    r = (np.float32(1.0) / a).astype(np.float32)
+    v = (x * np.repeat(r, bs)[:n]).astype(np.float32)
+    assert v.dtype == np.float32
+    for i in rng.choice(n, 300, replace=False):
+        b = i // bs
+        assert r[b] == frac_to_f32(1 / Fraction(float(a[b])))
+        assert v[i] == frac_to_f32(Fraction(float(x[i])) * Fraction(float(r[b])))
+    assert np.array_equal(codes, _r6_vectorised(qtype, v).astype(np.uint8))
+    # away from the rounded midpoints the codes are the exact nearest entries
+    sample = rng.choice(n, 2000, replace=False)
+    for i in sample:
+        if v[i] not in set(_r6_midpoints(qtype)):
+            assert codes[i] == brute_nearest(qtype, v[i])
+
+
 # ------------------------------------------------------- double quantization
 def test_double_quant_offset_is_exact_mean():
     rng = np.random.default_rng(7)
