@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "bnb4.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -31,32 +33,37 @@ int current_device(int* dev) {
   return BNB4_OK;
 }
 
+// Per-device caches of values that never change while the process runs.
+// Host threads may fill them concurrently: each slot is an atomic written
+// with the same value by whichever thread gets there, read relaxed.
 int num_sms(int* out) {
-  static int cache[kMaxDevices];
+  static std::atomic<int> cache[kMaxDevices];
   int dev;
   if (current_device(&dev) != BNB4_OK) return BNB4_ERR_CUDA;
-  if (cache[dev] == 0) {
-    int v = 0;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) !=
             cudaSuccess || v <= 0)
       return BNB4_ERR_CUDA;
-    cache[dev] = v;
+    cache[dev].store(v, std::memory_order_relaxed);
   }
-  *out = cache[dev];
+  *out = v;
   return BNB4_OK;
 }
 
 int error_word(int** out) {
-  static int* cache[kMaxDevices];
+  static std::atomic<int*> cache[kMaxDevices];
   int dev;
   if (current_device(&dev) != BNB4_OK) return BNB4_ERR_CUDA;
-  if (cache[dev] == nullptr) {
+  int* w = cache[dev].load(std::memory_order_relaxed);
+  if (w == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess || !p)
       return BNB4_ERR_CUDA;
-    cache[dev] = static_cast<int*>(p);
+    w = static_cast<int*>(p);
+    cache[dev].store(w, std::memory_order_relaxed);
   }
-  *out = cache[dev];
+  *out = w;
   return BNB4_OK;
 }
 
@@ -99,25 +106,71 @@ int check_weight(const bnb4_qstate* W, int64_t N, int64_t K) {
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? BNB4_OK : BNB4_ERR_CUDA; }
 
-// Input a kernel reads: device or managed memory, or page-locked host memory
-// mapped into the device's address space (read over the bus -- quantize on
-// load).  Pageable host memory is rejected before anything is launched.
-// *dev receives the address the device uses.
-int readable_input(const void* p, const void** dev) {
+}  // namespace
+
+// Where a pointer that a kernel will dereference lives (declared in
+// kernels.h, shared with the allocation-free entry point).  Device memory
+// is used as it is; managed memory too where `where` allows it; page-locked
+// host memory, where allowed, through the device address the runtime maps
+// it to (the quantize kernels then stream it over the bus -- quantize on
+// load).  Anything else, pageable host memory in particular, is refused
+// before anything is launched: a kernel given a plain host address would
+// fault.  *dev receives the address the device uses.
+int bnb4::resolve_ptr(const void* p, Residency where, const void** dev) {
   cudaPointerAttributes a;
   if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
     cudaGetLastError();  // clear the (non-sticky) error the failed query recorded
     return BNB4_ERR_INVALID_ARG;
   }
-  if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) {
+  if (a.type == cudaMemoryTypeDevice) {
     *dev = p;
     return BNB4_OK;
   }
-  if (a.type == cudaMemoryTypeHost && a.devicePointer) {
+  if (a.type == cudaMemoryTypeManaged && where != Residency::kDevice) {
+    *dev = p;
+    return BNB4_OK;
+  }
+  if (a.type == cudaMemoryTypeHost && a.devicePointer &&
+      where == Residency::kDeviceOrPinnedHost) {
     *dev = a.devicePointer;
     return BNB4_OK;
   }
   return BNB4_ERR_INVALID_ARG;
+}
+
+namespace {
+
+// The pointers of a quantization state that a kernel touches: device or
+// managed memory.  `scales_of_reader`: only the scale arrays a consumer reads
+// (absmax without double quantization, the three double-quant arrays with
+// it); otherwise every non-null array the quantize kernels write.
+int check_state_memory(const bnb4_qstate* st, bool scales_of_reader,
+                       bnb4::Residency where = bnb4::Residency::kDeviceOrManaged) {
+  const void* d;
+  int rc;
+  if ((rc = bnb4::resolve_ptr(st->codes, where, &d)) != BNB4_OK) return rc;
+  const bool want_absmax = scales_of_reader ? !st->double_quant : st->absmax != nullptr;
+  const bool want_dq = st->double_quant != 0;
+  if (want_absmax && (rc = bnb4::resolve_ptr(st->absmax, where, &d)) != BNB4_OK) return rc;
+  if (want_dq) {
+    if ((rc = bnb4::resolve_ptr(st->absmax_q, where, &d)) != BNB4_OK) return rc;
+    if ((rc = bnb4::resolve_ptr(st->scale2, where, &d)) != BNB4_OK) return rc;
+    if ((rc = bnb4::resolve_ptr(st->offset, where, &d)) != BNB4_OK) return rc;
+  }
+  return BNB4_OK;
+}
+
+// Activations, outputs and bias of the linear entry points: device memory
+// (the kernels read x and write y through TMA on the larger tiers).
+int check_linear_memory(const void* x, const void* y, const void* bias,
+                        const bnb4_qstate* W) {
+  const void* d;
+  int rc;
+  const auto dev = bnb4::Residency::kDevice;
+  if ((rc = bnb4::resolve_ptr(x, dev, &d)) != BNB4_OK) return rc;
+  if ((rc = bnb4::resolve_ptr(y, dev, &d)) != BNB4_OK) return rc;
+  if (bias && (rc = bnb4::resolve_ptr(bias, dev, &d)) != BNB4_OK) return rc;
+  return check_state_memory(W, true, dev);
 }
 
 // A row-major [rows, cols] view with row stride ld over a state of n = rows
@@ -152,8 +205,14 @@ int quantize_impl(const void* x, int32_t x_dtype, const bnb4_qstate* st, void* w
   }
   int sms;
   if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
-  const void* xd;
-  if ((rc = readable_input(x, &xd)) != BNB4_OK) return rc;
+  const void *xd, *ws_dev;
+  if ((rc = bnb4::resolve_ptr(x, bnb4::Residency::kDeviceOrPinnedHost, &xd)) != BNB4_OK)
+    return rc;
+  if ((rc = check_state_memory(st, false)) != BNB4_OK) return rc;
+  if (st->double_quant &&
+      (rc = bnb4::resolve_ptr(workspace, bnb4::Residency::kDeviceOrManaged, &ws_dev)) !=
+          BNB4_OK)
+    return rc;
   const int grid = bnb4::quant_grid(st->n, x_dtype, sms);
   return from_cuda(bnb4::launch_quantize(xd, x_dtype, *st, static_cast<double*>(workspace),
                                          grid, static_cast<cudaStream_t>(stream), view));
@@ -169,6 +228,10 @@ int dequantize_impl(const bnb4_qstate* st, void* out, int32_t out_dtype, void* s
   if (!aligned(out, 16)) return BNB4_ERR_ALIGNMENT;
   int sms;
   if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
+  const void* od;
+  if ((rc = bnb4::resolve_ptr(out, bnb4::Residency::kDeviceOrManaged, &od)) != BNB4_OK)
+    return rc;
+  if ((rc = check_state_memory(st, true)) != BNB4_OK) return rc;
   const int grid = bnb4::dequant_grid(st->n, out_dtype, sms);
   return from_cuda(bnb4::launch_dequantize(*st, out, out_dtype, grid,
                                            static_cast<cudaStream_t>(stream), view));
@@ -264,6 +327,7 @@ int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstate* W,
   if (!aligned(x, 16) || !aligned(y, 2)) return BNB4_ERR_ALIGNMENT;
   int sms;
   if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
+  if ((rc = check_linear_memory(x, y, nullptr, W)) != BNB4_OK) return rc;
   if (B <= kGemvMaxB)
     return from_cuda(bnb4::launch_gemv(x, B, K, *W, N, y, nullptr, BNB4_BF16, sms,
                                        static_cast<cudaStream_t>(stream)));
@@ -283,6 +347,7 @@ int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstate* W,
   if (!aligned(X, 16) || !aligned(Y, 16)) return BNB4_ERR_ALIGNMENT;
   int sms;
   if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
+  if ((rc = check_linear_memory(X, Y, nullptr, W)) != BNB4_OK) return rc;
   int* err;
   if ((rc = error_word(&err)) != BNB4_OK) return rc;
   if (M <= kGemvMaxB)
@@ -307,6 +372,7 @@ int bnb_linear_4bit(const void* x, int32_t dtype, int64_t M, int64_t K, const bn
     return BNB4_ERR_ALIGNMENT;
   int sms;
   if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
+  if ((rc = check_linear_memory(x, y, bias, W)) != BNB4_OK) return rc;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (M <= kGemvMaxB)
     return from_cuda(bnb4::launch_gemv(x, M, K, *W, N, y, bias, dtype, sms, s));
@@ -329,6 +395,7 @@ int bnb4_debug_gemm_withhold(const void* X, int64_t M, int64_t K,
   if (!aligned(X, 16) || !aligned(Y, 16)) return BNB4_ERR_ALIGNMENT;
   int sms;
   if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
+  if ((rc = check_linear_memory(X, Y, nullptr, W)) != BNB4_OK) return rc;
   int* err;
   if ((rc = error_word(&err)) != BNB4_OK) return rc;
   return from_cuda(bnb4::launch_gemm(X, M, K, *W, N, Y, nullptr, BNB4_BF16, err, sms,
@@ -339,6 +406,9 @@ int bnb4_debug_gemm_withhold(const void* X, int64_t M, int64_t K,
 int bnb4_debug_check_rcp(void* result, void* stream) {
   if (!result) return BNB4_ERR_INVALID_ARG;
   if (!aligned(result, 8)) return BNB4_ERR_ALIGNMENT;
+  const void* d;
+  const int rc = bnb4::resolve_ptr(result, bnb4::Residency::kDeviceOrManaged, &d);
+  if (rc != BNB4_OK) return rc;
   return from_cuda(bnb4::launch_check_rcp(result, static_cast<cudaStream_t>(stream)));
 }
 

@@ -11,6 +11,15 @@ namespace bnb4 {
 
 struct View2D;  // a strided 2-D view (common.cuh)
 
+// Where a pointer a kernel dereferences may live: device memory only;
+// device or managed memory; device, managed or page-locked host memory.
+enum class Residency { kDevice, kDeviceOrManaged, kDeviceOrPinnedHost };
+
+// BNB4_OK with the address the device uses in *dev, or BNB4_ERR_INVALID_ARG
+// (pageable host memory, a pointer the runtime does not know, or a kind of
+// memory `where` excludes).  Host-only; launches nothing.
+int resolve_ptr(const void* p, Residency where, const void** dev);
+
 // Upper bound on the quantize grid; the double-quant workspace holds one fp64
 // partial sum per CTA.
 constexpr int kMaxPartials = 4096;

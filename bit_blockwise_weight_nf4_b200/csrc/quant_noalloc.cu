@@ -14,6 +14,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "bnb4.h"
 #include "kernels.h"
 
@@ -37,34 +39,42 @@ bool aligned(const void* p, uintptr_t a) {
 // Device address of the scratch array on the current device.  In host code
 // `g_noalloc_scratch` names a host-side stand-in, not device memory, so the
 // address is looked up once per device (with that device current) and cached.
+// The lookup also loads the module holding the array on that device (lazy
+// module loading), which maps its memory: that first call can therefore fail
+// with BNB4_ERR_CUDA when the device is out of memory.  Two host threads may
+// make their first call at once; both store the same address (atomic slot).
 int scratch_address(unsigned char** out) {
-  static unsigned char* cache[kMaxDevices];
+  static std::atomic<unsigned char*> cache[kMaxDevices];
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
     return BNB4_ERR_CUDA;
-  if (cache[dev] == nullptr) {
+  unsigned char* a = cache[dev].load(std::memory_order_relaxed);
+  if (a == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
       return BNB4_ERR_CUDA;
-    cache[dev] = static_cast<unsigned char*>(p);
+    }
+    a = static_cast<unsigned char*>(p);
+    cache[dev].store(a, std::memory_order_relaxed);
   }
-  *out = cache[dev];
+  *out = a;
   return BNB4_OK;
 }
 
 int sm_count(int* out) {
-  static int cache[kMaxDevices];
+  static std::atomic<int> cache[kMaxDevices];
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
     return BNB4_ERR_CUDA;
-  if (cache[dev] == 0) {
-    int v = 0;
+  int v = cache[dev].load(std::memory_order_relaxed);
+  if (v == 0) {
     if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         v <= 0)
       return BNB4_ERR_CUDA;
-    cache[dev] = v;
+    cache[dev].store(v, std::memory_order_relaxed);
   }
-  *out = cache[dev];
+  *out = v;
   return BNB4_OK;
 }
 
@@ -91,6 +101,19 @@ extern "C" BNB4_API int bnb_quantize_4bit_noalloc(const void* x, int32_t x_dtype
 
   int sms = 0, rc;
   if ((rc = sm_count(&sms)) != BNB4_OK) return rc;
+  // x follows bnb_quantize_4bit's rules (device, managed or page-locked host
+  // memory, the latter read through its device address); the outputs must
+  // be device or managed memory.  A pointer query allocates nothing.
+  const void* xd = nullptr;
+  const void* d = nullptr;
+  if ((rc = bnb4::resolve_ptr(x, bnb4::Residency::kDeviceOrPinnedHost, &xd)) != BNB4_OK)
+    return rc;
+  const auto out_mem = bnb4::Residency::kDeviceOrManaged;
+  if ((rc = bnb4::resolve_ptr(st->codes, out_mem, &d)) != BNB4_OK ||
+      (rc = bnb4::resolve_ptr(st->absmax_q, out_mem, &d)) != BNB4_OK ||
+      (rc = bnb4::resolve_ptr(st->scale2, out_mem, &d)) != BNB4_OK ||
+      (rc = bnb4::resolve_ptr(st->offset, out_mem, &d)) != BNB4_OK)
+    return rc;
   unsigned char* scratch = nullptr;
   if ((rc = scratch_address(&scratch)) != BNB4_OK) return rc;
   const int grid = bnb4::quant_grid(st->n, x_dtype, sms);
@@ -99,7 +122,7 @@ extern "C" BNB4_API int bnb_quantize_4bit_noalloc(const void* x, int32_t x_dtype
   bnb4_qstate s = *st;  // same kernels, with the intermediate absmax in scratch
   s.absmax = reinterpret_cast<float*>(scratch + kPartialsBytes);
   const cudaError_t e = bnb4::launch_quantize(
-      x, x_dtype, s, reinterpret_cast<double*>(scratch), grid,
+      xd, x_dtype, s, reinterpret_cast<double*>(scratch), grid,
       static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BNB4_OK : BNB4_ERR_CUDA;
 }

@@ -20,6 +20,14 @@
  *  - All data pointers are DEVICE pointers owned and allocated by the caller.
  *    The library never allocates, frees or synchronizes (except
  *    bnb4_device_status, which synchronizes the stream it is given).
+ *  - Memory kinds (checked with cudaPointerGetAttributes before any launch):
+ *    the linear entry points (bnb_gemv_4bit, bnb_gemm_4bit, bnb_linear_4bit)
+ *    take device memory only, for x, y, bias and the weight's arrays (their
+ *    larger tiers move tiles with TMA); quantize and dequantize take device
+ *    or managed memory, and the quantize input x may also be page-locked host
+ *    memory.  Any other pointer -- pageable host memory in particular, which
+ *    a kernel cannot dereference -- returns BNB4_ERR_INVALID_ARG with nothing
+ *    launched.
  *  - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
  *    stream.  Work is enqueued asynchronously on it.
  *  - Every call returns a status (BNB4_OK = 0, negative on error).  On an
@@ -169,9 +177,15 @@ BNB4_API int bnb_quantize_4bit(const void* x, int32_t x_dtype, const bnb4_qstate
  *    larger inputs return BNB4_ERR_SCRATCH_LIMIT and launch nothing.
  *  - st->double_quant must be 1 (without double quantization
  *    bnb_quantize_4bit needs no workspace anyway): else INVALID_ARG.
+ *  - x follows the rules of bnb_quantize_4bit (device, managed or
+ *    page-locked host memory; pageable host memory returns INVALID_ARG);
+ *    the outputs must be device or managed memory.
  *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress, once per device, with that device current); make
- *    that first call before any stream capture on the device.
+ *    (cudaGetSymbolAddress, once per device, with that device current).
+ *    With lazy module loading (CUDA's default) that lookup also loads the
+ *    array's module and maps its 4 MiB on the device, so the first call can
+ *    return BNB4_ERR_CUDA when the device is out of memory: make it at
+ *    start-up, before any stream capture on the device.
  *  - Every call shares the one array, and a call overwrites all of the
  *    scratch it reads, so nothing carries over from the previous call; calls
  *    that overlap on the GPU (different streams, or devices sharing a

@@ -5,9 +5,10 @@ hand the library a workspace (a plugin whose host framework owns every
 device allocation, or a latency-critical loader that must not call
 cudaMalloc).  It keeps its scratch in a fixed array inside the library, so
 these tests check that two calls in a row -- the second on a different input,
-after the first has left its own values in that shared array -- give exactly
-the codes and double-quant scales of bnb_quantize_4bit, and that inputs
-larger than the fixed scratch are refused before anything is launched.
+after the first has left its own values in that shared array, also a small
+input right after a large one -- give exactly the codes and double-quant
+scales of bnb_quantize_4bit and of the CPU oracle, and that inputs larger
+than the fixed scratch are refused before anything is launched.
 
 This file is collected last (pytest orders files by name), so a run that
 stops at the first failure has already run every other test; it also passes
@@ -18,6 +19,7 @@ import pytest
 import torch
 
 import bit_blockwise_weight_nf4_b200 as bnb4
+import oracle
 import synth
 
 pytestmark = pytest.mark.gpu
@@ -50,34 +52,65 @@ def _regular(x, blocksize, qtype):
 
 CASES = [
     # (shape, dtype, blocksize, qtype): bf16 Llama-sized matrix with
-    # outliers, fp32 vector, ragged bf16 length with blocksize 32
+    # outliers, fp32 vector, ragged bf16 length with blocksize 32, fp16
     ((4096, 4096), "bf16", 64, bnb4.NF4),
     ((1 << 20,), "f32", 64, bnb4.FP4),
     ((100003,), "bf16", 32, bnb4.NF4),
+    ((3 * 65536 + 40,), "f16", 128, bnb4.FP4),
 ]
+DT = {"f32": bnb4.F32, "bf16": bnb4.BF16, "f16": bnb4.F16}
 
 
 def _input(shape, dtype, seed):
     if dtype == "f32":
         return synth.normal_f32(shape, seed=seed, std=0.02).cuda()
+    if dtype == "f16":
+        return synth.normal_f32(shape, seed=seed, std=0.02).to(torch.float16).cuda()
     if len(shape) == 2:
         return synth.weight_bf16(shape[0], shape[1], seed=seed,
                                  outlier_frac=synth.OUTLIER_FRAC).cuda().view(-1)
     return synth.normal_f32(shape, seed=seed, std=0.02).to(torch.bfloat16).cuda()
 
 
+def _oracle(x, blocksize, qtype):
+    h = x.cpu()
+    if h.dtype == torch.bfloat16:
+        h = synth.bf16_bits(h)
+    else:
+        h = h.numpy()
+    return oracle.quantize(h, blocksize, qtype, True)
+
+
+def _assert_equal(g, w, orc):
+    for k in ("codes", "absmax_q", "scale2", "offset"):
+        assert torch.equal(g[k], w[k]), k
+        assert np.array_equal(g[k].cpu().numpy(), orc[k]), k
+
+
 @pytest.mark.parametrize("shape,dtype,blocksize,qtype", CASES)
 def test_noalloc_matches_regular_two_calls_in_a_row(shape, dtype, blocksize, qtype):
-    dt = bnb4.F32 if dtype == "f32" else bnb4.BF16
+    dt = DT[dtype]
     xs = [_input(shape, dtype, seed) for seed in (21, 22)]
     got = [_noalloc(x, dt, blocksize, qtype) for x in xs]   # back to back
     want = [_regular(x, blocksize, qtype) for x in xs]
     torch.cuda.synchronize()
-    for g, w in zip(got, want):
-        for k in ("codes", "absmax_q", "scale2", "offset"):
-            assert torch.equal(g[k], w[k]), k
+    for x, g, w in zip(xs, got, want):
+        _assert_equal(g, w, _oracle(x, blocksize, qtype))
     # the two inputs differ, so equal outputs would mean stale scratch
     assert not torch.equal(got[0]["codes"], got[1]["codes"])
+
+
+def test_noalloc_large_then_small():
+    """A large call fills the shared scratch (every CTA's partial sum, every
+    block's absmax); the small call right after uses a smaller grid and
+    fewer blocks and must not read any of the leftovers."""
+    big = _input((4096, 4096), "bf16", 31)
+    small = _input((100003,), "bf16", 32)
+    g_big = _noalloc(big, bnb4.BF16, 64, bnb4.NF4)
+    g_small = _noalloc(small, bnb4.BF16, 64, bnb4.NF4)
+    torch.cuda.synchronize()
+    _assert_equal(g_big, _regular(big, 64, bnb4.NF4), _oracle(big, 64, bnb4.NF4))
+    _assert_equal(g_small, _regular(small, 64, bnb4.NF4), _oracle(small, 64, bnb4.NF4))
 
 
 def test_noalloc_refuses_inputs_beyond_its_scratch():
