@@ -1,30 +1,47 @@
 #!/usr/bin/env python3
-"""Benchmark of the 4-bit NF4 path on a Llama-7B-shaped stack.
+"""Benchmark of the 4-bit NF4 / FP4 path: the five workloads of the method's
+brief, each timed in isolation, inside one step.
 
-One step = one pass of the whole hot path over the 224 linears of a 32-layer
-Llama-7B-shaped stack (q/k/v/o 4096x4096, gate/up 11008x4096, down
-4096x11008; bf16 weights ~ N(0, 0.02^2) resident in HBM).  For every linear,
-in layer order:
-  1. quantize the bf16 weight to NF4, blocksize 64, with double quantization;
-  2. dequantize the packed weight back to bf16;
-  3. prefill GEMM: X bf16 [2048, K] ~ N(0, 1) times the 4-bit weight;
-  4. decode GEMV: x bf16 [1, K] ~ N(0, 1) times the 4-bit weight.
-``value`` is the stack's packed 4-bit weight bytes per step divided by the
-step time (GB/s), summed over ranks; per-row throughputs and roofline
-fractions are reported under ``rows``.  Inputs (12.95 GB of bf16 weights) are
-larger than L2, so no flush is needed between steps.
+One step runs, in this order, every row below; each row is a run of
+back-to-back calls of one kind on buffers that no other row touches, so a
+call never finds its inputs in L2 (every row's working set, and the 3.34 GB
+stack pass between two steps, evicts the others):
 
-Multi-GPU: every rank runs its own replica of the stack (independent
-problems, no collective on the data path); ``value`` counts all ranks.
+  cfg1  NF4 round trip of an fp32 vector of 2^20 elements ~ N(0, 0.02^2)
+        (seed 0), blocksize 64, double quant: quantize, then dequantize to
+        fp32 (8 calls each, over 8 copies);
+  cfg2  bf16 4096 x 4096 ~ N(0, 0.02^2) with 0.1% outliers x20, blocksize
+        64, double quant: quantize and dequantize to bf16, NF4 and FP4
+        (4 calls each, over 4 copies);
+  cfg3  decode GEMV, bf16 x [B, K] ~ N(0, 1), B in {1, 8}, NF4 weights
+        11008 x 4096 and 4096 x 11008 (4 calls each, over 4 weights);
+  cfg4  prefill GEMM, bf16 X [2048, K] ~ N(0, 1), the three Llama-7B shapes,
+        NF4 blocksize 64, NF4 blocksize 128 and FP4 blocksize 64;
+  cfg5  the 32-layer Llama-7B-shaped stack (q/k/v/o 4096x4096, gate/up
+        11008x4096, down 4096x11008; 6.48 B weights NF4-quantized with
+        double quant at set-up): batch-1 GEMV through all 224 linears.
 
-``--impl reference`` times the CPU oracle (single thread) on a bounded sample
-of the same workload instead.
+``value`` is configuration 5's figure: the bytes of the stack's 4-bit
+weights (codes, 8-bit scales and their scales, 3.341 GB) streamed per pass,
+divided by the pass time (GB/s), summed over ranks.  ``rows`` gives every
+row's time per call, throughput and fraction of the measured peak; the
+stack's quantization (set-up of configuration 5) is timed once as its own
+row.  The timed steps replay as one CUDA graph with CUDA events around every
+row.
+
+Multi-GPU: every rank runs its own replica (independent problems, no
+collective on the data path); ``value`` counts all ranks.
+
+``--impl reference`` times the CPU oracle (single thread) on a bounded
+sample of configuration 5 instead.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 """
 import argparse
+import hashlib
 import json
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -35,44 +52,55 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "4-bit GEMV weight-GB/s & GEMM TFLOPS; quant/dequant GB/s; % of roofline"
-WORKLOAD = ("llama7b-shaped stack, 32 layers x 7 linears (224): per linear "
-            "quantize bf16->NF4 (bs 64, double quant) + dequantize->bf16 + "
-            "prefill GEMM M=2048 + decode GEMV B=1")
+WORKLOAD = ("five workloads per step, each row isolated on its own buffers: "
+            "cfg1 NF4 round trip fp32 2^20; cfg2 NF4/FP4 quantize+dequantize bf16 "
+            "4096x4096 with outliers; cfg3 GEMV B=1,8 on 11008x4096 and 4096x11008; "
+            "cfg4 GEMM M=2048 on the three Llama-7B shapes, NF4 bs64/bs128, FP4; "
+            "cfg5 batch-1 GEMV through the 224 linears of a 32-layer "
+            "Llama-7B-shaped NF4 stack (value)")
 GEMM_M = 2048
 BS = 64
+ROUNDTRIP_COPIES = 8
+MATRIX_COPIES = 4
+GEMV_WEIGHTS = 4
 
-# DRAM bytes (read + write) per GEMM launch, averaged over the seven GEMMs of
-# one layer, from one ncu capture (profiles/gemm4_dram_traffic_llama7b_layer.md).
-# Reported only while the GEMM kernel's sources are the ones captured.
-GEMM_TRAFFIC_BYTES = 37468818
-GEMM_TRAFFIC_SOURCES = ("bit_blockwise_weight_nf4_b200/csrc/gemm.cu",
-                        "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
-                        "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh")
-GEMM_TRAFFIC_SHA256 = "82bff8b020a3a34fcf3c9d310104139b8333349765e4ae10d819569003c77780"
+# DRAM bytes (read + write) per launch of a kernel family, from one ncu
+# capture each, with the sources hashed at capture time: a figure is
+# reported only while the kernel's sources are the ones that were captured.
+TRAFFIC = {
+    "gemm": {"bytes": 37468818,
+             "launch": "one prefill GEMM launch, averaged over the seven Llama-7B linears",
+             "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemm.cu",
+                         "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
+                         "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
+             "sha256": "82bff8b020a3a34fcf3c9d310104139b8333349765e4ae10d819569003c77780"},
+}
 
 
-def gemm_traffic():
-    """Measured DRAM bytes per GEMM launch, or None when the kernel sources
-    changed since the capture."""
-    import hashlib
+def traffic_of(family):
+    """Measured DRAM bytes per launch of `family`, or None when unmeasured or
+    when its sources changed since the capture."""
+    t = TRAFFIC.get(family)
+    if t is None:
+        return None
     h = hashlib.sha256()
     try:
-        for p in GEMM_TRAFFIC_SOURCES:
+        for p in t["sources"]:
             with open(os.path.join(ROOT, p), "rb") as f:
                 h.update(f.read())
     except OSError:
         return None
-    return GEMM_TRAFFIC_BYTES if h.hexdigest() == GEMM_TRAFFIC_SHA256 else None
+    return t if h.hexdigest() == t["sha256"] else None
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=32,
-                    help="decoder layers in the stack (32 = the Llama-7B workload)")
+                    help="decoder layers of the configuration-5 stack (32 = Llama-7B)")
     ap.add_argument("--eager", action="store_true",
                     help="launch the timed steps one call at a time instead of "
                          "replaying them as one CUDA graph")
@@ -85,9 +113,12 @@ def load_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return p["hbm_gbs"], p["bf16_tflops"], p["bf16_tflops_sustained"], "measured"
-    except (OSError, KeyError, ValueError):
-        return 6650.0, 1590.0, 1400.0, "fallback"
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p["bf16_tflops_sustained"]),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError, TypeError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
 
 
 # ------------------------------------------------------------- distributed
@@ -132,10 +163,11 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, device_index):
+    def __init__(self, device_index, interval_ms=50):
         self.proc = None
         self.path = None
         self.dev = device_index
+        self.interval = interval_ms
 
     def start(self):
         try:
@@ -143,7 +175,7 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.interval)],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -151,7 +183,6 @@ class ClockSampler:
     def stop(self):
         if self.proc is None:
             return None
-        time.sleep(0.25)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -189,186 +220,324 @@ def physical_gpu_index(local):
     return local
 
 
-# ------------------------------------------------------------ workload
-def stack_linears(n_layers):
-    import synth
-    return synth.llama7b_stack(n_layers)
+def host_description():
+    model = platform.processor() or "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"nproc": os.cpu_count(), "cpu_model": model}
 
 
-def packed_bytes(N, K):
-    nb = N * K // BS
-    return N * K // 2 + nb + 4 * -(-nb // 256) + 4
+# ------------------------------------------------------- algorithmic work
+def state_bytes(n, bs=BS, dq=True):
+    """Bytes of a quantization state of n elements: packed codes, and the
+    8-bit scales with their fp32 group scales and offset (double quant) or
+    the fp32 absmax."""
+    nb = -(-n // bs)
+    if dq:
+        return (n + 1) // 2 + nb + 4 * -(-nb // 256) + 4
+    return (n + 1) // 2 + 4 * nb
 
 
-def build_stack(n_layers, device):
-    """Resident bf16 weights, their quantization states and the activations."""
+def quantize_bytes(n, elt, bs=BS):
+    """Algorithmic bytes of one quantize call: read the input, write the state."""
+    return elt * n + state_bytes(n, bs)
+
+
+def dequantize_bytes(n, elt_out, bs=BS):
+    return state_bytes(n, bs) + elt_out * n
+
+
+def gemv_bytes(N, K, B, bs=BS):
+    return state_bytes(N * K, bs) + 2 * B * K + 2 * B * N
+
+
+# ---------------------------------------------------------------- rows
+class Row:
+    """A timed row: `calls` (C-ABI launches, each a zero-argument callable
+    returning the status) run back to back on the current stream."""
+
+    def __init__(self, name, cfg, family, bound, work, calls, kernels_per_call, **extra):
+        self.name, self.cfg, self.family, self.bound = name, cfg, family, bound
+        self.work = work                      # algorithmic bytes or flops per call
+        self.calls = calls
+        self.kpc = kernels_per_call
+        self.extra = extra
+
+    def run(self):
+        for c in self.calls:
+            rc = c()
+            if rc != 0:
+                raise RuntimeError("%s: launch failed with status %d" % (self.name, rc))
+
+
+def build_rows(dev, n_layers):
+    """Every row's inputs, resident on `dev`, and the calls that time it.
+    Returns (rows, stack) where stack describes configuration 5."""
     import torch
     import synth
-    import bit_blockwise_weight_nf4_b200 as bnb4
-    lins = stack_linears(n_layers)
-    W, states = [], []
+    import bit_blockwise_weight_nf4_b200 as b
+    S = lambda: b._stream()
+    rows = []
+
+    def fresh(n, bs, qt):
+        return b.QuantState(n, bs, qt, True, dev)
+
+    # cfg1: NF4 round trip of a 2^20-element fp32 vector
+    n1 = synth.ROUNDTRIP_N
+    x1 = synth.normal_f32((n1,), seed=0, std=synth.WEIGHT_STD, device=dev)
+    xs1 = [x1.clone() for _ in range(ROUNDTRIP_COPIES)]
+    q1 = [fresh(n1, BS, b.NF4) for _ in xs1]
+    d1 = [b.quantize_4bit(x, BS, b.NF4, True) for x in xs1]   # read by the dequantize row
+    o1 = [torch.empty(n1, dtype=torch.float32, device=dev) for _ in xs1]
+    ws = b.workspace_for(q1[0])
+    wsp, wsn = ws.data_ptr(), ws.numel()
+
+    def qcall(x, st, dt):
+        c = st.cstruct()
+        return lambda: b.bnb_quantize_4bit(x.data_ptr(), dt, c, wsp, wsn, S())
+
+    def dcall(st, out, dt):
+        c = st.cstruct()
+        return lambda: b.bnb_dequantize_4bit(c, out.data_ptr(), dt, S())
+
+    rows.append(Row("cfg1_quantize", "cfg1", "quantize", "hbm", quantize_bytes(n1, 4),
+                    [qcall(x, s, b.F32) for x, s in zip(xs1, q1)], 2))
+    rows.append(Row("cfg1_dequantize", "cfg1", "dequantize", "hbm", dequantize_bytes(n1, 4),
+                    [dcall(s, o, b.F32) for s, o in zip(d1, o1)], 1))
+
+    # cfg2: bf16 4096 x 4096 with outliers, NF4 and FP4
+    R, C = synth.MATRIX_4096
+    n2 = R * C
+    w2 = synth.weight_bf16(R, C, seed=2, outlier_frac=synth.OUTLIER_FRAC, device=dev).view(-1)
+    for qname, qt in (("nf4", b.NF4), ("fp4", b.FP4)):
+        xs = [w2.clone() for _ in range(MATRIX_COPIES)]
+        qs = [fresh(n2, BS, qt) for _ in xs]
+        ds = [b.quantize_4bit(w2, BS, qt, True) for _ in xs]
+        os_ = [torch.empty(n2, dtype=torch.bfloat16, device=dev) for _ in xs]
+        rows.append(Row("cfg2_quantize_" + qname, "cfg2", "quantize", "hbm",
+                        quantize_bytes(n2, 2), [qcall(x, s, b.BF16) for x, s in zip(xs, qs)], 2))
+        rows.append(Row("cfg2_dequantize_" + qname, "cfg2", "dequantize", "hbm",
+                        dequantize_bytes(n2, 2), [dcall(s, o, b.BF16) for s, o in zip(ds, os_)],
+                        1))
+    del w2
+
+    # cfg3: decode GEMV
+    def gemv_call(x, st, N, y):
+        c = st.cstruct()
+        B, K = x.shape
+        return lambda: b.bnb_gemv_4bit(x.data_ptr(), B, K, c, N, y.data_ptr(), S())
+
+    for N, K in synth.GEMV_SHAPES:
+        for Bt in synth.GEMV_BATCHES:
+            x = synth.activations_bf16(Bt, K, seed=1, device=dev)
+            sts = []
+            for i in range(GEMV_WEIGHTS):
+                w = synth.weight_bf16(N, K, seed=300 + 10 * Bt + i, device=dev)
+                sts.append(b.quantize_4bit(w.view(-1), BS, b.NF4, True))
+                del w
+            y = torch.empty(Bt, N, dtype=torch.bfloat16, device=dev)
+            rows.append(Row("cfg3_gemv_b%d_%dx%d" % (Bt, N, K), "cfg3", "gemv", "hbm",
+                            gemv_bytes(N, K, Bt), [gemv_call(x, s, N, y) for s in sts], 1,
+                            weight_bytes=N * K // 2))
+
+    # cfg4: prefill GEMM
+    def gemm_call(X, st, N, Y):
+        c = st.cstruct()
+        M, K = X.shape
+        return lambda: b.bnb_gemm_4bit(X.data_ptr(), M, K, c, N, Y.data_ptr(), S())
+
+    Xs = {K: synth.activations_bf16(GEMM_M, K, seed=1, device=dev)
+          for K in (synth.HIDDEN, synth.FFN)}
+    for vname, bs, qt in (("nf4_bs64", 64, b.NF4), ("nf4_bs128", 128, b.NF4),
+                          ("fp4_bs64", 64, b.FP4)):
+        for N, K in synth.GEMM_SHAPES:
+            w = synth.weight_bf16(N, K, seed=400 + N + K, device=dev)
+            st = b.quantize_4bit(w.view(-1), bs, qt, True)
+            del w
+            Y = torch.empty(GEMM_M, N, dtype=torch.bfloat16, device=dev)
+            rows.append(Row("cfg4_gemm_%s_%dx%d" % (vname, N, K), "cfg4", "gemm", "tensor",
+                            2 * GEMM_M * N * K, [gemm_call(Xs[K], st, N, Y)], 1))
+
+    # cfg5: the Llama-7B-shaped stack, quantized at set-up (timed once)
+    lins = synth.llama7b_stack(n_layers)
+    names = [l.name for l in synth.llama7b_layer()]
+    states = []
+    qtime = 0.0
+    qwork = 0
     for layer, lin in lins:
-        idx = [l.name for l in synth.llama7b_layer()].index(lin.name)
-        w = synth.weight_bf16(lin.N, lin.K, seed=synth.stack_weight_seed(layer, idx),
-                              device=device)
-        W.append(w.view(-1))
-        states.append(bnb4.QuantState(lin.N * lin.K, BS, bnb4.NF4, True, device))
-    X = {K: synth.activations_bf16(GEMM_M, K, seed=11 + K, device=device)
-         for K in (synth.HIDDEN, synth.FFN)}
-    x = {K: synth.activations_bf16(1, K, seed=13 + K, device=device)
-         for K in (synth.HIDDEN, synth.FFN)}
-    return lins, W, states, X, x
+        w = synth.weight_bf16(lin.N, lin.K, seed=synth.stack_weight_seed(
+            layer, names.index(lin.name)), device=dev).view(-1)
+        st = fresh(lin.N * lin.K, BS, b.NF4)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        rc = b.bnb_quantize_4bit(w.data_ptr(), b.BF16, st.cstruct(), wsp, wsn, S())
+        e1.record()
+        if rc != 0:
+            raise RuntimeError("stack quantize failed with status %d" % rc)
+        torch.cuda.synchronize()
+        qtime += e0.elapsed_time(e1) * 1e-3
+        qwork += quantize_bytes(lin.N * lin.K, 2)
+        states.append(st)
+        del w
+    xk = {K: synth.activations_bf16(1, K, seed=1, device=dev) for K in (synth.HIDDEN, synth.FFN)}
+    ys = [torch.empty(1, lin.N, dtype=torch.bfloat16, device=dev) for _, lin in lins]
+    calls = [gemv_call(xk[lin.K], st, lin.N, y) for (_, lin), st, y in zip(lins, states, ys)]
+    stack_state = sum(state_bytes(lin.N * lin.K) for _, lin in lins)
+    stack_row = Row("cfg5_gemv_stack_pass", "cfg5", "gemv", "hbm",
+                    sum(gemv_bytes(lin.N, lin.K, 1) for _, lin in lins) / len(lins), calls, 1,
+                    weight_bytes=sum(lin.N * lin.K // 2 for _, lin in lins) / len(lins))
+    rows.append(stack_row)
+    stack = {"lins": lins, "states": states, "x": xk, "y": ys, "state_bytes": stack_state,
+             "row": stack_row, "quantize_s": qtime, "quantize_bytes": qwork}
+    return rows, stack
 
 
 class Step:
-    """All launches of one step on the current stream, with an event before
-    and after every row so row times are measured inside the timed region."""
+    """The rows of one step, with an event at every row boundary."""
 
-    ROWS = ("quantize", "dequantize", "gemm", "gemv")
-
-    def __init__(self, lins, W, states, X, x, device):
-        import torch
-        import bit_blockwise_weight_nf4_b200 as bnb4
-        self.bnb4 = bnb4
-        self.lins, self.W, self.states, self.X, self.x = lins, W, states, X, x
-        maxnk = max(l.N * l.K for _, l in lins)
-        maxn = max(l.N for _, l in lins)
-        self.deq = torch.empty(maxnk, dtype=torch.bfloat16, device=device)
-        self.Y = torch.empty(GEMM_M * maxn, dtype=torch.bfloat16, device=device)
-        self.y = [torch.empty(1, l.N, dtype=torch.bfloat16, device=device)
-                  for _, l in lins]
-        self.ws = bnb4.workspace_for(states[0])
-        self.launches_per_step = 5 * len(lins)  # quantize is 2 kernels
+    def __init__(self, rows):
+        self.rows = rows
 
     def new_events(self):
-        """Timing events of one step; `external` makes a record captured in a
-        CUDA graph a timed event-record node."""
         import torch
-        return [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)]
-                for _ in self.lins]
+        return [torch.cuda.Event(enable_timing=True, external=True)
+                for _ in range(len(self.rows) + 1)]
 
     def run(self, events=None):
-        b = self.bnb4
-        stream = b._stream()
-        timed = events is not None
-        for i, (_, lin) in enumerate(self.lins):
-            st = self.states[i]
-            ev = events[i] if timed else None
-            if timed:
-                ev[0].record()
-            rc = b.bnb_quantize_4bit(self.W[i].data_ptr(), b.BF16, st.cstruct(),
-                                     self.ws.data_ptr(), self.ws.numel(), stream)
-            if timed:
-                ev[1].record()
-            rc |= b.bnb_dequantize_4bit(st.cstruct(), self.deq.data_ptr(), b.BF16, stream)
-            if timed:
-                ev[2].record()
-            rc |= b.bnb_gemm_4bit(self.X[lin.K].data_ptr(), GEMM_M, lin.K, st.cstruct(),
-                                  lin.N, self.Y.data_ptr(), stream)
-            if timed:
-                ev[3].record()
-            rc |= b.bnb_gemv_4bit(self.x[lin.K].data_ptr(), 1, lin.K, st.cstruct(),
-                                  lin.N, self.y[i].data_ptr(), stream)
-            if timed:
-                ev[4].record()
-            if rc != 0:
-                raise RuntimeError("launch failed on linear %d" % i)
+        for i, r in enumerate(self.rows):
+            if events is not None:
+                events[i].record()
+            r.run()
+        if events is not None:
+            events[-1].record()
 
-    def row_times(self, events, t=None):
-        """Seconds spent per row over the steps of `events` (after a
-        synchronize), added to t."""
-        t = t if t is not None else dict.fromkeys(self.ROWS, 0.0)
-        for ev in events:
-            for j, r in enumerate(self.ROWS):
-                t[r] += ev[j].elapsed_time(ev[j + 1]) * 1e-3
-        return t
-
-
-def row_work(lins):
-    """Algorithmic bytes / flops of one step per row."""
-    q = dq = gv = gm = 0
-    wb = 0
-    for _, l in lins:
-        n = l.N * l.K
-        nb = n // BS
-        ng = -(-nb // 256)
-        state = n // 2 + nb + 4 * ng + 4
-        q += 2 * n + state + 4 * nb            # read bf16, write state + fp32 absmax
-        dq += state + 2 * n                   # read state, write bf16
-        gv += state + 2 * l.K + 2 * l.N       # read state + x, write y
-        gm += 2 * GEMM_M * l.N * l.K
-        wb += n // 2
-    return {"quantize": q, "dequantize": dq, "gemv": gv, "gemm": gm, "weight_bytes": wb}
+    def kernels(self):
+        return sum(r.kpc * len(r.calls) for r in self.rows)
 
 
 # ------------------------------------------------------------ CPU oracle
-def oracle_sample(budget_layers=1):
-    """Time the single-threaded CPU oracle on layer 0's seven linears:
-    quantize (bs 64, double quant) + dequantize to bf16 + GEMV B=1 in full,
-    GEMM on 8 sampled rows of X extrapolated to 2048 rows.  Returns the
-    4-bit weight GB/s of the full path and a description."""
-    import numpy as np
+def _oracle_stack_linear(layer, lin, names):
+    """(state bytes, seconds) of the oracle's GEMV of one stack linear:
+    dequantize to bf16 and the fp64 dot products, from the oracle's own
+    quantization (not timed)."""
     import oracle
     import synth
-    lins = stack_linears(budget_layers)
-    t_q = t_dq = t_gv = t_gm = 0.0
-    wbytes = 0
-    rows = 8
-    for layer, lin in lins:
-        idx = [l.name for l in synth.llama7b_layer()].index(lin.name)
-        Wb = synth.bf16_bits(synth.weight_bf16(
-            lin.N, lin.K, seed=synth.stack_weight_seed(layer, idx)).view(-1))
-        t0 = time.perf_counter()
-        st = oracle.quantize(Wb, BS, oracle.NF4, True)
-        t1 = time.perf_counter()
-        Wh = oracle.dequantize(st, oracle.BF16).reshape(lin.N, lin.K)
-        t2 = time.perf_counter()
-        x = synth.bf16_bits(synth.activations_bf16(1, lin.K, seed=13 + lin.K))
-        oracle.linear_ref(x, Wh)
-        t3 = time.perf_counter()
-        X = synth.bf16_bits(synth.activations_bf16(rows, lin.K, seed=11 + lin.K))
-        oracle.linear_ref(X, Wh)
-        t4 = time.perf_counter()
-        t_q += t1 - t0
-        t_dq += t2 - t1
-        t_gv += t3 - t2
-        t_gm += (t4 - t3) * GEMM_M / rows
-        wbytes += lin.N * lin.K // 2
-    total = t_q + t_dq + t_gv + t_gm
-    return {
-        "value": wbytes / total / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-        "sample": ("layer 0 of the stack (7 linears, %.3f GB packed): quantize + "
-                   "dequantize + GEMV B=1 timed in full, GEMM timed on %d of 2048 "
-                   "rows and extrapolated; measured %.1f s, extrapolated %.1f s"
-                   % (wbytes / 1e9, rows, t_q + t_dq + t_gv + t_gm * rows / GEMM_M,
-                      total)),
-        "rows_s": {"quantize": t_q, "dequantize": t_dq, "gemv": t_gv,
-                   "gemm_extrapolated": t_gm},
-    }
+    Wb = synth.bf16_bits(synth.weight_bf16(
+        lin.N, lin.K, seed=synth.stack_weight_seed(layer, names.index(lin.name))).view(-1))
+    st = oracle.quantize(Wb, BS, oracle.NF4, True)
+    x = synth.bf16_bits(synth.activations_bf16(1, lin.K, seed=1))
+    t0 = time.perf_counter()
+    Wh = oracle.dequantize(st, oracle.BF16).reshape(lin.N, lin.K)
+    oracle.linear_ref(x, Wh)
+    return state_bytes(lin.N * lin.K), time.perf_counter() - t0
+
+
+def oracle_baseline():
+    """The single-threaded CPU oracle timed on bounded samples of every
+    configuration; `value` is configuration 5's figure (state GB/s of the
+    GEMV pass) from layers 0 and 31, extrapolated x16."""
+    import oracle
+    import synth
+    per = {}
+    t0 = time.perf_counter()
+    # cfg1 in full
+    x1 = synth.normal_f32((synth.ROUNDTRIP_N,), seed=0, std=synth.WEIGHT_STD).numpy()
+    a = time.perf_counter()
+    st = oracle.quantize(x1, BS, oracle.NF4, True)
+    b_ = time.perf_counter()
+    oracle.dequantize(st, oracle.F32)
+    c = time.perf_counter()
+    per["cfg1_quantize_GB/s"] = quantize_bytes(x1.size, 4) / (b_ - a) / 1e9
+    per["cfg1_dequantize_GB/s"] = dequantize_bytes(x1.size, 4) / (c - b_) / 1e9
+    # cfg2 in full, NF4
+    R, C = synth.MATRIX_4096
+    w2 = synth.bf16_bits(synth.weight_bf16(R, C, seed=2, outlier_frac=synth.OUTLIER_FRAC)
+                         .view(-1))
+    a = time.perf_counter()
+    st2 = oracle.quantize(w2, BS, oracle.NF4, True)
+    b_ = time.perf_counter()
+    oracle.dequantize(st2, oracle.BF16)
+    c = time.perf_counter()
+    per["cfg2_quantize_nf4_GB/s"] = quantize_bytes(R * C, 2) / (b_ - a) / 1e9
+    per["cfg2_dequantize_nf4_GB/s"] = dequantize_bytes(R * C, 2) / (c - b_) / 1e9
+    # cfg3: B = 8 on 11008 x 4096 in full (dequantize + fp64 dot products)
+    N, K = synth.GEMV_SHAPES[0]
+    wb = synth.bf16_bits(synth.weight_bf16(N, K, seed=300).view(-1))
+    st3 = oracle.quantize(wb, BS, oracle.NF4, True)
+    x8 = synth.bf16_bits(synth.activations_bf16(8, K, seed=1))
+    a = time.perf_counter()
+    Wh = oracle.dequantize(st3, oracle.BF16).reshape(N, K)
+    oracle.linear_ref(x8, Wh)
+    per["cfg3_gemv_b8_%dx%d_GB/s" % (N, K)] = gemv_bytes(N, K, 8) / (time.perf_counter() - a) / 1e9
+    # cfg4: 8 of 2048 rows of the 4096 x 4096 GEMM, extrapolated
+    X = synth.bf16_bits(synth.activations_bf16(8, K, seed=1))
+    Wq = Wh[:synth.HIDDEN]
+    a = time.perf_counter()
+    oracle.linear_ref(X, Wq)
+    t8 = time.perf_counter() - a
+    per["cfg4_gemm_4096x4096_TFLOP/s_extrapolated"] = \
+        2 * GEMM_M * synth.HIDDEN * K / (t8 * GEMM_M / 8) / 1e12
+    # cfg5: layers 0 and 31, extrapolated x16
+    names = [l.name for l in synth.llama7b_layer()]
+    sb = st_s = 0.0
+    for layer in (0, synth.N_LAYERS - 1):
+        for lin in synth.llama7b_layer():
+            nb, s = _oracle_stack_linear(layer, lin, names)
+            sb += nb
+            st_s += s
+    v = sb / st_s / 1e9
+    wall = time.perf_counter() - t0
+    return dict({
+        "value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
+        "sample": ("configuration 5 (GEMV pass, bytes of the 4-bit weight state per "
+                   "second): the oracle's dequantize + fp64 dot products on layers 0 and 31 "
+                   "(14 linears, %.3f GB), extrapolated x16; also cfg1 and cfg2 (NF4) in "
+                   "full, cfg3 B=8 on 11008x4096 in full, cfg4 on 8 of 2048 rows "
+                   "(extrapolated); %.1f s of CPU work in all" % (sb / 1e9, wall)),
+        "per_config": per,
+    }, **host_description())
 
 
 def run_reference(args):
+    """The oracle as the reference arm: each step is one linear of layers 0
+    and 31 of the configuration-5 stack (dequantize + fp64 dot products),
+    cycling; value = state bytes per second over the steps."""
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
-    samples = []
-    for _ in range(args.warmup):
-        pass  # the oracle has no warm-up effects worth timing separately
+    import synth
+    names = [l.name for l in synth.llama7b_layer()]
+    sample = [(layer, lin) for layer in (0, synth.N_LAYERS - 1)
+              for lin in synth.llama7b_layer()]
+    for i in range(args.warmup):
+        _oracle_stack_linear(*sample[i % len(sample)], names)
+    tot_b = tot_s = 0.0
     t0 = time.perf_counter()
-    for _ in range(max(1, args.steps)):
-        samples.append(oracle_sample())
+    for i in range(max(1, args.steps)):
+        nb, s = _oracle_stack_linear(*sample[i % len(sample)], names)
+        tot_b += nb
+        tot_s += s
     wall = time.perf_counter() - t0
-    v = statistics.median(s["value"] for s in samples)
-    cb = dict(samples[0], value=v)
-    cb.pop("rows_s", None)
+    v = tot_b / tot_s / 1e9
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": wall / max(1, args.steps) * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64/f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD + " (CPU oracle, bounded sample per step)"},
-        "cpu_baseline": cb,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "configuration 5 (batch-1 GEMV through the Llama-7B-shaped "
+                               "NF4 stack), CPU oracle, one linear of layers 0 / 31 per step"},
+        "cpu_baseline": dict({"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                              "sample": "one linear of layers 0 / 31 per step, cycling "
+                                        "(%d steps)" % max(1, args.steps)},
+                             **host_description()),
         "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -382,14 +551,14 @@ def run_ours(args):
     bnb4.load()
     rank, world, local = dist_init()
     dev = torch.device("cuda", local)
-    hbm, tf_burst, tf_sus, peak_src = load_peaks()
+    peaks = load_peaks()
 
-    lins, W, states, X, x = build_stack(args.layers, dev)
-    step = Step(lins, W, states, X, x, dev)
-    work = row_work(lins)
+    rows, stack = build_rows(dev, args.layers)
+    step = Step(rows)
     torch.cuda.synchronize()
 
-    for _ in range(max(3, args.warmup)):
+    warm = max(3, args.warmup)
+    for _ in range(warm):
         step.run()
     torch.cuda.synchronize()
     if bnb4.bnb4_device_status(torch.cuda.current_stream().cuda_stream) != 0:
@@ -398,7 +567,7 @@ def run_ours(args):
     events = [step.new_events() for _ in range(args.steps)]
     graph = None
     if not args.eager:
-        # the K timed steps (every launch and the per-row events) as one CUDA
+        # the K timed steps (every launch and the row events) as one CUDA
         # graph: the same kernels on the same buffers, without per-call host
         # launch overhead between them
         graph = torch.cuda.CUDAGraph()
@@ -412,6 +581,7 @@ def run_ours(args):
         torch.cuda.synchronize()
     clocks = ClockSampler(physical_gpu_index(local))
     clocks.start()
+    time.sleep(0.1)
     barrier(world)
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
@@ -427,67 +597,100 @@ def run_ours(args):
     barrier(world)
     elapsed = t_start.elapsed_time(t_end) * 1e-3
     clk = clocks.stop()
-    rows_t = None
-    for ev in events:
-        rows_t = step.row_times(ev, rows_t)
-    rows_t = {k: v / args.steps for k, v in rows_t.items()}  # per step
-    elapsed_max = max_over_ranks(elapsed, world)
     status = bnb4.bnb4_device_status(torch.cuda.current_stream().cuda_stream)
     if status != 0:
         raise RuntimeError("device error word set: %s" % bnb4.bnb4_strerror(status))
 
-    value = world * work["weight_bytes"] * args.steps / elapsed_max / 1e9
-    n_gemm = len(lins)
-    gemm_tflops = work["gemm"] / rows_t["gemm"] / 1e12
-    rows = {
-        "quantize": {"GB/s": work["quantize"] / rows_t["quantize"] / 1e9,
-                     "frac_hbm": work["quantize"] / rows_t["quantize"] / 1e9 / hbm,
-                     "ms": rows_t["quantize"] * 1e3},
-        "dequantize": {"GB/s": work["dequantize"] / rows_t["dequantize"] / 1e9,
-                       "frac_hbm": work["dequantize"] / rows_t["dequantize"] / 1e9 / hbm,
-                       "ms": rows_t["dequantize"] * 1e3},
-        "gemv_b1": {"weight_GB/s": work["weight_bytes"] / rows_t["gemv"] / 1e9,
-                    "GB/s": work["gemv"] / rows_t["gemv"] / 1e9,
-                    "frac_hbm": work["gemv"] / rows_t["gemv"] / 1e9 / hbm,
-                    "ms": rows_t["gemv"] * 1e3},
-        "gemm_m2048": {"TFLOP/s": gemm_tflops, "frac_bf16_sustained": gemm_tflops / tf_sus,
-                       "frac_bf16_burst": gemm_tflops / tf_burst,
-                       "ms": rows_t["gemm"] * 1e3},
+    # seconds per call of every row, averaged over the timed steps
+    per_call = {}
+    for i, r in enumerate(rows):
+        t = sum(ev[i].elapsed_time(ev[i + 1]) for ev in events) * 1e-3 / args.steps
+        per_call[r.name] = t / len(r.calls)
+    srow = stack["row"]
+    t_pass = max_over_ranks(per_call[srow.name] * len(srow.calls), world)
+    elapsed_max = max_over_ranks(elapsed, world)
+    value = world * stack["state_bytes"] / t_pass / 1e9
+
+    # burst peaks for rows timed at boost clocks, sustained below them
+    burst = clk is None or clk["sm_mhz"] >= 0.9 * clk["sm_max_mhz"]
+    tf_peak = peaks["bf16_tflops"] if burst else peaks["bf16_tflops_sustained"]
+    tf_kind = "bf16 burst" if burst else "bf16 sustained"
+    out_rows = {}
+    for r in rows:
+        t = per_call[r.name]
+        d = {"config": r.cfg, "kernel_family": r.family, "calls_per_step": len(r.calls),
+             "us_per_call": t * 1e6}
+        if r.bound == "tensor":
+            a = r.work / t / 1e12
+            d.update({"TFLOP/s": a, "frac_bf16_burst": a / peaks["bf16_tflops"],
+                      "frac_bf16_sustained": a / peaks["bf16_tflops_sustained"]})
+        else:
+            a = r.work / t / 1e9
+            d.update({"GB/s": a, "frac_hbm": a / peaks["hbm_gbs"]})
+            if "weight_bytes" in r.extra:
+                d["weight_GB/s"] = r.extra["weight_bytes"] / t / 1e9
+        out_rows[r.name] = d
+    out_rows[srow.name].update({
+        "ms_per_pass": t_pass * 1e3, "state_bytes_per_pass": stack["state_bytes"],
+        "target_ms_at_70pct_hbm": stack["state_bytes"] / (0.7 * peaks["hbm_gbs"] * 1e9) * 1e3})
+    out_rows["cfg5_quantize_stack_setup"] = {
+        "config": "cfg5", "kernel_family": "quantize", "calls": len(stack["lins"]),
+        "note": "set-up of configuration 5, timed once call by call (not in the step)",
+        "GB/s": stack["quantize_bytes"] / stack["quantize_s"] / 1e9,
+        "frac_hbm": stack["quantize_bytes"] / stack["quantize_s"] / 1e9 / peaks["hbm_gbs"],
+        "ms": stack["quantize_s"] * 1e3}
+
+    # the kernel family with the most time per step
+    fam = {}
+    for r in rows:
+        f = fam.setdefault(r.family, {"s": 0.0, "work": 0.0, "launches": 0, "bound": r.bound})
+        f["s"] += per_call[r.name] * len(r.calls)
+        f["work"] += r.work * len(r.calls)
+        f["launches"] += len(r.calls)
+    dom_name = max(fam, key=lambda k: fam[k]["s"])
+    dom = fam[dom_name]
+    tr = traffic_of(dom_name)
+    if dom["bound"] == "tensor":
+        ach, peak, unit = dom["work"] / dom["s"] / 1e12, tf_peak, "TFLOP/s"
+        psrc = "%s %s" % (peaks["source"], tf_kind)
+    else:
+        ach, peak, unit = dom["work"] / dom["s"] / 1e9, peaks["hbm_gbs"], "GB/s"
+        psrc = "%s HBM copy bandwidth" % peaks["source"]
+    roofline = {
+        "bound": dom["bound"], "kernel": dom_name, "achieved": ach, "peak": peak,
+        "unit": unit, "frac": ach / peak, "traffic": tr["bytes"] if tr else None,
+        "traffic_launch": tr["launch"] if tr else None,
+        "peak_source": psrc,
+        "per_launch": "algorithmic work of the %d launches per step of this family "
+                      "over their summed event time" % dom["launches"],
+        "share_of_step": dom["s"] / (elapsed_max / args.steps),
     }
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
-        "steps": args.steps, "warmup": max(3, args.warmup),
+        "steps": args.steps, "warmup": warm,
         "ms_per_step": elapsed_max / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "layers": args.layers, "linears": len(lins),
-                   "weight_format": "nf4, blocksize 64, double quant",
-                   "packed_weight_bytes": work["weight_bytes"],
-                   "gemm_m": GEMM_M, "gemv_batch": 1,
-                   "l2": "inputs larger than L2 (%.2f GB of bf16 weights), no flush"
-                         % (sum(w.numel() * 2 for w in W) / 1e9),
+        "config": {"workload": WORKLOAD, "layers": args.layers,
+                   "value": "configuration 5: 4-bit weight state bytes of the stack "
+                            "(codes + 8-bit scales + group scales, %.3f GB) per GEMV pass "
+                            "time" % (stack["state_bytes"] / 1e9),
+                   "weight_format": "nf4 unless named, blocksize 64 unless named, double quant",
+                   "l2": "no flush: every row runs on its own buffers, each call on a "
+                         "different copy, and the 3.34 GB stack pass evicts L2 between steps",
                    "parallelism": "replicas x%d" % world,
                    "launch": "eager, one call per kernel" if args.eager
                              else "the timed steps replayed as one CUDA graph"},
-        "roofline": {"bound": "tensor", "kernel": "gemm4 (fused dequant + tcgen05)",
-                     "achieved": gemm_tflops, "peak": tf_sus, "unit": "TFLOP/s",
-                     "frac": gemm_tflops / tf_sus, "traffic": gemm_traffic(),
-                     "traffic_unit": "bytes per launch (dram read + write, ncu)",
-                     "peak_source": "%s bf16 sustained (kernel inside a long step)"
-                                    % peak_src,
-                     "per_launch": "2*2048*N*K flops; %d launches per step" % n_gemm},
-        "rows": rows,
-        "gpu_launches": step.launches_per_step * args.steps,
+        "roofline": roofline,
+        "rows": out_rows,
+        "gpu_launches": step.kernels() * args.steps,
         "clocks": clk,
-        "peaks": {"hbm_gbs": hbm, "bf16_tflops": tf_burst,
-                  "bf16_tflops_sustained": tf_sus, "source": peak_src},
+        "peaks": peaks,
     }
     del graph
     if not args.no_e2e:
-        line["e2e"] = run_e2e(step, W, X, x, lins, world, args)
+        line["e2e"] = run_e2e(stack, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = oracle_sample()
-        cb.pop("rows_s", None)
-        line["cpu_baseline"] = cb
+        line["cpu_baseline"] = oracle_baseline()
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
@@ -495,29 +698,26 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_e2e(step, W, X, x, lins, world, args):
-    """Same step through the C ABI with the inputs in pinned HOST memory:
-    every step copies the bf16 weights and activations host->device and reads
-    the decode outputs back, all inside the timed region."""
+def run_e2e(stack, world, steps=10):
+    """Configuration 5 through the public Python API, eager, with the
+    activations coming from page-locked HOST memory and every output read
+    back: per step, copy x in, call gemv_4bit for each of the 224 linears,
+    copy the 224 outputs out -- all inside the timed region."""
     import torch
-    host_W = [w.cpu().pin_memory() for w in W]
-    host_X = {k: v.cpu().pin_memory() for k, v in X.items()}
-    host_x = {k: v.cpu().pin_memory() for k, v in x.items()}
-    host_y = [y.cpu().pin_memory() for y in step.y]
-    h2d = sum(t.numel() * 2 for t in host_W) + sum(t.numel() * 2 for t in host_X.values()) \
-        + sum(t.numel() * 2 for t in host_x.values())
+    import bit_blockwise_weight_nf4_b200 as bnb4
+    xs = stack["x"]
+    host_x = {k: v.cpu().pin_memory() for k, v in xs.items()}
+    host_y = [y.cpu().pin_memory() for y in stack["y"]]
+    h2d = sum(t.numel() * 2 for t in host_x.values())
     d2h = sum(t.numel() * 2 for t in host_y)
-    k_e2e = max(1, min(args.steps, 3))
 
     def one():
-        for d, h in zip(W, host_W):
-            d.copy_(h, non_blocking=True)
-        for k in X:
-            X[k].copy_(host_X[k], non_blocking=True)
-            x[k].copy_(host_x[k], non_blocking=True)
-        step.run()
-        for h, d in zip(host_y, step.y):
-            h.copy_(d, non_blocking=True)
+        for k in xs:
+            xs[k].copy_(host_x[k], non_blocking=True)
+        for (_, lin), st, y in zip(stack["lins"], stack["states"], stack["y"]):
+            bnb4.gemv_4bit(xs[lin.K], st, lin.N, out=y)
+        for h, y in zip(host_y, stack["y"]):
+            h.copy_(y, non_blocking=True)
 
     one()
     torch.cuda.synchronize()
@@ -525,16 +725,16 @@ def run_e2e(step, W, X, x, lins, world, args):
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record()
-    for _ in range(k_e2e):
+    for _ in range(steps):
         one()
     b.record()
     torch.cuda.synchronize()
     barrier(world)
     t = max_over_ranks(a.elapsed_time(b) * 1e-3, world)
-    wbytes = sum(l.N * l.K // 2 for _, l in lins)
-    return {"value": world * wbytes * k_e2e / t / 1e9, "unit": "GB/s",
+    return {"value": world * stack["state_bytes"] * steps / t / 1e9, "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": k_e2e, "ms_per_step": t / k_e2e * 1e3}
+            "steps": steps, "ms_per_step": t / steps * 1e3,
+            "path": "gemv_4bit (Python binding -> C ABI), one call per linear, eager"}
 
 
 def main():
