@@ -19,11 +19,15 @@ stack pass between two steps, evicts the others):
         NF4 blocksize 64, NF4 blocksize 128 and FP4 blocksize 64;
   cfg5  the 32-layer Llama-7B-shaped stack (q/k/v/o 4096x4096, gate/up
         11008x4096, down 4096x11008; 6.48 B weights NF4-quantized with
-        double quant at set-up): batch-1 GEMV through all 224 linears.
+        double quant at set-up): batch-1 GEMV through all 224 linears, as a
+        decoder launches them (per layer: q/k/v in one grouped launch, o,
+        gate/up in one grouped launch, down: 128 launches), and for
+        comparison as 224 single calls and as two grouped calls (one per K).
 
 ``value`` is configuration 5's figure: the bytes of the stack's 4-bit
-weights (codes, 8-bit scales and their scales, 3.341 GB) streamed per pass,
-divided by the pass time (GB/s), summed over ranks.  ``rows`` gives every
+weights (codes, 8-bit scales and their scales, 3.341 GB) streamed per pass
+of the per-layer launches, divided by the pass time (GB/s), summed over
+ranks.  ``rows`` gives every
 row's time per call, throughput and fraction of the measured peak; the
 stack's quantization (set-up of configuration 5) is timed once as its own
 row.  The timed steps replay as one CUDA graph with CUDA events around every
@@ -57,7 +61,7 @@ WORKLOAD = ("five workloads per step, each row isolated on its own buffers: "
             "4096x4096 with outliers; cfg3 GEMV B=1,8 on 11008x4096 and 4096x11008; "
             "cfg4 GEMM M=2048 on the three Llama-7B shapes, NF4 bs64/bs128, FP4; "
             "cfg5 batch-1 GEMV through the 224 linears of a 32-layer "
-            "Llama-7B-shaped NF4 stack (value)")
+            "Llama-7B-shaped NF4 stack, per-layer launches (value)")
 GEMM_M = 2048
 BS = 64
 ROUNDTRIP_COPIES = 8
@@ -258,6 +262,20 @@ def gemv_bytes(N, K, B, bs=BS):
 
 
 # ---------------------------------------------------------------- rows
+class Call:
+    """One C-ABI launch: the entry point, its arguments (raw pointers) and
+    the tensors those pointers point into, held for as long as the call may
+    run; the stream is torch's current one at call time (the capture stream
+    while a graph is being captured)."""
+
+    def __init__(self, fn, *args, keep=()):
+        self.fn, self.args, self.keep = fn, args, keep
+
+    def __call__(self):
+        import bit_blockwise_weight_nf4_b200 as b
+        return self.fn(*self.args, b._stream())
+
+
 class Row:
     """A timed row: `calls` (C-ABI launches, each a zero-argument callable
     returning the status) run back to back on the current stream."""
@@ -296,15 +314,14 @@ def build_rows(dev, n_layers):
     d1 = [b.quantize_4bit(x, BS, b.NF4, True) for x in xs1]   # read by the dequantize row
     o1 = [torch.empty(n1, dtype=torch.float32, device=dev) for _ in xs1]
     ws = b.workspace_for(q1[0])
-    wsp, wsn = ws.data_ptr(), ws.numel()
+    wsn = ws.numel()
 
     def qcall(x, st, dt):
-        c = st.cstruct()
-        return lambda: b.bnb_quantize_4bit(x.data_ptr(), dt, c, wsp, wsn, S())
+        return Call(b.bnb_quantize_4bit, x.data_ptr(), dt, st.cstruct(), ws.data_ptr(), wsn,
+                    keep=(x, st, ws))
 
     def dcall(st, out, dt):
-        c = st.cstruct()
-        return lambda: b.bnb_dequantize_4bit(c, out.data_ptr(), dt, S())
+        return Call(b.bnb_dequantize_4bit, st.cstruct(), out.data_ptr(), dt, keep=(st, out))
 
     rows.append(Row("cfg1_quantize", "cfg1", "quantize", "hbm", quantize_bytes(n1, 4),
                     [qcall(x, s, b.F32) for x, s in zip(xs1, q1)], 2))
@@ -329,9 +346,9 @@ def build_rows(dev, n_layers):
 
     # cfg3: decode GEMV
     def gemv_call(x, st, N, y):
-        c = st.cstruct()
         B, K = x.shape
-        return lambda: b.bnb_gemv_4bit(x.data_ptr(), B, K, c, N, y.data_ptr(), S())
+        return Call(b.bnb_gemv_4bit, x.data_ptr(), B, K, st.cstruct(), N, y.data_ptr(),
+                    keep=(x, st, y))
 
     for N, K in synth.GEMV_SHAPES:
         for Bt in synth.GEMV_BATCHES:
@@ -348,9 +365,9 @@ def build_rows(dev, n_layers):
 
     # cfg4: prefill GEMM
     def gemm_call(X, st, N, Y):
-        c = st.cstruct()
         M, K = X.shape
-        return lambda: b.bnb_gemm_4bit(X.data_ptr(), M, K, c, N, Y.data_ptr(), S())
+        return Call(b.bnb_gemm_4bit, X.data_ptr(), M, K, st.cstruct(), N, Y.data_ptr(),
+                    keep=(X, st, Y))
 
     Xs = {K: synth.activations_bf16(GEMM_M, K, seed=1, device=dev)
           for K in (synth.HIDDEN, synth.FFN)}
@@ -377,7 +394,7 @@ def build_rows(dev, n_layers):
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        rc = b.bnb_quantize_4bit(w.data_ptr(), b.BF16, st.cstruct(), wsp, wsn, S())
+        rc = b.bnb_quantize_4bit(w.data_ptr(), b.BF16, st.cstruct(), ws.data_ptr(), wsn, S())
         e1.record()
         if rc != 0:
             raise RuntimeError("stack quantize failed with status %d" % rc)
@@ -388,14 +405,45 @@ def build_rows(dev, n_layers):
         del w
     xk = {K: synth.activations_bf16(1, K, seed=1, device=dev) for K in (synth.HIDDEN, synth.FFN)}
     ys = [torch.empty(1, lin.N, dtype=torch.bfloat16, device=dev) for _, lin in lins]
-    calls = [gemv_call(xk[lin.K], st, lin.N, y) for (_, lin), st, y in zip(lins, states, ys)]
     stack_state = sum(state_bytes(lin.N * lin.K) for _, lin in lins)
-    stack_row = Row("cfg5_gemv_stack_pass", "cfg5", "gemv", "hbm",
-                    sum(gemv_bytes(lin.N, lin.K, 1) for _, lin in lins) / len(lins), calls, 1,
-                    weight_bytes=sum(lin.N * lin.K // 2 for _, lin in lins) / len(lins))
+    pass_bytes = sum(gemv_bytes(lin.N, lin.K, 1) for _, lin in lins)
+    pass_weights = sum(lin.N * lin.K // 2 for _, lin in lins)
+
+    def group_call(idx):
+        probs = (b.GemvProblem * len(idx))()
+        for j, i in enumerate(idx):
+            lin = lins[i][1]
+            probs[j] = b.GemvProblem(xk[lin.K].data_ptr(), states[i].cstruct(), lin.K, lin.N,
+                                     None, ys[i].data_ptr())
+        return Call(b.bnb_gemv_4bit_grouped, probs, 1, b.BF16,
+                    keep=[states[i] for i in idx] + [ys[i] for i in idx] + list(xk.values()))
+
+    # the decoder's natural launches per layer: q/k/v (one input), o,
+    # gate/up (one input), down
+    layer_groups = []
+    for L in range(n_layers):
+        base = 7 * L
+        layer_groups += [[base, base + 1, base + 2], [base + 3], [base + 4, base + 5],
+                         [base + 6]]
+
+    def pass_row(name, calls):
+        return Row(name, "cfg5", "gemv", "hbm", pass_bytes / len(calls), calls, 1,
+                   weight_bytes=pass_weights / len(calls))
+
+    stack_row = pass_row("cfg5_gemv_stack_layer_groups", [group_call(g) for g in layer_groups])
     rows.append(stack_row)
+    rows.append(pass_row("cfg5_gemv_stack_single_calls",
+                         [gemv_call(xk[lin.K], st, lin.N, y)
+                          for (_, lin), st, y in zip(lins, states, ys)]))
+    # the whole list in as few calls as the one-K rule allows: every linear
+    # with K = 4096 in one call, every K = 11008 one in another
+    by_k = {}
+    for i, (_, lin) in enumerate(lins):
+        by_k.setdefault(lin.K, []).append(i)
+    rows.append(pass_row("cfg5_gemv_stack_by_k", [group_call(ix) for ix in by_k.values()]))
     stack = {"lins": lins, "states": states, "x": xk, "y": ys, "state_bytes": stack_state,
-             "row": stack_row, "quantize_s": qtime, "quantize_bytes": qwork}
+             "row": stack_row, "groups": layer_groups, "quantize_s": qtime,
+             "quantize_bytes": qwork}
     return rows, stack
 
 
@@ -630,9 +678,15 @@ def run_ours(args):
             if "weight_bytes" in r.extra:
                 d["weight_GB/s"] = r.extra["weight_bytes"] / t / 1e9
         out_rows[r.name] = d
-    out_rows[srow.name].update({
-        "ms_per_pass": t_pass * 1e3, "state_bytes_per_pass": stack["state_bytes"],
-        "target_ms_at_70pct_hbm": stack["state_bytes"] / (0.7 * peaks["hbm_gbs"] * 1e9) * 1e3})
+    for r in rows:
+        if r.cfg == "cfg5":
+            t = per_call[r.name] * len(r.calls)
+            out_rows[r.name].update({
+                "ms_per_pass": t * 1e3, "launches_per_pass": len(r.calls),
+                "state_GB/s": stack["state_bytes"] / t / 1e9,
+                "state_bytes_per_pass": stack["state_bytes"],
+                "target_ms_at_70pct_hbm":
+                    stack["state_bytes"] / (0.7 * peaks["hbm_gbs"] * 1e9) * 1e3})
     out_rows["cfg5_quantize_stack_setup"] = {
         "config": "cfg5", "kernel_family": "quantize", "calls": len(stack["lins"]),
         "note": "set-up of configuration 5, timed once call by call (not in the step)",
@@ -673,7 +727,8 @@ def run_ours(args):
         "config": {"workload": WORKLOAD, "layers": args.layers,
                    "value": "configuration 5: 4-bit weight state bytes of the stack "
                             "(codes + 8-bit scales + group scales, %.3f GB) per GEMV pass "
-                            "time" % (stack["state_bytes"] / 1e9),
+                            "time, 4 launches per layer (q/k/v grouped, o, gate/up grouped, "
+                            "down)" % (stack["state_bytes"] / 1e9),
                    "weight_format": "nf4 unless named, blocksize 64 unless named, double quant",
                    "l2": "no flush: every row runs on its own buffers, each call on a "
                          "different copy, and the 3.34 GB stack pass evicts L2 between steps",
@@ -701,8 +756,8 @@ def run_ours(args):
 def run_e2e(stack, world, steps=10):
     """Configuration 5 through the public Python API, eager, with the
     activations coming from page-locked HOST memory and every output read
-    back: per step, copy x in, call gemv_4bit for each of the 224 linears,
-    copy the 224 outputs out -- all inside the timed region."""
+    back: per step, copy x in, make the pass's 128 grouped calls, copy the
+    224 outputs out -- all inside the timed region."""
     import torch
     import bit_blockwise_weight_nf4_b200 as bnb4
     xs = stack["x"]
@@ -711,12 +766,15 @@ def run_e2e(stack, world, steps=10):
     h2d = sum(t.numel() * 2 for t in host_x.values())
     d2h = sum(t.numel() * 2 for t in host_y)
 
+    lins, states, ys = stack["lins"], stack["states"], stack["y"]
+
     def one():
         for k in xs:
             xs[k].copy_(host_x[k], non_blocking=True)
-        for (_, lin), st, y in zip(stack["lins"], stack["states"], stack["y"]):
-            bnb4.gemv_4bit(xs[lin.K], st, lin.N, out=y)
-        for h, y in zip(host_y, stack["y"]):
+        for grp in stack["groups"]:
+            bnb4.gemv_4bit_grouped([(xs[lins[i][1].K], states[i], lins[i][1].N) for i in grp],
+                                   outs=[ys[i] for i in grp])
+        for h, y in zip(host_y, ys):
             h.copy_(y, non_blocking=True)
 
     one()
@@ -734,7 +792,8 @@ def run_e2e(stack, world, steps=10):
     return {"value": world * stack["state_bytes"] * steps / t / 1e9, "unit": "GB/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "steps": steps, "ms_per_step": t / steps * 1e3,
-            "path": "gemv_4bit (Python binding -> C ABI), one call per linear, eager"}
+            "path": "gemv_4bit_grouped (Python binding -> C ABI), 4 calls per layer "
+                    "as in the timed pass, eager"}
 
 
 def main():

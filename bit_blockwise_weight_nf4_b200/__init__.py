@@ -4,11 +4,13 @@ Two layers, both argument marshalling only -- every step of the
 quantize / dequantize / GEMV / GEMM path runs in the CUDA library:
 
 * raw ctypes entry points with the C names (``bnb_quantize_4bit``,
-  ``bnb_quantize_4bit_noalloc``, ``bnb_dequantize_4bit``, ``bnb_gemv_4bit``, ``bnb_gemm_4bit``,
+  ``bnb_quantize_4bit_noalloc``, ``bnb_dequantize_4bit``, ``bnb_gemv_4bit``,
+  ``bnb_gemv_4bit_grouped``, ``bnb_gemm_4bit``,
   ``bnb_linear_4bit``, ``bnb4_query_sizes``, ``bnb4_device_status``,
   ``bnb4_strerror``, ``bnb4_abi_version``), returning the C status;
 * torch helpers (``QuantState``, ``quantize_4bit``, ``dequantize_4bit``,
-  ``gemv_4bit``, ``gemm_4bit``, ``linear_4bit``) that allocate device buffers
+  ``gemv_4bit``, ``gemv_4bit_grouped``, ``gemm_4bit``, ``linear_4bit``) that
+  allocate device buffers
   with torch, call the entry points on torch's current stream and raise
   ``Bnb4Error`` on a non-zero status.
 
@@ -39,7 +41,8 @@ F32 = 0
 BF16 = 1
 F16 = 2
 
-ABI_VERSION = 2
+ABI_VERSION = 3
+GROUP_MAX = 256
 
 
 class QState(ctypes.Structure):
@@ -49,6 +52,12 @@ class QState(ctypes.Structure):
                 ("offset", ctypes.c_void_p), ("n", ctypes.c_int64),
                 ("blocksize", ctypes.c_int32), ("qtype", ctypes.c_int32),
                 ("double_quant", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class GemvProblem(ctypes.Structure):
+    """``bnb4_gemv_problem``: one linear of a grouped decode launch."""
+    _fields_ = [("x", ctypes.c_void_p), ("W", QState), ("K", ctypes.c_int64),
+                ("N", ctypes.c_int64), ("bias", ctypes.c_void_p), ("y", ctypes.c_void_p)]
 
 
 class Sizes(ctypes.Structure):
@@ -89,6 +98,8 @@ def load():
         "bnb_dequantize_4bit_2d": ([QP, p, i32, i64, i64, i64, p], ctypes.c_int),
         "bnb_gemv_4bit": ([p, i64, i64, QP, i64, p, p], ctypes.c_int),
         "bnb_gemm_4bit": ([p, i64, i64, QP, i64, p, p], ctypes.c_int),
+        "bnb_gemv_4bit_grouped": ([ctypes.POINTER(GemvProblem), i32, i64, i32, p],
+                                  ctypes.c_int),
         "bnb_linear_4bit": ([p, i32, i64, i64, QP, i64, p, p, p], ctypes.c_int),
         "bnb4_device_status": ([p, i32], ctypes.c_int),
         "bnb4_debug_gemm_withhold": ([p, i64, i64, QP, i64, p, i32, p], ctypes.c_int),
@@ -154,6 +165,13 @@ def bnb_gemv_4bit(x, B, K, W, N, y, stream):
 
 def bnb_gemm_4bit(X, M, K, W, N, Y, stream):
     return load().bnb_gemm_4bit(X, M, K, ctypes.byref(W), N, Y, stream)
+
+
+def bnb_gemv_4bit_grouped(problems, B, dtype, stream):
+    """``problems``: a sequence of GemvProblem (or a ctypes array of them)."""
+    if not isinstance(problems, ctypes.Array):
+        problems = (GemvProblem * len(problems))(*problems)
+    return load().bnb_gemv_4bit_grouped(problems, len(problems), B, dtype, stream)
 
 
 def bnb_linear_4bit(x, dtype, M, K, W, N, bias, y, stream):
@@ -342,6 +360,29 @@ def linear_4bit(x, state, N, bias=None, out=None):
                          _stream())
     _check(rc, "bnb_linear_4bit")
     return out
+
+
+def gemv_4bit_grouped(items, outs=None):
+    """Several decode linears in one launch: ``items`` is a list of (x,
+    state, N) or (x, state, N, bias) with x [B, K] (bf16 or fp16, the same B
+    and dtype for all; x may be shared); returns the outputs [B, N] (or
+    writes ``outs``).  Bit-identical to calling linear_4bit on each."""
+    torch = _torch()
+    if outs is None:
+        outs = [torch.empty(it[0].shape[0], it[2], dtype=it[0].dtype, device=it[0].device)
+                for it in items]
+    dt = {"torch.bfloat16": BF16, "torch.float16": F16}.get(str(items[0][0].dtype))
+    if dt is None:
+        raise TypeError("gemv_4bit_grouped takes bfloat16 or float16 activations")
+    probs = (GemvProblem * len(items))()
+    for i, (it, y) in enumerate(zip(items, outs)):
+        x, state, N = it[0], it[1], it[2]
+        bias = it[3] if len(it) > 3 else None
+        probs[i] = GemvProblem(x.data_ptr(), state.cstruct(), x.shape[1], N,
+                               None if bias is None else bias.data_ptr(), y.data_ptr())
+    rc = bnb_gemv_4bit_grouped(probs, items[0][0].shape[0], dt, _stream())
+    _check(rc, "bnb_gemv_4bit_grouped")
+    return outs
 
 
 def state_from_arrays(arrs, device="cuda"):

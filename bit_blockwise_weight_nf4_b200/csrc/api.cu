@@ -67,6 +67,12 @@ int error_word(int** out) {
   return BNB4_OK;
 }
 
+}  // namespace
+
+int bnb4::device_error_word(int** out) { return error_word(out); }
+
+namespace {
+
 // Fields shared by every state check.
 int check_state_common(const bnb4_qstate* st) {
   if (!st || !st->codes || st->n <= 0) return BNB4_ERR_INVALID_ARG;
@@ -77,6 +83,8 @@ int check_state_common(const bnb4_qstate* st) {
   if (st->reserved != 0) return BNB4_ERR_INVALID_ARG;
   if (!valid_blocksize(st->blocksize)) return BNB4_ERR_UNSUPPORTED;
   if (!aligned(st->codes, 16)) return BNB4_ERR_ALIGNMENT;
+  // the decode kernel copies the aligned 4-byte word holding each scale byte
+  if (st->double_quant && st->absmax_q && !aligned(st->absmax_q, 4)) return BNB4_ERR_ALIGNMENT;
   return BNB4_OK;
 }
 
@@ -116,9 +124,19 @@ int from_cuda(cudaError_t e) { return e == cudaSuccess ? BNB4_OK : BNB4_ERR_CUDA
 // load).  Anything else, pageable host memory in particular, is refused
 // before anything is launched: a kernel given a plain host address would
 // fault.  *dev receives the address the device uses.
+//
+// The query is a host-side lookup that enqueues nothing; a caller may be in
+// the middle of capturing a stream into a CUDA graph, whose default (global)
+// mode forbids such calls.  The query therefore runs with this thread's
+// capture interaction mode switched to relaxed and restored right after, so
+// the checks behave the same inside and outside a capture.
 int bnb4::resolve_ptr(const void* p, Residency where, const void** dev) {
   cudaPointerAttributes a;
-  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+  cudaStreamCaptureMode mode = cudaStreamCaptureModeRelaxed;
+  const bool swapped = cudaThreadExchangeStreamCaptureMode(&mode) == cudaSuccess;
+  const cudaError_t q = cudaPointerGetAttributes(&a, p);
+  if (swapped) cudaThreadExchangeStreamCaptureMode(&mode);
+  if (q != cudaSuccess) {
     cudaGetLastError();  // clear the (non-sticky) error the failed query recorded
     return BNB4_ERR_INVALID_ARG;
   }
@@ -198,9 +216,7 @@ int quantize_impl(const void* x, int32_t x_dtype, const bnb4_qstate* st, void* w
     if (!st->absmax_q || !st->scale2 || !st->offset) return BNB4_ERR_INVALID_ARG;
     if (!aligned(st->scale2, 4) || !aligned(st->offset, 4))
       return BNB4_ERR_ALIGNMENT;
-    if (!workspace ||
-        workspace_bytes < sizeof(double) * static_cast<size_t>(bnb4::kMaxPartials))
-      return BNB4_ERR_WORKSPACE;
+    if (!workspace || workspace_bytes < bnb4::kDqWorkspaceBytes) return BNB4_ERR_WORKSPACE;
     if (!aligned(workspace, 16)) return BNB4_ERR_ALIGNMENT;
   }
   int sms;
@@ -213,9 +229,10 @@ int quantize_impl(const void* x, int32_t x_dtype, const bnb4_qstate* st, void* w
       (rc = bnb4::resolve_ptr(workspace, bnb4::Residency::kDeviceOrManaged, &ws_dev)) !=
           BNB4_OK)
     return rc;
-  const int grid = bnb4::quant_grid(st->n, x_dtype, sms);
-  return from_cuda(bnb4::launch_quantize(xd, x_dtype, *st, static_cast<double*>(workspace),
-                                         grid, static_cast<cudaStream_t>(stream), view));
+  int* err = nullptr;
+  if (st->double_quant && (rc = error_word(&err)) != BNB4_OK) return rc;
+  return from_cuda(bnb4::launch_quantize(xd, x_dtype, *st, workspace, err, sms,
+                                         static_cast<cudaStream_t>(stream), view));
 }
 
 int dequantize_impl(const bnb4_qstate* st, void* out, int32_t out_dtype, void* stream,
@@ -277,8 +294,7 @@ int bnb4_query_sizes(int64_t n, int32_t blocksize, int32_t double_quant,
   out->absmax_q = double_quant ? static_cast<size_t>(nb) : 0;
   out->scale2 = double_quant ? static_cast<size_t>(4 * ng) : 0;
   out->offset = double_quant ? 4 : 0;
-  out->workspace =
-      double_quant ? sizeof(double) * static_cast<size_t>(bnb4::kMaxPartials) : 0;
+  out->workspace = double_quant ? bnb4::kDqWorkspaceBytes : 0;
   return BNB4_OK;
 }
 
@@ -324,16 +340,51 @@ int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstate* W,
   int rc = check_weight(W, N, K);
   if (rc != BNB4_OK) return rc;
   if (B < 1 || B > kSmallMaxM) return BNB4_ERR_SHAPE;
+  if (N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return BNB4_ERR_SHAPE;
   if (!aligned(x, 16) || !aligned(y, 2)) return BNB4_ERR_ALIGNMENT;
   int sms;
   if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
   if ((rc = check_linear_memory(x, y, nullptr, W)) != BNB4_OK) return rc;
-  if (B <= kGemvMaxB)
-    return from_cuda(bnb4::launch_gemv(x, B, K, *W, N, y, nullptr, BNB4_BF16, sms,
-                                       static_cast<cudaStream_t>(stream)));
   int* err;
   if ((rc = error_word(&err)) != BNB4_OK) return rc;
+  if (B <= kGemvMaxB)
+    return from_cuda(bnb4::launch_gemv(x, B, K, *W, N, y, nullptr, BNB4_BF16, sms, err,
+                                       static_cast<cudaStream_t>(stream)));
   return from_cuda(bnb4::launch_gemm_small(x, B, K, *W, N, y, nullptr, BNB4_BF16, err, sms,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+int bnb_gemv_4bit_grouped(const bnb4_gemv_problem* problems, int32_t count, int64_t B,
+                          int32_t dtype, void* stream) {
+  if (!problems || count < 1) return BNB4_ERR_INVALID_ARG;
+  if (count > BNB4_GROUP_MAX) return BNB4_ERR_SHAPE;
+  if (dtype != BNB4_BF16 && dtype != BNB4_F16) return BNB4_ERR_UNSUPPORTED;
+  if (B < 1 || B > kGemvMaxB) return BNB4_ERR_SHAPE;
+  bnb4::GemvLinear lin[BNB4_GROUP_MAX];
+  const bnb4_qstate& W0 = problems[0].W;
+  for (int32_t i = 0; i < count; ++i) {
+    const bnb4_gemv_problem& p = problems[i];
+    if (!p.x || !p.y) return BNB4_ERR_INVALID_ARG;
+    int rc = check_weight(&p.W, p.N, p.K);
+    if (rc != BNB4_OK) return rc;
+    if (p.N >= (int64_t(1) << 31) || p.K >= (int64_t(1) << 31) || p.K != problems[0].K)
+      return BNB4_ERR_SHAPE;
+    if (p.W.blocksize != W0.blocksize || p.W.qtype != W0.qtype ||
+        p.W.double_quant != W0.double_quant)
+      return BNB4_ERR_UNSUPPORTED;
+    if (!aligned(p.x, 16) || !aligned(p.y, 2) || !aligned(p.bias, 16))
+      return BNB4_ERR_ALIGNMENT;
+    lin[i] = bnb4::GemvLinear{p.x, &p.W, p.K, p.N, p.bias, p.y};
+  }
+  int sms, rc;
+  if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
+  for (int32_t i = 0; i < count; ++i) {
+    const bnb4_gemv_problem& p = problems[i];
+    if ((rc = check_linear_memory(p.x, p.y, p.bias, &p.W)) != BNB4_OK) return rc;
+  }
+  int* err;
+  if ((rc = error_word(&err)) != BNB4_OK) return rc;
+  return from_cuda(bnb4::launch_gemv_group(lin, count, B, dtype, sms, err,
                                            static_cast<cudaStream_t>(stream)));
 }
 
@@ -342,7 +393,8 @@ int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstate* W,
   if (!X || !Y) return BNB4_ERR_INVALID_ARG;
   int rc = check_weight(W, N, K);
   if (rc != BNB4_OK) return rc;
-  if (M < 1 || N % 8 != 0 || M > (int64_t(1) << 31) || N > (int64_t(1) << 31))
+  if (M < 1 || N % 8 != 0 || M > (int64_t(1) << 31) || N >= (int64_t(1) << 31) ||
+      K >= (int64_t(1) << 31))
     return BNB4_ERR_SHAPE;
   if (!aligned(X, 16) || !aligned(Y, 16)) return BNB4_ERR_ALIGNMENT;
   int sms;
@@ -351,7 +403,7 @@ int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstate* W,
   int* err;
   if ((rc = error_word(&err)) != BNB4_OK) return rc;
   if (M <= kGemvMaxB)
-    return from_cuda(bnb4::launch_gemv(X, M, K, *W, N, Y, nullptr, BNB4_BF16, sms,
+    return from_cuda(bnb4::launch_gemv(X, M, K, *W, N, Y, nullptr, BNB4_BF16, sms, err,
                                        static_cast<cudaStream_t>(stream)));
   if (M <= kSmallMaxM)
     return from_cuda(bnb4::launch_gemm_small(X, M, K, *W, N, Y, nullptr, BNB4_BF16, err,
@@ -366,7 +418,8 @@ int bnb_linear_4bit(const void* x, int32_t dtype, int64_t M, int64_t K, const bn
   if (dtype != BNB4_BF16 && dtype != BNB4_F16) return BNB4_ERR_UNSUPPORTED;
   int rc = check_weight(W, N, K);
   if (rc != BNB4_OK) return rc;
-  if (M < 1 || M > (int64_t(1) << 31) || N > (int64_t(1) << 31)) return BNB4_ERR_SHAPE;
+  if (M < 1 || M > (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
+    return BNB4_ERR_SHAPE;
   if (M > kSmallMaxM && N % 8 != 0) return BNB4_ERR_SHAPE;
   if (!aligned(x, 16) || !aligned(y, M > kSmallMaxM ? 16 : 2) || !aligned(bias, 16))
     return BNB4_ERR_ALIGNMENT;
@@ -374,10 +427,10 @@ int bnb_linear_4bit(const void* x, int32_t dtype, int64_t M, int64_t K, const bn
   if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
   if ((rc = check_linear_memory(x, y, bias, W)) != BNB4_OK) return rc;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (M <= kGemvMaxB)
-    return from_cuda(bnb4::launch_gemv(x, M, K, *W, N, y, bias, dtype, sms, s));
   int* err;
   if ((rc = error_word(&err)) != BNB4_OK) return rc;
+  if (M <= kGemvMaxB)
+    return from_cuda(bnb4::launch_gemv(x, M, K, *W, N, y, bias, dtype, sms, err, s));
   if (M <= kSmallMaxM)
     return from_cuda(bnb4::launch_gemm_small(x, M, K, *W, N, y, bias, dtype, err, sms, s));
   return from_cuda(bnb4::launch_gemm(x, M, K, *W, N, y, bias, dtype, err, sms, s));

@@ -20,6 +20,7 @@
 // ragged tile at the end takes a bounds-checked path.
 #include "common.cuh"
 #include "kernels.h"
+#include "lut.cuh"
 
 namespace bnb4 {
 namespace {
@@ -41,11 +42,6 @@ struct Out<BNB4_F32> {
   static constexpr int kPerChunk = 4;
 };
 
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(s));
-  return d;
-}
 
 // Raw scale inputs of a block: absmax_q byte and scale2 (double quant) or the
 // absmax bits.

@@ -20,16 +20,22 @@ enum class Residency { kDevice, kDeviceOrManaged, kDeviceOrPinnedHost };
 // memory `where` excludes).  Host-only; launches nothing.
 int resolve_ptr(const void* p, Residency where, const void** dev);
 
-// Upper bound on the quantize grid; the double-quant workspace holds one fp64
-// partial sum per CTA.
+// Upper bound on the quantize grid.  The double-quant workspace holds a call
+// counter and, per CTA, a tag and an fp64 partial sum of its blocks' absmax
+// (8-byte words: counter at 0, tags from 8, sums from 8 + kMaxPartials).
 constexpr int kMaxPartials = 4096;
+constexpr size_t kDqWorkspaceBytes = 8 * (8 + 2 * static_cast<size_t>(kMaxPartials));
 
 int quant_grid(int64_t n, int x_dtype, int num_sms);
-// view: x is a row-major 2-D view with a row stride (see View2D), or null
-// for a contiguous x.
+// workspace: kDqWorkspaceBytes, 16-byte aligned (double quant only); err:
+// the device error word.  view: x is a row-major 2-D view with a row stride
+// (see View2D), or null for a contiguous x.
 cudaError_t launch_quantize(const void* x, int x_dtype, const bnb4_qstate& st,
-                            double* partials, int grid, cudaStream_t s,
+                            void* workspace, int* err, int num_sms, cudaStream_t s,
                             const View2D* view = nullptr);
+
+// The library's device error word on the current device (api.cu).
+int device_error_word(int** out);
 
 int dequant_grid(int64_t n, int out_dtype, int num_sms);
 cudaError_t launch_dequantize(const bnb4_qstate& st, void* out, int out_dtype,
@@ -41,9 +47,24 @@ cudaError_t launch_check_rcp(void* result, cudaStream_t s);
 
 // The linear kernels take the 16-bit compute format `fmt` (BNB4_BF16 or
 // BNB4_F16) of x, y and bias; bias (N elements) may be null.
+// err: the device error word (set when a bounded wait of the decode kernel
+// expires).
 cudaError_t launch_gemv(const void* x, int64_t B, int64_t K,
                         const bnb4_qstate& W, int64_t N, void* y, const void* bias,
-                        int fmt, int num_sms, cudaStream_t s);
+                        int fmt, int num_sms, int* err, cudaStream_t s);
+
+// One decode linear of a grouped launch (x [B, K], W [N, K], bias, y [B, N]).
+struct GemvLinear {
+  const void* x;
+  const bnb4_qstate* W;
+  int64_t K, N;
+  const void* bias;
+  void* y;
+};
+// 1..BNB4_GROUP_MAX linears of one format (blocksize, code table, scale
+// format) and one batch size B <= 8 in one persistent launch.
+cudaError_t launch_gemv_group(const GemvLinear* lin, int count, int64_t B, int fmt,
+                              int num_sms, int* err, cudaStream_t s);
 
 // wait_limit_ns = 0 selects the normal bound of every mbarrier wait (2 s);
 // withhold_first_x != 0 is the failure-detection diagnostic (the first X

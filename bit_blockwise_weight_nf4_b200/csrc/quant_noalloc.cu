@@ -6,10 +6,10 @@
 // allocation, a loader working under a fixed device-memory budget, or a
 // latency-critical path where cudaMalloc (which may synchronize the device or
 // fail under memory pressure) is not acceptable.  This entry point keeps its
-// scratch -- one fp64 partial sum per CTA for the mean of the block scales and
-// the exact fp32 absmax of every block, which double quantization consumes
-// and nobody reads afterwards -- in a fixed array in the library's own device
-// memory instead.  The caller still passes the input and the outputs (codes,
+// scratch -- the bookkeeping of the grid-wide mean of the block scales (a call
+// counter, per-CTA tags and fp64 partial sums) and the exact fp32 absmax of
+// every block, which double quantization consumes and nobody reads
+// afterwards -- in a fixed array in the library's own device memory instead.  The caller still passes the input and the outputs (codes,
 // absmax_q, scale2, offset).
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -21,10 +21,11 @@
 
 namespace {
 
-// Scratch layout: kMaxPartials fp64 partial sums, then up to
-// BNB4_NOALLOC_MAX_BLOCKS fp32 absmax values: 32 KiB + 4 MiB.  Every GPU that
-// loads the library holds this array until the process exits.
-constexpr size_t kPartialsBytes = sizeof(double) * bnb4::kMaxPartials;
+// Scratch layout: the double quantization's bookkeeping (a call counter and,
+// per CTA, a tag and an fp64 partial sum: 64 KiB), then up to
+// BNB4_NOALLOC_MAX_BLOCKS fp32 absmax values (4 MiB).  Every GPU that loads
+// the library holds this array until the process exits; it starts zeroed.
+constexpr size_t kPartialsBytes = (bnb4::kDqWorkspaceBytes + 255) / 256 * 256;
 constexpr size_t kScratchBytes =
     kPartialsBytes + sizeof(float) * static_cast<size_t>(BNB4_NOALLOC_MAX_BLOCKS);
 
@@ -93,8 +94,8 @@ extern "C" BNB4_API int bnb_quantize_4bit_noalloc(const void* x, int32_t x_dtype
       st->blocksize != 256)
     return BNB4_ERR_UNSUPPORTED;
   if (!st->absmax_q || !st->scale2 || !st->offset) return BNB4_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(st->codes, 16) || !aligned(st->scale2, 4) ||
-      !aligned(st->offset, 4))
+  if (!aligned(x, 16) || !aligned(st->codes, 16) || !aligned(st->absmax_q, 4) ||
+      !aligned(st->scale2, 4) || !aligned(st->offset, 4))
     return BNB4_ERR_ALIGNMENT;
   const int64_t nb = (st->n + st->blocksize - 1) / st->blocksize;
   if (nb > BNB4_NOALLOC_MAX_BLOCKS) return BNB4_ERR_SCRATCH_LIMIT;
@@ -116,13 +117,12 @@ extern "C" BNB4_API int bnb_quantize_4bit_noalloc(const void* x, int32_t x_dtype
     return rc;
   unsigned char* scratch = nullptr;
   if ((rc = scratch_address(&scratch)) != BNB4_OK) return rc;
-  const int grid = bnb4::quant_grid(st->n, x_dtype, sms);
-  if (grid > bnb4::kMaxPartials) return BNB4_ERR_SCRATCH_LIMIT;
+  int* err = nullptr;
+  if ((rc = bnb4::device_error_word(&err)) != BNB4_OK) return rc;
 
-  bnb4_qstate s = *st;  // same kernels, with the intermediate absmax in scratch
+  bnb4_qstate s = *st;  // same kernel, with the intermediate absmax in scratch
   s.absmax = reinterpret_cast<float*>(scratch + kPartialsBytes);
-  const cudaError_t e = bnb4::launch_quantize(
-      xd, x_dtype, s, reinterpret_cast<double*>(scratch), grid,
-      static_cast<cudaStream_t>(stream));
+  const cudaError_t e = bnb4::launch_quantize(xd, x_dtype, s, scratch, err, sms,
+                                              static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? BNB4_OK : BNB4_ERR_CUDA;
 }

@@ -1,7 +1,7 @@
 // sm100.cuh -- building blocks of the tcgen05 kernels (sm_100a): mbarriers
 // with bounded waits, cluster addressing, TMA tensor copies, shared-memory
-// matrix descriptors, the 4-bit -> bf16 byte-permute dequantization and the
-// host-side tensor-map encoding.  Shared by the prefill GEMM and the
+// matrix descriptors and the host-side tensor-map encoding (the 4-bit ->
+// 16-bit byte-permute dequantization is in lut.cuh).  Shared by the prefill GEMM and the
 // small-M GEMM; no TMA load here uses cluster multicast.
 #pragma once
 
@@ -9,6 +9,7 @@
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
+#include "lut.cuh"
 
 namespace bnb4 {
 namespace {
@@ -162,65 +163,6 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
   d |= static_cast<uint64_t>(1u) << 46;          // descriptor version
   d |= static_cast<uint64_t>(2u) << 61;          // SWIZZLE_128B
   return d;
-}
-
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t s) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(s));
-  return d;
-}
-
-struct Lut {
-  uint32_t L[4], H[4];
-};
-
-// Per-block table of the 16 dequantized values in the 16-bit compute format F
-// (BNB4_BF16 or BNB4_F16), split by byte: L[q] holds the low bytes of
-// entries 4q..4q+3, H[q] the high bytes.
-template <int QT, int F>
-__device__ __forceinline__ Lut make_lut(float ah) {
-  uint32_t P[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int c0 = 2 * j, c1 = 2 * j + 1;
-    const float t0 = QT == kQtNF4 ? nf4_value(c0)
-                                  : ((c0 & 8) ? -fp4_magnitude(c0 & 7) : fp4_magnitude(c0 & 7));
-    const float t1 = QT == kQtNF4 ? nf4_value(c1)
-                                  : ((c1 & 8) ? -fp4_magnitude(c1 & 7) : fp4_magnitude(c1 & 7));
-    P[j] = pack2<F>(__fmul_rn(t0, ah), __fmul_rn(t1, ah));
-  }
-  Lut l;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    l.L[q] = prmt(P[2 * q], P[2 * q + 1], 0x6420);
-    l.H[q] = prmt(P[2 * q], P[2 * q + 1], 0x7531);
-  }
-  return l;
-}
-
-// 8 codes of one packed 32-bit word (natural order k0..k7) -> 8 16-bit values in k
-// order as 4 words.  The low 3 bits of each code select from the two
-// 8-entry halves of the table, bit 3 picks the half; one mask / shift of the
-// whole word serves both 4-code halves (prmt reads the low 16 selector bits).
-__device__ __forceinline__ uint4 dq8(const Lut& l, uint32_t w) {
-  const uint32_t sel = w & 0x77777777u;
-  const uint32_t mix = ((w >> 1) & 0x44444444u) | 0x32103210u;
-  uint4 o;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    const uint32_t s = h ? sel >> 16 : sel;
-    const uint32_t m = h ? mix >> 16 : mix;
-    const uint32_t lo = prmt(prmt(l.L[0], l.L[1], s), prmt(l.L[2], l.L[3], s), m);
-    const uint32_t hi = prmt(prmt(l.H[0], l.H[1], s), prmt(l.H[2], l.H[3], s), m);
-    if (h == 0) {
-      o.x = prmt(lo, hi, 0x4051);
-      o.y = prmt(lo, hi, 0x6273);
-    } else {
-      o.z = prmt(lo, hi, 0x4051);
-      o.w = prmt(lo, hi, 0x6273);
-    }
-  }
-  return o;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {

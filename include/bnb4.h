@@ -37,7 +37,8 @@
  *    features K) is quantized as the flat array of N*K elements, so its
  *    blocks run along K.
  *  - Alignment: x / out / codes / X / Y pointers must be 16-byte aligned;
- *    fp32 arrays 4-byte aligned.  Misalignment returns BNB4_ERR_ALIGNMENT.
+ *    fp32 arrays and absmax_q 4-byte aligned.  Misalignment returns
+ *    BNB4_ERR_ALIGNMENT.
  *  - Results are deterministic for a given input and device: codes, absmax,
  *    double-quant fields and dequantized values are bit-identical to the
  *    reference definition below.  The GEMV / GEMM accumulate in fp32 and round
@@ -53,7 +54,7 @@
 extern "C" {
 #endif
 
-#define BNB4_ABI_VERSION 2
+#define BNB4_ABI_VERSION 3
 
 /* Every entry point is exported from the shared library (the library is
  * built with hidden visibility by default). */
@@ -93,6 +94,7 @@ extern "C" {
  *            modes; read by the consumers only when double_quant == 0.
  *  absmax_q  uint8[nb]: u = q + 128, q = clamp(rint((absmax - offset) / s),
  *            -127, 127) with s the scale of the block's group (double quant).
+ *            4-byte aligned.
  *  scale2    float[ng]: s = max |absmax - offset| over the group / 127.
  *  offset    float[1]: mean of absmax (fp64 sum, rounded to fp32).
  * The decoded scale of block b is fma(u_b - 128, scale2[b/256], offset) with
@@ -144,7 +146,15 @@ BNB4_API int bnb4_query_sizes(int64_t n, int32_t blocksize, int32_t double_quant
  *              always; absmax_q, scale2 and offset when st->double_quant.
  *  workspace   device scratch of at least bnb4_query_sizes(...).workspace
  *              bytes, 16-byte aligned (may be NULL when the size is 0).
- *              Its contents on entry do not matter.
+ *              Any contents on first use; between calls it keeps a call
+ *              counter that the next call on it relies on, so do not write
+ *              to it, and do not share one workspace between calls that
+ *              may overlap on the GPU (different streams).
+ * With double quantization the launch is cooperative (all of its CTAs are
+ * resident at once): the grid-wide mean of the absmax is formed inside the
+ * one kernel, each CTA waiting -- at most 2 s, after which it sets the
+ * device error word (bnb4_device_status reports BNB4_ERR_DEVICE_TIMEOUT) and
+ * leaves the double-quant outputs unwritten -- for the others' partial sums.
  * Per block: a = max|x|; r = RN(1/a) (0 for a = 0); v = RN(x*r); code =
  * number of fp32 codebook midpoints RN(RN(t[i]+t[i+1])*0.5) strictly below v
  * (FP4: of magnitude midpoints below |v|, sign bit set for v < 0 with a
@@ -169,9 +179,10 @@ BNB4_API int bnb_quantize_4bit(const void* x, int32_t x_dtype, const bnb4_qstate
  * Same method and bit-identical results as bnb_quantize_4bit with
  * st->double_quant = 1, except that the exact fp32 absmax is not returned:
  * st->absmax is ignored (may be NULL) and the intermediate absmax and the
- * per-CTA fp64 partial sums live in a fixed array in the library's own
- * device memory (32 KiB + 4 MiB per GPU that loads the library, held until
- * the process exits).  The caller passes x and the outputs codes, absmax_q,
+ * bookkeeping of the grid-wide mean (a call counter, per-CTA tags and fp64
+ * partial sums) live in a fixed array in the library's own device memory
+ * (64 KiB + 4 MiB per GPU that loads the library, held until the process
+ * exits).  The caller passes x and the outputs codes, absmax_q,
  * scale2 and offset, with the alignment rules of bnb_quantize_4bit.
  *  - Limit: at most BNB4_NOALLOC_MAX_BLOCKS blocks (ceil(n / blocksize));
  *    larger inputs return BNB4_ERR_SCRATCH_LIMIT and launch nothing.
@@ -186,10 +197,11 @@ BNB4_API int bnb_quantize_4bit(const void* x, int32_t x_dtype, const bnb4_qstate
  *    array's module and maps its 4 MiB on the device, so the first call can
  *    return BNB4_ERR_CUDA when the device is out of memory: make it at
  *    start-up, before any stream capture on the device.
- *  - Every call shares the one array, and a call overwrites all of the
- *    scratch it reads, so nothing carries over from the previous call; calls
- *    that overlap on the GPU (different streams, or devices sharing a
- *    context) race on it and must be serialized by the caller.
+ *  - Every call shares the one array.  A call overwrites all of the scratch
+ *    it reads except the call counter of its grid-wide mean, which each call
+ *    advances, so no result carries over from the previous call; calls that
+ *    overlap on the GPU (different streams) race on it and must be
+ *    serialized by the caller.
  * Allocates nothing and calls no allocating routine.
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, SCRATCH_LIMIT, CUDA.
  */
@@ -243,13 +255,56 @@ BNB4_API int bnb_dequantize_4bit_2d(const bnb4_qstate* st, void* out, int32_t ou
  * exact, fp32 accumulation (order unspecified), one final rounding to bf16.
  *  x  device bf16 [B, K], 16-byte aligned;   y  device bf16 [B, N].
  *  W  quantization state of the weight [N, K] (W->n == N*K).
- * Constraints: 1 <= B <= 256; K % 64 == 0; K % W->blocksize == 0.
- * B <= 8 runs the decode kernel (mma.sync, one 8-column group); larger
- * batches run the small-batch tcgen05 kernel of bnb_gemm_4bit.
+ * Constraints: 1 <= B <= 256; K % 64 == 0; K % W->blocksize == 0; N, K <
+ * 2^31.  B <= 8 runs the decode kernel (persistent, one CTA per SM; the
+ * packed weight tiles staged in shared memory by TMA; mma.sync, one 8-column
+ * group; partial sums over K added in a fixed order, so results are
+ * bit-reproducible); larger batches run the small-batch tcgen05 kernel of
+ * bnb_gemm_4bit.
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, SHAPE, CUDA.
  */
 BNB4_API int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstate* W,
                   int64_t N, void* y, void* stream);
+
+/*
+ * Several decode GEMVs in one launch (release notes 0.50.0 / gemv_4bit, as
+ * used by a decoder step: the linears that read the same activations, such
+ * as q / k / v or gate / up, or any list of independent batch-B linears):
+ * for every problem i,
+ *   y_i[b, n] = h( sum_k x_i[b, k] * What_i[n, k] + bias_i[n] ),
+ * the arithmetic of bnb_linear_4bit with M = B (exact products, fp32
+ * accumulation, one rounding).  One persistent grid streams all the weights,
+ * so the start-up of a launch is paid once for the whole list.  The order of
+ * the fp32 sums over K follows how the row groups of the whole list are
+ * split over the SMs, so a problem's result can differ in the last bit from
+ * a single call; the same list on the same device gives identical bits.
+ *  problems  host array of `count` descriptors (read during the call only):
+ *            x device [B, K] of dtype, 16-byte aligned; W the quantization
+ *            state of the weight [N, K] (W.n == N * K); bias device [N] of
+ *            dtype, 16-byte aligned, or NULL; y device [B, N] of dtype,
+ *            2-byte aligned.  x may be shared between problems; the y must
+ *            not overlap each other or any x.
+ *  count     1 .. BNB4_GROUP_MAX.
+ *  B         1 .. 8 rows of every x.
+ *  dtype     BNB4_BF16 or BNB4_F16 (the compute type of every problem).
+ * Constraints: every problem has the same K (K % 64 == 0, K % blocksize ==
+ * 0, K < 2^31) and every W the same blocksize, qtype and double_quant (the
+ * linears that share an input, such as q / k / v, satisfy both); N < 2^31.
+ * Lists longer than 32 problems run as several launches of up to 32.
+ * Errors: INVALID_ARG, UNSUPPORTED (dtype, or mixed weight formats),
+ * ALIGNMENT, SHAPE (including different K), CUDA.
+ */
+#define BNB4_GROUP_MAX 256
+typedef struct bnb4_gemv_problem {
+  const void* x;
+  bnb4_qstate W;
+  int64_t K;
+  int64_t N;
+  const void* bias;
+  void* y;
+} bnb4_gemv_problem;
+BNB4_API int bnb_gemv_4bit_grouped(const bnb4_gemv_problem* problems, int32_t count,
+                                   int64_t B, int32_t dtype, void* stream);
 
 /*
  * Prefill GEMM with the dequantization fused in (release notes 0.50.0):

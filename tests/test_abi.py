@@ -88,6 +88,7 @@ def good_state(**kw):
     ({"n": 0}, A16, 1, A16, 1 << 20, bnb4.ERR_INVALID_ARG),
     ({"reserved": 1}, A16, 1, A16, 1 << 20, bnb4.ERR_INVALID_ARG),
     ({"codes": A16 + 8}, A16, 1, A16, 1 << 20, bnb4.ERR_ALIGNMENT),
+    ({"absmax_q": A16 + 0x2001}, A16, 1, A16, 1 << 20, bnb4.ERR_ALIGNMENT),
     ({}, A16 + 4, 1, A16, 1 << 20, bnb4.ERR_ALIGNMENT),
     ({}, A16, 1, None, 0, bnb4.ERR_WORKSPACE),
     ({}, A16, 1, A16, 64, bnb4.ERR_WORKSPACE),
@@ -126,6 +127,30 @@ def test_gemv_argument_errors(lib):
     assert call(W=good_state(n=128 * 64, blocksize=128), N=128) == bnb4.ERR_SHAPE
     assert call(x=A16 + 8) == bnb4.ERR_ALIGNMENT
     assert call(y=A16 + 1) == bnb4.ERR_ALIGNMENT
+    assert call(W=good_state(n=64 * 64, absmax_q=A16 + 0x2002)) == bnb4.ERR_ALIGNMENT
+
+
+def test_grouped_gemv_argument_errors(lib):
+    def prob(**kw):
+        d = dict(x=A16, W=good_state(n=64 * 64), K=64, N=64, bias=None, y=A16)
+        d.update(kw)
+        return bnb4.GemvProblem(d["x"], d["W"], d["K"], d["N"], d["bias"], d["y"])
+
+    def call(probs, B=1, dt=bnb4.BF16):
+        return bnb4.bnb_gemv_4bit_grouped(probs, B, dt, None)
+    assert lib.bnb_gemv_4bit_grouped(None, 1, 1, bnb4.BF16, None) == bnb4.ERR_INVALID_ARG
+    assert call([prob()] * (bnb4.GROUP_MAX + 1)) == bnb4.ERR_SHAPE
+    assert call([prob()], dt=bnb4.F32) == bnb4.ERR_UNSUPPORTED
+    assert call([prob()], B=9) == bnb4.ERR_SHAPE
+    assert call([prob()], B=0) == bnb4.ERR_SHAPE
+    assert call([prob(), prob(x=None)]) == bnb4.ERR_INVALID_ARG
+    assert call([prob(), prob(N=65)]) == bnb4.ERR_SHAPE
+    assert call([prob(), prob(K=128, W=good_state(n=64 * 128))]) == bnb4.ERR_SHAPE  # K differs
+    assert call([prob(K=128, W=good_state(n=64 * 128)),
+                 prob(W=good_state(n=64 * 128, blocksize=128), K=128)]) == bnb4.ERR_UNSUPPORTED
+    assert call([prob(), prob(W=good_state(n=64 * 64, qtype=bnb4.FP4))]) == bnb4.ERR_UNSUPPORTED
+    assert call([prob(), prob(bias=A16 + 2)]) == bnb4.ERR_ALIGNMENT
+    assert call([prob(x=A16 + 8)]) == bnb4.ERR_ALIGNMENT
 
 
 def test_gemm_argument_errors(lib):

@@ -1,6 +1,7 @@
 """GPU prefill GEMM (tcgen05, fused dequantization) against the fp64 oracle
 over the dequantized bf16 weight, with the tolerance of the method's brief.
-Full-size shapes are checked on a seeded sample of rows of X (all columns);
+Full-size shapes are checked on a seeded sample of 128 rows of X (8 from
+every 128-row sub-tile, its edge rows included; all columns);
 small shapes, including ragged M, are checked in full."""
 import numpy as np
 import pytest
@@ -22,9 +23,18 @@ def case(M, N, K, bs, qtype, dq, seed, n_rows=None):
     Xb = synth.bf16_bits(X)
     rows = None
     if n_rows is not None and n_rows < M:
+        # stratified: the same number of rows from every 128-row sub-tile
+        # (each CTA of a pair holds 128-row sub-tiles of X), its first and
+        # last row included
         rng = np.random.default_rng(seed)
-        rows = np.unique(np.concatenate([[0, M - 1],
-                                         rng.choice(M, n_rows - 2, replace=False)]))
+        per = max(2, n_rows // -(-M // 128))
+        picks = []
+        for t0 in range(0, M, 128):
+            t1 = min(t0 + 128, M)
+            inner = np.arange(t0 + 1, t1 - 1)
+            k = min(per - 2, inner.size)
+            picks += [t0, t1 - 1] + list(rng.choice(inner, k, replace=False) if k > 0 else [])
+        rows = np.unique(np.array(picks))
     y64 = oracle.linear_ref(Xb, What, rows=rows)
     g = bnb4.state_from_arrays(st)
     Y = bnb4.gemm_4bit(X.cuda(), g, N)
@@ -40,13 +50,13 @@ def case(M, N, K, bs, qtype, dq, seed, n_rows=None):
 def test_prefill_shapes_nf4_bs64(N, K):
     """X bf16 [2048, K] ~ N(0, 1); NF4 weight ~ N(0, 0.02^2), blocksize 64,
     double quant."""
-    case(synth.GEMM_M, N, K, 64, bnb4.NF4, True, seed=N + 3 * K, n_rows=48)
+    case(synth.GEMM_M, N, K, 64, bnb4.NF4, True, seed=N + 3 * K, n_rows=128)
 
 
 @pytest.mark.parametrize("qtype,bs", [(bnb4.NF4, 128), (bnb4.FP4, 64),
                                       (bnb4.FP4, 128)])
 def test_prefill_variants(qtype, bs):
-    case(synth.GEMM_M, 4096, 4096, bs, qtype, True, seed=bs + qtype, n_rows=48)
+    case(synth.GEMM_M, 4096, 4096, bs, qtype, True, seed=bs + qtype, n_rows=128)
 
 
 @pytest.mark.parametrize("qtype", [bnb4.NF4, bnb4.FP4])

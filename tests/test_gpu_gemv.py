@@ -46,11 +46,26 @@ def test_small_ragged(qtype, bs, dq, N, K, B):
 
 
 @pytest.mark.parametrize("N,K,B", [(4099, 4096, 1), (1030, 2112, 2), (517, 11008, 4),
-                                   (30001, 256, 8), (4096, 64, 1), (22, 1344, 2)])
+                                   (30001, 256, 8), (4096, 64, 1), (22, 1344, 2),
+                                   (40003, 1024, 1), (38000, 2048, 3), (2400, 4352, 8)])
 def test_row_groups_and_warp_splits(N, K, B):
-    """16-row groups with ragged N, 1 to 8 warps holding K steps (K from 64
-    to 11008: a warp with no step, a last step with empty segments)."""
+    """16-row groups with ragged N; K split over the CTA's warps (K of at
+    least one 256-wide chunk per warp, or few row groups per CTA: 1 to 16
+    warps, a last chunk with empty segments) or whole row groups per warp
+    (short K and many row groups: 40003 x 1024, 38000 x 2048)."""
     case(N, K, B, 64, bnb4.NF4, True, seed=N + 3 * K + B)
+
+
+@pytest.mark.parametrize("N,K", [(11008, 4096), (4096, 11008), (40003, 1024)])
+def test_decode_is_bit_reproducible(N, K):
+    """The partial sums over K are added in a fixed order: repeated launches
+    give identical bits."""
+    W = synth.weight_bf16(N, K, seed=9)
+    g = bnb4.quantize_4bit(W.cuda().view(-1), 64, bnb4.NF4, True)
+    x = synth.activations_bf16(1, K, seed=10).cuda()
+    ys = [bnb4.gemv_4bit(x, g, N) for _ in range(3)]
+    torch.cuda.synchronize()
+    assert all(torch.equal(ys[0], y) for y in ys[1:])
 
 
 @pytest.mark.parametrize("B", [9, 16, 17, 24, 32, 33, 40, 63, 64])

@@ -170,3 +170,76 @@ def test_fast_reciprocal_exhaustive():
     mismatches, first = res.cpu().tolist()
     assert mismatches == 0, "first mismatching input bits 0x%08x" % (first & 0xffffffff)
     assert first & 0xffffffff == 0xffffffff
+
+
+# ---- the grid-wide mean of double quantization inside one cooperative kernel
+
+
+def _bits(x):
+    return synth.bf16_bits(x.cpu().view(-1)) if x.dtype == torch.bfloat16 else \
+        x.cpu().view(-1).numpy()
+
+
+def _check_dq(st, x, bs=64, qtype=bnb4.NF4):
+    orc = oracle.quantize(_bits(x), bs, qtype, True)
+    assert orc["sum_exact"]
+    assert_state_equal(bnb4.state_to_arrays(st), orc, True)
+
+
+def test_workspace_reused_across_inputs_and_sizes():
+    """One workspace, calls of different sizes and data in a row: the call
+    counter each call advances keeps a call from taking another call's
+    partial sums."""
+    ws = None
+    xs = [synth.weight_bf16(4096, 4096, seed=s, outlier_frac=synth.OUTLIER_FRAC).cuda().view(-1)
+          for s in (1, 2)] + [synth.normal_f32((100003,), seed=3, std=0.02).cuda()]
+    sts = []
+    for x in xs + xs[::-1]:
+        st = bnb4.QuantState(x.numel(), 64, bnb4.NF4, True)
+        ws = ws if ws is not None else bnb4.workspace_for(st)
+        sts.append((bnb4.quantize_4bit(x, 64, bnb4.NF4, True, state=st, workspace=ws), x))
+    torch.cuda.synchronize()
+    for st, x in sts:
+        _check_dq(st, x)
+    assert bnb4.bnb4_device_status(torch.cuda.current_stream().cuda_stream) == bnb4.OK
+
+
+def test_fresh_workspace_with_arbitrary_contents():
+    """A workspace's contents on first use do not matter."""
+    x = synth.weight_bf16(1024, 4096, seed=8).cuda().view(-1)
+    st = bnb4.QuantState(x.numel(), 64, bnb4.NF4, True)
+    for fill in (0x00, 0xFF, None):
+        ws = bnb4.workspace_for(st)
+        if fill is None:
+            ws.copy_(torch.randint(0, 256, ws.shape, dtype=torch.uint8))
+        else:
+            ws.fill_(fill)
+        bnb4.quantize_4bit(x, 64, bnb4.NF4, True, state=st, workspace=ws)
+        torch.cuda.synchronize()
+        _check_dq(st, x)
+
+
+def test_graph_replay_with_new_data_each_time():
+    """A quantize call captured once in a CUDA graph and replayed on new
+    input values each time: every replay forms its own mean (the kernel, not
+    the captured arguments, numbers the calls)."""
+    n = 4096 * 1024
+    x = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+    st = bnb4.QuantState(n, 64, bnb4.FP4, True)
+    ws = bnb4.workspace_for(st)
+    x.copy_(synth.weight_bf16(4096, 1024, seed=20).view(-1))
+    bnb4.quantize_4bit(x, 64, bnb4.FP4, True, state=st, workspace=ws)  # warm
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s), torch.cuda.graph(g, stream=s):
+        bnb4.quantize_4bit(x, 64, bnb4.FP4, True, state=st, workspace=ws)
+    torch.cuda.current_stream().wait_stream(s)
+    for seed in (21, 22, 23):
+        src = synth.weight_bf16(4096, 1024, seed=seed, outlier_frac=synth.OUTLIER_FRAC)
+        x.copy_(src.view(-1))
+        g.replay()
+        torch.cuda.synchronize()
+        _check_dq(st, src.view(-1), qtype=bnb4.FP4)
+    del g
