@@ -8,32 +8,30 @@
 // over the blockwise NF4 / FP4 format of the CSDN article (section
 // "数学原理对比"), nested (double) quantization decoded in-kernel.
 //
-// Design (bound by the packed-byte stream from HBM and by instruction issue):
-//  * Persistent grid, one CTA per SM; each CTA owns a contiguous, balanced
-//    range of 16-row groups.  A work item is 16 rows x 256 K (2 KB of codes):
-//    lane (g, t) of a warp owns rows g and g + 8 and the 64-element K segment
-//    t of the item.
-//  * Every consumer warp streams its items through a private ring of
-//    shared-memory stages filled by cp.async, several items ahead.  Each lane
-//    copies exactly the 2 x 32 code bytes and the scale words it later reads,
-//    so completion is tracked per thread (cp.async.wait_group) and no lane
-//    waits on another; the HBM latency is hidden without holding loads in
-//    registers.
-//  * Split-K mode (K of at least one item per consumer warp): the CTA's items
-//    are its (row group, K chunk) pairs in row-major order, dealt to the
-//    warps round-robin; a warp sums its chunks of a row group in registers
-//    and hands the partial sums to a reducer warp through a double-buffered
-//    shared-memory slot (named barriers FULL / EMPTY).  The reducer adds them
-//    in warp order -- a fixed order, so results are bit-reproducible --,
-//    adds the bias and stores y.  Short K: each warp takes whole row groups
-//    and stores y itself.
+// Design.  The exact table lookup costs about 2.5 integer-ALU operations per
+// weight (byte permutes run at half the FMA rate), so on B200 the kernel is
+// bound by the ALU pipe before HBM; everything else is kept off the
+// per-weight path.
+//  * Persistent grid, one CTA of 16 warps per SM; each CTA owns a balanced,
+//    contiguous range of 16-row groups.  A work item is 16 rows x 256 K (2 KB
+//    of codes); lane (g, t) of a warp owns rows g and g + 8 and the
+//    64-element K segment t of the item.
+//  * The CTA's items, in row-major order (row group, K chunk), are cut into
+//    16 contiguous runs, one per warp.  A warp sums each row group it covers
+//    in registers and stores it; only a row group that two or more warps
+//    share (at most one per run boundary) goes through shared memory, added
+//    after one barrier at the end in warp order -- a fixed order, so results
+//    are bit-reproducible for a given problem list and SM count.
+//  * Each warp streams its run through a private 4-stage ring: lane 0 starts
+//    a 2-D TMA copy of the code tile (128-byte swizzle) on the stage's
+//    mbarrier, the lanes copy the words holding their blocks' scales with
+//    cp.async, four items ahead of the math.
 //  * Dequantization by byte permutes (lut.cuh): per (row, quant block) a lane
 //    builds the 16-entry table of h(RN(t[i] * a_hat)), bit-identical to
 //    dequantizing every element.  Products on mma.sync m16n8k16 (weights as
-//    the A operand, 16 rows; x as B, batch columns): one 128-bit load of x
-//    feeds two MMAs, and K is permuted identically in both operands, which
-//    leaves the dot products unchanged.  Batch columns beyond B read a valid
-//    row whose outputs are never stored.
+//    the A operand, 16 rows; x as B, batch columns): K is permuted
+//    identically in both operands, which leaves the dot products unchanged.
+//    Lanes of batch columns beyond B hold zeros and load nothing.
 #include "common.cuh"
 #include "kernels.h"
 #include "lut.cuh"
@@ -42,31 +40,25 @@
 namespace bnb4 {
 namespace {
 
-constexpr int kConsumers = 16;                    // warps per CTA
-constexpr int kThreads = kConsumers * 32;
+constexpr int kWarps = 16;                        // warps per CTA
+constexpr int kThreads = kWarps * 32;
 constexpr int kStages = 4;                        // ring depth per warp
 constexpr int kRows = 16;                         // rows of an item (MMA M)
 constexpr int kItemK = 256;                       // K of an item (4 lanes x 64)
 
 constexpr int kTileBytes = kRows * kItemK / 2;    // packed codes of one item: 2 KB
 
-// Per consumer warp, a ring of kStages items: the code tile (16 rows x 128
-// bytes, written by TMA with the 128-byte swizzle: 16-byte chunk c of row r
-// sits at chunk c ^ (r & 7)), the lane-major scale words (each lane copies
-// the words it reads), and the tile's "full" mbarrier.
+// Per warp, a ring of kStages items: the code tile (16 rows x 128 bytes,
+// written by TMA with the 128-byte swizzle: 16-byte chunk c of row r sits at
+// chunk c ^ (r & 7)), the lane-major scale words and the tile's "full"
+// mbarrier; and the warp's partial sums of the (at most two) row groups it
+// shares with its neighbours.
 struct Smem {
-  uint8_t tiles[kConsumers][kStages][kTileBytes];
-  uint32_t sc[kConsumers][kStages][4][32];  // dq: [u word g, u word g+8, scale2 g, scale2 g+8]
-                                            // else [absmax g, absmax g+8, next g, next g+8]
-  // per item and lane, written by the fetching lane and read back by the
-  // same lane when it computes the item: {row group, problem, K offset of
-  // the lane's segment, flags: row g ok, row g + 8 ok, byte of u in each
-  // scale word}
-  int4 rec[kConsumers][kStages][32];
-  float4 red[2][kConsumers][32];            // partial sums of two row groups in flight
-  uint64_t full[kConsumers][kStages];
-  int arrived[2];  // warps that deposited their partials in slot s
-  int reduced[2];  // the CTA-local row group last reduced out of slot s
+  uint8_t tiles[kWarps][kStages][kTileBytes];
+  uint32_t sc[kWarps][kStages][4][32];  // dq: [u word g, u word g+8, scale2 g, scale2 g+8]
+                                        // else [absmax g, absmax g+8, next g, next g+8]
+  float4 part[2][kWarps][32];           // [0]: the warp's first row group, [1]: its last
+  uint64_t full[kWarps][kStages];
 };
 constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + alignment of the tiles
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -132,20 +124,6 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-// Bounded wait until a shared-memory word equals `want` (set by another warp
-// of the CTA); on expiry the device error word is set and the caller goes
-// on, so nothing hangs.
-__device__ __forceinline__ void wait_word(const int* word, int want, int* err) {
-  if (*reinterpret_cast<const volatile int*>(word) == want) return;
-  const uint64_t t0 = global_ns();
-  while (*reinterpret_cast<const volatile int*>(word) != want) {
-    if (global_ns() - t0 > kWaitLimitNs) {
-      atomicExch(err, 1);
-      return;
-    }
-    __nanosleep(32);
-  }
-}
 
 // D[16 x 8] += A[16 x 16] (weight rows) * B[16 x 8] (x columns), bf16 or
 // fp16 in (format F), fp32 accumulate.
@@ -204,81 +182,80 @@ __device__ __forceinline__ void store_rows(const float4& v, int rl, int lane, co
   }
 }
 
-// The item sequence of one consumer warp and the copies of each item.  All
-// state is 32-bit except the block index; advancing costs a few integer
-// operations, a new row group a few more, a new problem a handful of
-// parameter loads.
+// A position in a CTA's item sequence: global row group rg, K chunk kc and
+// the problem p that rg belongs to.  Stepping costs an increment and a
+// compare, a new row group one more compare, a new problem one parameter
+// load.
+template <int MAXP>
+struct Pos {
+  int rg, kc, p, next_rg0;
+  __device__ void seek(const Group<MAXP>& grp, int rg_, int kc_, int p_from) {
+    rg = rg_;
+    kc = kc_;
+    p = p_from;
+    while (p + 1 < grp.count && rg >= grp.p[p + 1].rg0) ++p;
+    next_rg0 = p + 1 < grp.count ? grp.p[p + 1].rg0 : 0x7fffffff;
+  }
+  // to the next item; true when that item begins a new row group
+  __device__ bool step(const Group<MAXP>& grp) {
+    if (++kc < grp.C) return false;
+    kc = 0;
+    if (++rg >= next_rg0) {
+      ++p;
+      next_rg0 = p + 1 < grp.count ? grp.p[p + 1].rg0 : 0x7fffffff;
+    }
+    return true;
+  }
+};
+
+// The copies of one warp's run of items, issued kStages items ahead of the
+// math: lane 0 arms the stage's barrier and starts the TMA of the code tile;
+// every lane copies the words holding its two rows' block scales.  Rows past
+// N and segments past K copy no scales (the TMA fills their codes with
+// zeros).
 template <int BS, bool DQ, int MAXP>
-struct Fetcher {
+struct Fetch {
   const Group<MAXP>& grp;
-  int lane, g, t;
-  bool split;
-  int nw;
-  int rg, rg_end, kc, p, rl, next_rg0;  // item (global row group, chunk), problem
-  int64_t blk0;                         // block of row g at k = 0
-  bool ok0, ok1, last;                  // rows g, g + 8 exist; last row group
+  int lane, t;
   // double quant with blocksize >= 64 and K % 256 == 0: the blocks of one
   // row of an item lie in one aligned 4-byte word of absmax_q and one scale2
   // group, so the 4 lanes of a quad copy their two rows' words together
   // (lane t: t = 0 the u word of row g, 1 of row g + 8, 2 / 3 their scale2)
   bool quad_sc;
+  Pos<MAXP> pos;
+  int left;             // items not yet issued
+  int row0;             // first row of the row group within its problem
+  int64_t blk0;         // block of row g at k = 0
+  bool ok0, ok1, last;  // rows g, g + 8 exist; the problem's last row group
 
-  __device__ Fetcher(const Group<MAXP>& gp, int lane_, bool split_, int nw_, int warp,
-                     int rg_begin, int rg_end_, int p_begin)
-      : grp(gp), lane(lane_), g(lane_ >> 2), t(lane_ & 3), split(split_), nw(nw_),
-        rg_end(rg_end_) {
+  __device__ Fetch(const Group<MAXP>& gp, int lane_, const Pos<MAXP>& start, int count)
+      : grp(gp), lane(lane_), t(lane_ & 3), pos(start), left(count) {
     quad_sc = DQ && BS >= 64 && grp.K % kItemK == 0;
-    rg = split ? rg_begin : rg_begin + warp;
-    kc = split ? warp : 0;
-    p = p_begin;
-    set_problem();
-    set_row_group();
+    enter();
   }
-  __device__ void set_problem() {
-    while (p + 1 < grp.count && rg >= grp.p[p + 1].rg0) ++p;
-    next_rg0 = p + 1 < grp.count ? grp.p[p + 1].rg0 : grp.n_rg;
-  }
-  __device__ void set_row_group() {
-    rl = rg - grp.p[p].rg0;
-    const int n0 = rl * kRows + g;
-    const int N = grp.p[p].N;
+  __device__ void enter() {
+    const Prob& a = grp.p[pos.p];
+    row0 = (pos.rg - a.rg0) * kRows;
+    const int n0 = row0 + (lane >> 2);
     blk0 = static_cast<int64_t>(n0) * grp.kb;
-    ok0 = n0 < N;
-    ok1 = n0 + 8 < N;
-    last = (rl + 1) * kRows >= N;
-  }
-  __device__ bool valid() const { return rg < rg_end; }
-  __device__ void advance() {
-    if (split) {
-      kc += nw;
-      if (kc < grp.C) return;
-      kc -= grp.C;
-      ++rg;
-    } else {
-      if (++kc < grp.C) return;
-      kc = 0;
-      rg += nw;
-    }
-    if (rg >= rg_end) return;
-    if (rg >= next_rg0) set_problem();
-    set_row_group();
+    ok0 = n0 < a.N;
+    ok1 = n0 + 8 < a.N;
+    last = row0 + kRows >= a.N;
   }
 
-  // lane 0 arms the stage's barrier and starts the TMA of the code tile;
-  // every lane copies the words holding its two rows' block scales and
-  // writes the item's record.  Rows past N and segments past K copy no
-  // scales (the TMA fills their codes with zeros).
-  __device__ void issue(uint8_t* tile, uint32_t* sc, int4* rec, uint32_t full) const {
+  __device__ void issue(uint8_t* tile, uint32_t* sc, uint32_t full) {
+    if (left == 0) return;
+    --left;
     if (lane == 0) {
       mbar_arrive_expect_tx(full, kTileBytes);
-      tma_load_2d(smem_u32(tile), &grp.maps[p], kc * (kItemK / 2), rl * kRows, full);
+      tma_load_2d(smem_u32(tile), &grp.maps[pos.p], pos.kc * (kItemK / 2), row0, full);
     }
-    const int koff = kc * kItemK + 64 * t;  // the lane's K segment
+    const int koff = pos.kc * kItemK + 64 * t;  // the lane's K segment
     const bool seg = koff < grp.K;
     const bool v0 = seg && ok0, v1 = seg && ok1;
     const int64_t b0 = blk0 + koff / BS;
     const int64_t b1 = b0 + static_cast<int64_t>(8) * grp.kb;
-    const Prob& a = grp.p[p];
+    const Prob& a = grp.p[pos.p];
     if (quad_sc) {
       const int r = t & 1;  // the row this lane copies a word of
       if (r ? v1 : v0) {
@@ -286,9 +263,9 @@ struct Fetcher {
         if (t < 2) {
           const int64_t wb = b & ~int64_t(3);
           if (last) {
-            const int64_t left = a.nb - wb;
+            const int64_t rest = a.nb - wb;
             cp_async4_part(smem_u32(sc + lane), a.absmax_q + wb,
-                           static_cast<uint32_t>(left < 4 ? left : 4));
+                           static_cast<uint32_t>(rest < 4 ? rest : 4));
           } else {
             cp_async4(smem_u32(sc + lane), a.absmax_q + wb);
           }
@@ -296,34 +273,32 @@ struct Fetcher {
           cp_async4(smem_u32(sc + lane), a.scale2 + (b >> 8));
         }
       }
-    }
+    } else {
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      if (quad_sc || !(r ? v1 : v0)) continue;
-      const int64_t b = r ? b1 : b0;
-      if constexpr (DQ) {
-        // the aligned 4-byte word holding u_b (and u_{b+1} at blocksize 32:
-        // b is even), cut at the end of the array in the last row group
-        const int64_t wb = b & ~int64_t(3);
-        if (last) {
-          const int64_t left = a.nb - wb;
-          cp_async4_part(smem_u32(sc + r * 32 + lane), a.absmax_q + wb,
-                         static_cast<uint32_t>(left < 4 ? left : 4));
+      for (int r = 0; r < 2; ++r) {
+        if (!(r ? v1 : v0)) continue;
+        const int64_t b = r ? b1 : b0;
+        if constexpr (DQ) {
+          // the aligned 4-byte word holding u_b (and u_{b+1} at blocksize
+          // 32: b is even), cut at the end of the array in the last row group
+          const int64_t wb = b & ~int64_t(3);
+          if (last) {
+            const int64_t rest = a.nb - wb;
+            cp_async4_part(smem_u32(sc + r * 32 + lane), a.absmax_q + wb,
+                           static_cast<uint32_t>(rest < 4 ? rest : 4));
+          } else {
+            cp_async4(smem_u32(sc + r * 32 + lane), a.absmax_q + wb);
+          }
+          cp_async4(smem_u32(sc + (2 + r) * 32 + lane), a.scale2 + (b >> 8));
         } else {
-          cp_async4(smem_u32(sc + r * 32 + lane), a.absmax_q + wb);
+          cp_async4(smem_u32(sc + r * 32 + lane), a.absmax + b);
+          if constexpr (BS == 32) cp_async4(smem_u32(sc + (2 + r) * 32 + lane), a.absmax + b + 1);
         }
-        cp_async4(smem_u32(sc + (2 + r) * 32 + lane), a.scale2 + (b >> 8));
-      } else {
-        cp_async4(smem_u32(sc + r * 32 + lane), a.absmax + b);
-        if constexpr (BS == 32) cp_async4(smem_u32(sc + (2 + r) * 32 + lane), a.absmax + b + 1);
       }
     }
-    const int flags = (v0 ? 1 : 0) | (v1 ? 2 : 0) | (static_cast<int>(b0 & 3) << 4) |
-                      (static_cast<int>(b1 & 3) << 8);
-    *rec = make_int4(rg, p, koff, flags);
+    if (pos.step(grp)) enter();
   }
 };
-
 // Decoded scale of a block from its staged words (u at byte `sh` of the u
 // word); 0 for an invalid row / segment (its products are then 0 or
 // discarded).
@@ -349,200 +324,183 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw + (((raw + 1023u) & ~1023u) - raw));
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int rg_begin = static_cast<int>(static_cast<int64_t>(grp.n_rg) * blockIdx.x / gridDim.x);
-  const int rg_end = static_cast<int>(static_cast<int64_t>(grp.n_rg) * (blockIdx.x + 1) / gridDim.x);
-  const int R = rg_end - rg_begin;
-  int p_begin = 0;
-  while (p_begin + 1 < grp.count && rg_begin >= grp.p[p_begin + 1].rg0) ++p_begin;
-  // Split K over nw consumer warps when the CTA has fewer row groups than
-  // warps; else whole row groups per warp (no hand-over at all).  nw <= C in
-  // split mode, so a warp's consecutive items are at most one row group
-  // apart and every warp contributes to every row group.
-  const bool split_k = R < kConsumers;
-  const int nw = split_k ? (grp.C < kConsumers ? grp.C : kConsumers) : kConsumers;
-  if (threadIdx.x == 0) {
-    sm.arrived[0] = sm.arrived[1] = 0;
-    sm.reduced[0] = -2;  // slot s first holds row group s
-    sm.reduced[1] = -1;
-  }
-  __syncthreads();
-  if (warp >= nw) return;
-
   const int g = lane >> 2, t = lane & 3;
-  uint64_t* full = sm.full[warp];
-  if (lane == 0) {
-    for (int d = 0; d < kStages; ++d) mbar_init(smem_u32(&full[d]), 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncwarp();
+  const int C = grp.C;
+  const int rb = static_cast<int>(static_cast<int64_t>(grp.n_rg) * blockIdx.x / gridDim.x);
+  const int re = static_cast<int>(static_cast<int64_t>(grp.n_rg) * (blockIdx.x + 1) / gridDim.x);
+  const int64_t items = static_cast<int64_t>(re - rb) * C;
+  // warp w's run of the CTA's items is [run(w), run(w + 1))
+  auto run = [&](int w) { return static_cast<int>(items * w / kWarps); };
+  const int i0 = run(warp), i1 = run(warp + 1);
+  const int cnt = i1 - i0;
+  int p_begin = 0;
+  while (p_begin + 1 < grp.count && rb >= grp.p[p_begin + 1].rg0) ++p_begin;
 
-  Fetcher<BS, DQ, MAXP> f(grp, lane, split_k, nw, warp, rg_begin, rg_end, p_begin);
-#pragma unroll
-  for (int d = 0; d < kStages; ++d) {
-    if (f.valid()) {
-      f.issue(sm.tiles[warp][d], &sm.sc[warp][d][0][0], &sm.rec[warp][d][lane],
-              smem_u32(&full[d]));
-      f.advance();
-    } else {
-      sm.rec[warp][d][lane] = make_int4(rg_end, 0, 0, 0);  // end marker
+  if (cnt > 0) {
+    uint64_t* full = sm.full[warp];
+    if (lane == 0) {
+      for (int d = 0; d < kStages; ++d) mbar_init(smem_u32(&full[d]), 1);
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    cp_async_commit();
-  }
-
-  float acc[2][4] = {};
-  int cur_rg = -1, cur_p = -1;
-  float off = 0.0f;
-  const uint16_t* xrow = nullptr;
-  const uint32_t k16 = grp.k16, k31 = grp.k31;
-  const bool quad_sc = f.quad_sc;
-  // split K with one chunk per warp per row group: the warp's chunk, hence
-  // its slice of x, never changes -- it is loaded once per problem
-  const bool x_fixed = split_k && grp.C == nw;
-  uint4 xb[8];
-
-  // Split K: the partial sums of CTA-local row group r go to slot r & 1; the
-  // warp that deposits last adds the nw partials in warp order (a fixed
-  // order: bit-reproducible), stores y, empties the slot and marks row group
-  // r reduced, which frees the slot for row group r + 2.
-  auto flush = [&]() {
-    const float4 v = make_float4(acc[0][0] + acc[1][0], acc[0][1] + acc[1][1],
-                                 acc[0][2] + acc[1][2], acc[0][3] + acc[1][3]);
-    if (split_k) {
-      const int r = cur_rg - rg_begin;
-      const int s = r & 1;
-      if (r >= 2) {  // the slot's previous row group has been reduced
-        if (lane == 0) wait_word(&sm.reduced[s], r - 2, grp.err);
-        __syncwarp();
-        __threadfence_block();
-      }
-      sm.red[s][warp][lane] = v;
-      __threadfence_block();
-      __syncwarp();
-      int before = 0;
-      if (lane == 0) before = atomicAdd(&sm.arrived[s], 1);
-      before = __shfl_sync(0xffffffffu, before, 0);
-      if (before == nw - 1) {  // the last to deposit: reduce
-        __threadfence_block();
-        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int w = 0; w < nw; ++w) {
-          const float4 q = sm.red[s][w][lane];
-          sum.x += q.x;
-          sum.y += q.y;
-          sum.z += q.z;
-          sum.w += q.w;
-        }
-        store_rows<F>(sum, cur_rg - grp.p[cur_p].rg0, lane, grp.p[cur_p], grp.B);
-        __threadfence_block();
-        __syncwarp();
-        if (lane == 0) {
-          sm.arrived[s] = 0;
-          __threadfence_block();
-          *reinterpret_cast<volatile int*>(&sm.reduced[s]) = r;
-        }
-      }
-    } else {
-      store_rows<F>(v, cur_rg - grp.p[cur_p].rg0, lane, grp.p[cur_p], grp.B);
-    }
-#pragma unroll
-    for (int c = 0; c < 2; ++c)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[c][e] = 0.f;
-  };
-
-  // items in the order they were issued; the ring holds the next kStages
-  for (int j = 0;; ++j) {
-    const int d = j & (kStages - 1);
-    const int4 rec = sm.rec[warp][d][lane];  // written by this lane
-    if (rec.x >= rg_end) break;              // the end marker
-    if (rec.x != cur_rg) {
-      if (cur_rg >= 0) flush();
-      if (rec.y != cur_p) {  // per-problem values
-        const Prob& a = grp.p[rec.y];
-        off = DQ ? __ldg(a.offset) : 0.0f;
-        xrow = a.x + static_cast<int64_t>(g < grp.B ? g : grp.B - 1) * grp.K;
-        cur_p = rec.y;
-        if (x_fixed) {  // (a segment past a ragged K reads no x)
-          const bool in_k = rec.z < grp.K;
-          const uint4* xs = reinterpret_cast<const uint4*>(xrow + (in_k ? rec.z : 0));
-#pragma unroll
-          for (int p = 0; p < 8; ++p) xb[p] = in_k ? __ldg(xs + p) : make_uint4(0, 0, 0, 0);
-        }
-      }
-      cur_rg = rec.x;
-    }
-    wait_tile(smem_u32(&full[d]), static_cast<uint32_t>(j / kStages) & 1u, grp.err);
-    cp_async_wait<kStages - 1>();  // this lane's scale copies of item j have landed
-    // rows g and g + 8, 16-byte chunks 2t and 2t + 1 (swizzled by row & 7 = g)
-    const uint8_t* tile = sm.tiles[warp][d];
-    uint4 c[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      c[q] = *reinterpret_cast<const uint4*>(tile + (g + 8 * (q >> 1)) * 128 +
-                                             (((2 * t + (q & 1)) ^ g) << 4));
-    uint32_t sw[4];
-    if (quad_sc) {
-      __syncwarp();  // the quad-mates' scale copies (each waited above) are visible
-#pragma unroll
-      for (int q = 0; q < 4; ++q) sw[q] = sm.sc[warp][d][0][(lane & ~3) | q];
-    } else {
-#pragma unroll
-      for (int q = 0; q < 4; ++q) sw[q] = sm.sc[warp][d][q][lane];
-    }
-    const int koff = rec.z;
-    const bool ok0 = rec.w & 1, ok1 = rec.w & 2;
-    const bool seg = koff < grp.K;
-    const int sh0 = (rec.w >> 4) & 3, sh1 = (rec.w >> 8) & 3;
-    const float a00 = scale_of<DQ>(sw[0], sw[2], sh0, off, ok0);
-    const float a10 = scale_of<DQ>(sw[1], sw[3], sh1, off, ok1);
-    float a01 = 0.f, a11 = 0.f;
-    if constexpr (BS == 32) {  // the segment's second block (b + 1: the next byte)
-      a01 = DQ ? scale_of<DQ>(sw[0], sw[2], sh0 + 1, off, ok0) : (ok0 ? __uint_as_float(sw[2]) : 0.f);
-      a11 = DQ ? scale_of<DQ>(sw[1], sw[3], sh1 + 1, off, ok1) : (ok1 ? __uint_as_float(sw[3]) : 0.f);
-    }
-
-    // refill this stage with the item kStages ahead once every lane's reads
-    // of it are done (the values above are in registers and used); the
-    // fence orders those shared-memory reads before the TMA's writes
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     __syncwarp();
-    if (f.valid()) {
-      f.issue(sm.tiles[warp][d], &sm.sc[warp][d][0][0], &sm.rec[warp][d][lane],
-              smem_u32(&full[d]));
-      f.advance();
-    } else {
-      sm.rec[warp][d][lane] = make_int4(rg_end, 0, 0, 0);  // end marker
-    }
-    cp_async_commit();
 
-    if (!x_fixed) {
-      const uint4* xs = reinterpret_cast<const uint4*>(xrow + (seg ? koff : 0));
+    Pos<MAXP> cp;  // the item the math is on
+    cp.seek(grp, rb + i0 / C, i0 % C, p_begin);
+    Fetch<BS, DQ, MAXP> f(grp, lane, cp, cnt);
 #pragma unroll
-      for (int p = 0; p < 8; ++p) xb[p] = seg ? __ldg(xs + p) : make_uint4(0, 0, 0, 0);
+    for (int d = 0; d < kStages; ++d) {
+      f.issue(sm.tiles[warp][d], &sm.sc[warp][d][0][0], smem_u32(&full[d]));
+      cp_async_commit();
     }
 
+    const uint32_t k16 = grp.k16, k31 = grp.k31;
+    const bool quad_sc = f.quad_sc;
+    // the row group being summed: its problem, row group within the problem,
+    // this lane's rows, decoded-scale offset, x row and block-index low bits
+    int cur_p = 0, rl = 0;
+    bool cok0 = false, cok1 = false;
+    float off = 0.0f;
+    const uint16_t* xrow = nullptr;
+    uint32_t blk_lo = 0;
+    auto enter = [&]() {
+      const Prob& a = grp.p[cp.p];
+      cur_p = cp.p;
+      rl = cp.rg - a.rg0;
+      const int n0 = rl * kRows + g;
+      cok0 = n0 < a.N;
+      cok1 = n0 + 8 < a.N;
+      off = DQ ? __ldg(a.offset) : 0.0f;
+      xrow = a.x + static_cast<int64_t>(g < grp.B ? g : 0) * grp.K;
+      blk_lo = static_cast<uint32_t>(n0) * static_cast<uint32_t>(grp.kb);
+    };
+    enter();
+    float acc[2][4] = {};
+    bool first = true;  // the row group is the run's first
+
+    for (int j = 0; j < cnt; ++j) {
+      const int d = j & (kStages - 1);
+      const int koff = cp.kc * kItemK + 64 * t;  // the lane's K segment
+      const bool seg = koff < grp.K;
+      // x of the segment (batch column g); columns past B stay zero
+      uint4 xb[8];
+      if (g < grp.B && seg) {
+        const uint4* xs = reinterpret_cast<const uint4*>(xrow + koff);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      // one table per (row, quant block): blocksize 32 switches at h = 1
-      Lut l0, l1;
-      if (BS == 32 && h == 1) {
-        l0 = make_lut<QT, F>(a01);
-        l1 = make_lut<QT, F>(a11);
+        for (int q = 0; q < 8; ++q) xb[q] = __ldg(xs + q);
       } else {
-        l0 = make_lut<QT, F>(a00);
-        l1 = make_lut<QT, F>(a10);
-      }
 #pragma unroll
-      for (int wi = 0; wi < 4; ++wi) {
-        const int p = 4 * h + wi;  // codes koff + 8p .. + 7 of both rows
-        const uint4 o0 = dq8_fma(l0, word(c[h], wi), k16, k31);
-        const uint4 o1 = dq8_fma(l1, word(c[2 + h], wi), k16, k31);
-        mma16<F>(acc[0], o0.x, o1.x, o0.y, o1.y, xb[p].x, xb[p].y);
-        mma16<F>(acc[1], o0.z, o1.z, o0.w, o1.w, xb[p].z, xb[p].w);
+        for (int q = 0; q < 8; ++q) xb[q] = make_uint4(0, 0, 0, 0);
+      }
+      wait_tile(smem_u32(&full[d]), static_cast<uint32_t>(j / kStages) & 1u, grp.err);
+      cp_async_wait<kStages - 1>();  // this lane's scale copies of item j have landed
+      // rows g and g + 8, 16-byte chunks 2t and 2t + 1 (swizzled by row & 7 = g)
+      const uint8_t* tile = sm.tiles[warp][d];
+      uint4 c[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        c[q] = *reinterpret_cast<const uint4*>(tile + (g + 8 * (q >> 1)) * 128 +
+                                               (((2 * t + (q & 1)) ^ g) << 4));
+      uint32_t sw[4];
+      if (quad_sc) {
+        __syncwarp();  // the quad-mates' scale copies (each waited above) are visible
+        const uint4 v = *reinterpret_cast<const uint4*>(&sm.sc[warp][d][0][lane & ~3]);
+        sw[0] = v.x;
+        sw[1] = v.y;
+        sw[2] = v.z;
+        sw[3] = v.w;
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) sw[q] = sm.sc[warp][d][q][lane];
+      }
+      // byte of u in each staged word: the block index mod 4
+      const uint32_t bl = blk_lo + static_cast<uint32_t>(koff / BS);
+      const int sh0 = static_cast<int>(bl & 3u);
+      const int sh1 = static_cast<int>((bl + 8u * static_cast<uint32_t>(grp.kb)) & 3u);
+      const float a00 = scale_of<DQ>(sw[0], sw[2], sh0, off, seg && cok0);
+      const float a10 = scale_of<DQ>(sw[1], sw[3], sh1, off, seg && cok1);
+      float a01 = 0.f, a11 = 0.f;
+      if constexpr (BS == 32) {  // the segment's second block (b + 1: the next byte)
+        a01 = DQ ? scale_of<DQ>(sw[0], sw[2], sh0 + 1, off, seg && cok0)
+                 : (seg && cok0 ? __uint_as_float(sw[2]) : 0.f);
+        a11 = DQ ? scale_of<DQ>(sw[1], sw[3], sh1 + 1, off, seg && cok1)
+                 : (seg && cok1 ? __uint_as_float(sw[3]) : 0.f);
+      }
+
+      // refill this stage with the item kStages ahead once every lane's reads
+      // of it are done (the values above are in registers); the fence orders
+      // those shared-memory reads before the TMA's writes
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      f.issue(sm.tiles[warp][d], &sm.sc[warp][d][0][0], smem_u32(&full[d]));
+      cp_async_commit();
+
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        // one table per (row, quant block): blocksize 32 switches at h = 1
+        Lut l0, l1;
+        if (BS == 32 && h == 1) {
+          l0 = make_lut<QT, F>(a01);
+          l1 = make_lut<QT, F>(a11);
+        } else {
+          l0 = make_lut<QT, F>(a00);
+          l1 = make_lut<QT, F>(a10);
+        }
+#pragma unroll
+        for (int wi = 0; wi < 4; ++wi) {
+          const int p = 4 * h + wi;  // codes koff + 8p .. + 7 of both rows
+          const uint4 o0 = dq8_fma(l0, word(c[h], wi), k16, k31);
+          const uint4 o1 = dq8_fma(l1, word(c[2 + h], wi), k16, k31);
+          mma16<F>(acc[0], o0.x, o1.x, o0.y, o1.y, xb[p].x, xb[p].y);
+          mma16<F>(acc[1], o0.z, o1.z, o0.w, o1.w, xb[p].z, xb[p].w);
+        }
+      }
+
+      // the end of a row group: store it, or leave it in shared memory when
+      // a neighbouring run holds part of it (the run's first row group when
+      // the run starts inside it, its last when the run ends inside it)
+      const bool more = j + 1 < cnt;
+      if (cp.step(grp) || !more) {
+        const float4 v = make_float4(acc[0][0] + acc[1][0], acc[0][1] + acc[1][1],
+                                     acc[0][2] + acc[1][2], acc[0][3] + acc[1][3]);
+        const bool shared = (first && i0 % C != 0) || (!more && i1 % C != 0);
+        if (shared)
+          sm.part[first ? 0 : 1][warp][lane] = v;
+        else
+          store_rows<F>(v, rl, lane, grp.p[cur_p], grp.B);
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[q][e] = 0.f;
+        first = false;
+        if (more) enter();
       }
     }
+    cp_async_wait<0>();
   }
-  cp_async_wait<0>();
-  if (cur_rg >= 0) flush();
+
+  // A shared row group is added up by the warp whose run holds its last
+  // item (then the row group is that run's first): the partial sums of the
+  // runs that hold part of it, in warp order.
+  __syncthreads();
+  if (cnt > 0 && i0 % C != 0 && i1 >= (i0 / C + 1) * C) {
+    const int lrg = i0 / C;  // the row group, CTA-local
+    int w_lo = warp - 1;     // the run holding its first item
+    while (run(w_lo) > lrg * C) --w_lo;
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int w = w_lo; w <= warp; ++w) {
+      const int a0 = run(w);
+      if (run(w + 1) == a0) continue;  // an empty run
+      const float4 q = sm.part[a0 / C == lrg ? 0 : 1][w][lane];
+      s.x += q.x;
+      s.y += q.y;
+      s.z += q.z;
+      s.w += q.w;
+    }
+    Pos<MAXP> rp;
+    rp.seek(grp, rb + lrg, 0, p_begin);
+    const Prob& a = grp.p[rp.p];
+    store_rows<F>(s, rb + lrg - a.rg0, lane, a, grp.B);
+  }
 }
 
 template <int BS, int QT, bool DQ, int F, int MAXP>

@@ -20,15 +20,14 @@ enum class Residency { kDevice, kDeviceOrManaged, kDeviceOrPinnedHost };
 // memory `where` excludes).  Host-only; launches nothing.
 int resolve_ptr(const void* p, Residency where, const void** dev);
 
-// Upper bound on the quantize grid.  The double-quant workspace holds a call
-// counter and, per CTA, a tag and an fp64 partial sum of its blocks' absmax
-// (8-byte words: counter at 0, tags from 8, sums from 8 + kMaxPartials).
+// Upper bound on the quantize grid.  The double-quant workspace holds one
+// fp64 partial sum of the blocks' absmax per CTA.
 constexpr int kMaxPartials = 4096;
-constexpr size_t kDqWorkspaceBytes = 8 * (8 + 2 * static_cast<size_t>(kMaxPartials));
+constexpr size_t kDqWorkspaceBytes = sizeof(double) * static_cast<size_t>(kMaxPartials);
 
 int quant_grid(int64_t n, int x_dtype, int num_sms);
 // workspace: kDqWorkspaceBytes, 16-byte aligned (double quant only); err:
-// the device error word.  view: x is a row-major 2-D view with a row stride
+// the device error word (unused: the quantize kernels have no waits).  view: x is a row-major 2-D view with a row stride
 // (see View2D), or null for a contiguous x.
 cudaError_t launch_quantize(const void* x, int x_dtype, const bnb4_qstate& st,
                             void* workspace, int* err, int num_sms, cudaStream_t s,

@@ -32,15 +32,9 @@
 //     the nibble order of the byte layout, so no shifts or ors are needed.
 // Any other row group (zero, subnormal or huge absmax, infinities) and the
 // one ragged tile at the end take an exact out-of-line path with the
-// correctly rounded reciprocal and a clamped lookup.
-// Double quantization needs the mean of every block's absmax before any
-// 8-bit code can be formed: a grid-wide dependency.  The launch is
-// cooperative (every CTA resident at once), each CTA publishes the fp64 sum
-// of its blocks' absmax tagged with this call's number, waits -- bounded in
-// time -- until every CTA's tag carries it, forms the mean from the partial
-// sums in one fixed order (every CTA alike, so they agree bit for bit) and
-// double-quantizes its share of the 256-block groups.  No second kernel, no
-// launch gap, no cold restart.
+// correctly rounded reciprocal and a clamped lookup.  The double
+// quantization runs as a second, tiny kernel that first reduces the per-CTA
+// fp64 partial sums in a fixed order.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -299,128 +293,11 @@ __device__ __noinline__ void chunk_exact(uint4 ch, float m, int64_t e, int64_t n
 // STR: x is a row-major [n / v.cols, v.cols] view with rows v.ld elements
 // apart (16-byte aligned rows, n < 2^32); blocks still run over the logical
 // element order, so the results equal those of the contiguous tensor.
-// Where the double quantization of a call goes.  ws: the caller's workspace
-// (or the allocation-free entry's scratch) -- word 0 counts the calls made
-// with it, words kTagsAt.. hold each CTA's tag, words kSumsAt.. each CTA's
-// fp64 partial sum.
-struct DqOut {
-  unsigned long long* ws;
-  uint8_t* absmax_q;
-  float* scale2;
-  float* offset;
-  int* err;  // the library's device error word (set when the wait expires)
-};
-constexpr int kTagsAt = 8;
-constexpr int kSumsAt = kTagsAt + kMaxPartials;
-static_assert(kDqWorkspaceBytes >= sizeof(unsigned long long) * (kSumsAt + kMaxPartials),
-              "workspace layout");
-constexpr uint64_t kDqWaitNs = 2000000000ull;  // bound of the grid-wide wait (2 s)
-
-__device__ __forceinline__ unsigned long long ld_relaxed(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release(unsigned long long* p, unsigned long long v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-__device__ __forceinline__ uint64_t now_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-// The double quantization of every block's absmax, once this CTA's partial
-// sum is published: wait until every CTA's tag carries this call's number,
-// sum the partials in a fixed order (thread i adds partials i, i + 256, ...,
-// a fixed xor tree per warp, then the warp sums in order -- identical in
-// every CTA), then one warp per 256-block group (grid-strided).  The sum is
-// exact whenever the absmax values span few enough binades, and then equals
-// the sequential fp64 sum.
-__device__ __noinline__ void dq_tail(const float* __restrict__ absmax, int64_t nb,
-                                     const DqOut& dq, unsigned long long epoch) {
-  __shared__ double red[kThreads / 32];
-  __shared__ int ok_all;
-  const int lane = threadIdx.x & 31;
-  const int warp = threadIdx.x >> 5;
-  const unsigned long long* tags = dq.ws + kTagsAt;
-  const double* sums = reinterpret_cast<const double*>(dq.ws + kSumsAt);
-  if (warp == 0) {
-    // every lane reads its share of the tags with relaxed loads, all in
-    // flight at once (an acquire load would hold back the next one); the
-    // fence after the last round makes the loop an acquire of every tag
-    const uint64_t t0 = now_ns();
-    bool ok;
-    for (;;) {
-      bool mine = true;
-      for (int i = lane; i < static_cast<int>(gridDim.x); i += 32)
-        mine &= ld_relaxed(tags + i) == epoch;
-      if (__all_sync(0xffffffffu, mine)) {
-        ok = true;
-        break;
-      }
-      if (now_ns() - t0 > kDqWaitNs) {
-        ok = false;
-        break;
-      }
-      __nanosleep(64);
-    }
-    if (lane == 0) ok_all = ok;
-  }
-  __threadfence();
-  __syncthreads();
-  if (!ok_all) {  // a CTA never published its sum: report, write nothing
-    if (threadIdx.x == 0) atomicExch(dq.err, 1);
-    return;
-  }
-  double sum = 0.0;
-  for (int i = threadIdx.x; i < static_cast<int>(gridDim.x); i += kThreads) sum += __ldcg(sums + i);
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane == 0) red[warp] = sum;
-  __syncthreads();
-  sum = 0.0;
-#pragma unroll
-  for (int w = 0; w < kThreads / 32; ++w) sum += red[w];
-  const float off = static_cast<float>(sum / static_cast<double>(nb));
-  if (blockIdx.x == 0 && threadIdx.x == 0) dq.offset[0] = off;
-
-  const int64_t ng = (nb + 255) / 256;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * (kThreads / 32);
-  for (int64_t g = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + warp; g < ng;
-       g += stride) {
-    float c[8];
-    float m = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {  // entry g*256 + lane + 32 j (coalesced)
-      const int64_t b = g * 256 + lane + 32 * j;
-      c[j] = b < nb ? __fsub_rn(__ldcg(absmax + b), off) : 0.0f;
-      m = fmaxf(m, fabsf(c[j]));
-    }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    const float sg = __fdiv_rn(m, 127.0f);
-    if (lane == 0) dq.scale2[g] = sg;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int64_t b = g * 256 + lane + 32 * j;
-      if (b < nb) {
-        float q = 0.0f;
-        if (sg != 0.0f) q = fminf(fmaxf(rintf(__fdiv_rn(c[j], sg)), -127.0f), 127.0f);
-        dq.absmax_q[b] = static_cast<uint8_t>(static_cast<int>(q) + 128);
-      }
-    }
-  }
-  // every CTA read the call counter before publishing its tag, and all tags
-  // are in: advance it for the next call on this workspace
-  if (blockIdx.x == 0 && threadIdx.x == 0) dq.ws[0] = epoch;
-}
-
 template <typename T, int BS, int QT, bool DQ, bool STR>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     quant4_kernel(const T* __restrict__ x, int64_t n,
                   uint8_t* __restrict__ codes, float* __restrict__ absmax,
-                  DqOut dq, View2D v) {
+                  double* __restrict__ partials, View2D v) {
   constexpr int EPL = Elem<T>::kPerChunk;  // elements per 16-byte chunk
   constexpr int LPB = BS / EPL;            // lanes (chunks) per block
   constexpr int ROW = 32 * EPL;            // elements per warp row
@@ -431,9 +308,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
   extern __shared__ uint2 lut[];
   __shared__ double red[kThreads / 32];
-  __shared__ unsigned long long epoch;  // this call's number (double quant)
-  if (DQ && threadIdx.x == 0)
-    epoch = *reinterpret_cast<volatile unsigned long long*>(dq.ws) + 1;
+  pdl_trigger();  // the double-quant kernel may be scheduled early
   build_lut<QT>(lut);
   __syncthreads();
 
@@ -535,15 +410,70 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
     if (lane == 0) red[warp] = acc;
-    __syncthreads();  // also: every absmax store of this CTA is done
+    __syncthreads();
     if (threadIdx.x == 0) {
       double s = 0.0;
       for (int w = 0; w < kThreads / 32; ++w) s += red[w];
-      reinterpret_cast<double*>(dq.ws + kSumsAt)[blockIdx.x] = s;
-      __threadfence();
-      st_release(dq.ws + kTagsAt + blockIdx.x, epoch);
+      partials[blockIdx.x] = s;
     }
-    dq_tail(absmax, nb, dq, epoch);
+  }
+}
+
+// Double quantization of the absmax array: one warp per group of 256 blocks
+// (grid-strided over the groups).  Every CTA first reduces the per-CTA
+// partial sums of the quantize kernel in the same fixed order -- thread i
+// adds partials i, i + 256, ... (independent loads, one round trip), then a
+// fixed xor tree per warp and the 8 warp sums in order -- so all CTAs agree
+// on the offset; the sum is exact whenever the absmax values span few
+// enough binades, and then equals the oracle's sequential sum.
+constexpr int kDqThreads = 256;
+
+__global__ void __launch_bounds__(kDqThreads)
+    dq_absmax_kernel(const float* __restrict__ absmax, int64_t nb,
+                     const double* __restrict__ partials, int n_partials,
+                     uint8_t* __restrict__ absmax_q, float* __restrict__ scale2,
+                     float* __restrict__ offset) {
+  __shared__ double red[kDqThreads / 32];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  pdl_wait();  // the quantize kernel's absmax and partial sums are complete
+  double sum = 0.0;
+  for (int i = threadIdx.x; i < n_partials; i += kDqThreads) sum += partials[i];
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (lane == 0) red[warp] = sum;
+  __syncthreads();
+  sum = 0.0;
+#pragma unroll
+  for (int w = 0; w < kDqThreads / 32; ++w) sum += red[w];
+  const float off = static_cast<float>(sum / static_cast<double>(nb));
+  if (blockIdx.x == 0 && threadIdx.x == 0) offset[0] = off;
+
+  const int64_t ng = (nb + 255) / 256;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * (kDqThreads / 32);
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * (kDqThreads / 32) + warp; g < ng;
+       g += stride) {
+    float c[8];
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {  // entry g*256 + lane + 32 j (coalesced)
+      const int64_t b = g * 256 + lane + 32 * j;
+      c[j] = b < nb ? __fsub_rn(__ldg(absmax + b), off) : 0.0f;
+      m = fmaxf(m, fabsf(c[j]));
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    const float sg = __fdiv_rn(m, 127.0f);
+    if (lane == 0) scale2[g] = sg;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t b = g * 256 + lane + 32 * j;
+      if (b < nb) {
+        float q = 0.0f;
+        if (sg != 0.0f) q = fminf(fmaxf(rintf(__fdiv_rn(c[j], sg)), -127.0f), 127.0f);
+        absmax_q[b] = static_cast<uint8_t>(static_cast<int>(q) + 128);
+      }
+    }
   }
 }
 
@@ -582,79 +512,39 @@ __global__ void __launch_bounds__(256) check_rcp_kernel(unsigned long long* res)
   }
 }
 
-// Resident CTAs per SM of a kernel (cached per device): the cooperative
-// launch of the double-quantizing kernels may not exceed them.
-template <class K>
-int resident_per_sm(K kern, size_t smem) {
-  static int cache[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (cache[dev] == 0) {
-    int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, smem) !=
-            cudaSuccess)
-      return 0;
-    cache[dev] = nb;
-  }
-  return cache[dev];
-}
-
-template <typename T, int BS, int QT, bool DQ, bool STR>
-cudaError_t launch_quant_t(const void* x, int64_t n, uint8_t* codes, float* absmax,
-                           const DqOut& dq, int grid, int num_sms, const View2D& view,
-                           cudaStream_t s) {
-  auto kern = quant4_kernel<T, BS, QT, DQ, STR>;
-  const size_t smem = kLutEntries * 32 * sizeof(uint2);
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  if constexpr (DQ) {
-    const int per_sm = resident_per_sm(kern, smem);
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    if (grid > per_sm * num_sms) grid = per_sm * num_sms;
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  }
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(x), n, codes, absmax, dq, view);
-}
-
 template <typename T, int BS, int QT, bool DQ>
-cudaError_t launch_quant(const void* x, int64_t n, uint8_t* codes, float* absmax,
-                         const DqOut& dq, int grid, int num_sms, const View2D* view,
+cudaError_t launch_quant(const void* x, int64_t n, uint8_t* codes,
+                         float* absmax, double* partials, int grid, const View2D* view,
                          cudaStream_t s) {
+  const size_t smem = kLutEntries * 32 * sizeof(uint2);
   if (view)
-    return launch_quant_t<T, BS, QT, DQ, true>(x, n, codes, absmax, dq, grid, num_sms, *view, s);
-  return launch_quant_t<T, BS, QT, DQ, false>(x, n, codes, absmax, dq, grid, num_sms, View2D{},
-                                              s);
+    return launch_kernel(quant4_kernel<T, BS, QT, DQ, true>, dim3(grid), dim3(kThreads), smem,
+                         s, false, static_cast<const T*>(x), n, codes, absmax, partials, *view);
+  return launch_kernel(quant4_kernel<T, BS, QT, DQ, false>, dim3(grid), dim3(kThreads), smem, s,
+                       false, static_cast<const T*>(x), n, codes, absmax, partials, View2D{});
 }
 
 template <typename T, int QT, bool DQ>
-cudaError_t dispatch_bs(int bs, const void* x, int64_t n, uint8_t* codes, float* absmax,
-                        const DqOut& dq, int grid, int sms, const View2D* view,
+cudaError_t dispatch_bs(int bs, const void* x, int64_t n, uint8_t* codes,
+                        float* absmax, double* partials, int grid, const View2D* view,
                         cudaStream_t s) {
   switch (bs) {
-    case 32: return launch_quant<T, 32, QT, DQ>(x, n, codes, absmax, dq, grid, sms, view, s);
-    case 64: return launch_quant<T, 64, QT, DQ>(x, n, codes, absmax, dq, grid, sms, view, s);
-    case 128: return launch_quant<T, 128, QT, DQ>(x, n, codes, absmax, dq, grid, sms, view, s);
-    default: return launch_quant<T, 256, QT, DQ>(x, n, codes, absmax, dq, grid, sms, view, s);
+    case 32: return launch_quant<T, 32, QT, DQ>(x, n, codes, absmax, partials, grid, view, s);
+    case 64: return launch_quant<T, 64, QT, DQ>(x, n, codes, absmax, partials, grid, view, s);
+    case 128: return launch_quant<T, 128, QT, DQ>(x, n, codes, absmax, partials, grid, view, s);
+    default: return launch_quant<T, 256, QT, DQ>(x, n, codes, absmax, partials, grid, view, s);
   }
 }
 
 template <typename T>
-cudaError_t dispatch_q(int qt, bool dq_on, int bs, const void* x, int64_t n, uint8_t* codes,
-                       float* absmax, const DqOut& dq, int grid, int sms, const View2D* view,
-                       cudaStream_t s) {
+cudaError_t dispatch_q(int qt, bool dq, int bs, const void* x, int64_t n,
+                       uint8_t* codes, float* absmax, double* partials,
+                       int grid, const View2D* view, cudaStream_t s) {
   if (qt == kQtNF4)
-    return dq_on ? dispatch_bs<T, kQtNF4, true>(bs, x, n, codes, absmax, dq, grid, sms, view, s)
-                 : dispatch_bs<T, kQtNF4, false>(bs, x, n, codes, absmax, dq, grid, sms, view,
-                                                 s);
-  return dq_on ? dispatch_bs<T, kQtFP4, true>(bs, x, n, codes, absmax, dq, grid, sms, view, s)
-               : dispatch_bs<T, kQtFP4, false>(bs, x, n, codes, absmax, dq, grid, sms, view, s);
+    return dq ? dispatch_bs<T, kQtNF4, true>(bs, x, n, codes, absmax, partials, grid, view, s)
+              : dispatch_bs<T, kQtNF4, false>(bs, x, n, codes, absmax, partials, grid, view, s);
+  return dq ? dispatch_bs<T, kQtFP4, true>(bs, x, n, codes, absmax, partials, grid, view, s)
+            : dispatch_bs<T, kQtFP4, false>(bs, x, n, codes, absmax, partials, grid, view, s);
 }
 
 }  // namespace
@@ -684,18 +574,30 @@ int quant_grid(int64_t n, int x_dtype, int num_sms) {
 cudaError_t launch_quantize(const void* x, int x_dtype, const bnb4_qstate& st,
                             void* workspace, int* err, int num_sms, cudaStream_t s,
                             const View2D* view) {
-  const bool dq_on = st.double_quant != 0;
-  const DqOut dq{static_cast<unsigned long long*>(workspace), st.absmax_q, st.scale2,
-                 st.offset, err};
+  (void)err;  // no bounded waits here
+  const bool dq = st.double_quant != 0;
   const int grid = quant_grid(st.n, x_dtype, num_sms);
-  if (x_dtype == BNB4_F32)
-    return dispatch_q<float>(st.qtype, dq_on, st.blocksize, x, st.n, st.codes, st.absmax, dq,
-                             grid, num_sms, view, s);
-  if (x_dtype == BNB4_F16)
-    return dispatch_q<Half16>(st.qtype, dq_on, st.blocksize, x, st.n, st.codes, st.absmax, dq,
-                              grid, num_sms, view, s);
-  return dispatch_q<uint16_t>(st.qtype, dq_on, st.blocksize, x, st.n, st.codes, st.absmax, dq,
-                              grid, num_sms, view, s);
+  double* partials = static_cast<double*>(workspace);
+  cudaError_t e =
+      x_dtype == BNB4_F32
+          ? dispatch_q<float>(st.qtype, dq, st.blocksize, x, st.n, st.codes,
+                              st.absmax, partials, grid, view, s)
+      : x_dtype == BNB4_F16
+          ? dispatch_q<Half16>(st.qtype, dq, st.blocksize, x, st.n, st.codes,
+                               st.absmax, partials, grid, view, s)
+          : dispatch_q<uint16_t>(st.qtype, dq, st.blocksize, x, st.n, st.codes,
+                                 st.absmax, partials, grid, view, s);
+  if (e != cudaSuccess || !dq) return e;
+  const int64_t nb = (st.n + st.blocksize - 1) / st.blocksize;
+  const int64_t ng = (nb + 255) / 256;
+  const int64_t warps_per_cta = kDqThreads / 32;
+  int64_t g2 = (ng + warps_per_cta - 1) / warps_per_cta;
+  if (g2 > 2048) g2 = 2048;
+  // programmatic: its predecessor is always the quantize kernel just launched
+  return launch_kernel(dq_absmax_kernel, dim3(static_cast<unsigned>(g2)), dim3(kDqThreads),
+                       0, s, true, static_cast<const float*>(st.absmax), nb,
+                    static_cast<const double*>(partials), grid, st.absmax_q, st.scale2,
+                    st.offset);
 }
 
 }  // namespace bnb4

@@ -6,10 +6,10 @@
 // allocation, a loader working under a fixed device-memory budget, or a
 // latency-critical path where cudaMalloc (which may synchronize the device or
 // fail under memory pressure) is not acceptable.  This entry point keeps its
-// scratch -- the bookkeeping of the grid-wide mean of the block scales (a call
-// counter, per-CTA tags and fp64 partial sums) and the exact fp32 absmax of
-// every block, which double quantization consumes and nobody reads
-// afterwards -- in a fixed array in the library's own device memory instead.  The caller still passes the input and the outputs (codes,
+// scratch -- one fp64 partial sum per CTA for the mean of the block scales and
+// the exact fp32 absmax of every block, which double quantization consumes
+// and nobody reads afterwards -- in a fixed array in the library's own device
+// memory instead.  The caller still passes the input and the outputs (codes,
 // absmax_q, scale2, offset).
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -21,10 +21,9 @@
 
 namespace {
 
-// Scratch layout: the double quantization's bookkeeping (a call counter and,
-// per CTA, a tag and an fp64 partial sum: 64 KiB), then up to
+// Scratch layout: kMaxPartials fp64 partial sums (32 KiB), then up to
 // BNB4_NOALLOC_MAX_BLOCKS fp32 absmax values (4 MiB).  Every GPU that loads
-// the library holds this array until the process exits; it starts zeroed.
+// the library holds this array until the process exits.
 constexpr size_t kPartialsBytes = (bnb4::kDqWorkspaceBytes + 255) / 256 * 256;
 constexpr size_t kScratchBytes =
     kPartialsBytes + sizeof(float) * static_cast<size_t>(BNB4_NOALLOC_MAX_BLOCKS);
@@ -120,7 +119,7 @@ extern "C" BNB4_API int bnb_quantize_4bit_noalloc(const void* x, int32_t x_dtype
   int* err = nullptr;
   if ((rc = bnb4::device_error_word(&err)) != BNB4_OK) return rc;
 
-  bnb4_qstate s = *st;  // same kernel, with the intermediate absmax in scratch
+  bnb4_qstate s = *st;  // same kernels, with the intermediate absmax in scratch
   s.absmax = reinterpret_cast<float*>(scratch + kPartialsBytes);
   const cudaError_t e = bnb4::launch_quantize(xd, x_dtype, s, scratch, err, sms,
                                               static_cast<cudaStream_t>(stream));

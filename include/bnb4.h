@@ -146,15 +146,14 @@ BNB4_API int bnb4_query_sizes(int64_t n, int32_t blocksize, int32_t double_quant
  *              always; absmax_q, scale2 and offset when st->double_quant.
  *  workspace   device scratch of at least bnb4_query_sizes(...).workspace
  *              bytes, 16-byte aligned (may be NULL when the size is 0).
- *              Any contents on first use; between calls it keeps a call
- *              counter that the next call on it relies on, so do not write
- *              to it, and do not share one workspace between calls that
- *              may overlap on the GPU (different streams).
- * With double quantization the launch is cooperative (all of its CTAs are
- * resident at once): the grid-wide mean of the absmax is formed inside the
- * one kernel, each CTA waiting -- at most 2 s, after which it sets the
- * device error word (bnb4_device_status reports BNB4_ERR_DEVICE_TIMEOUT) and
- * leaves the double-quant outputs unwritten -- for the others' partial sums.
+ *              Any contents; every call overwrites what it reads.  Do not
+ *              share one workspace between calls that may overlap on the
+ *              GPU (different streams).
+ * With double quantization two kernels run: the quantize kernel (codes,
+ * absmax and one fp64 partial sum of the absmax per CTA), then, as a
+ * programmatic dependent launch of it, the double quantization (the mean of
+ * the partial sums in a fixed order, then the 8-bit codes of each group of
+ * 256 absmax).
  * Per block: a = max|x|; r = RN(1/a) (0 for a = 0); v = RN(x*r); code =
  * number of fp32 codebook midpoints RN(RN(t[i]+t[i+1])*0.5) strictly below v
  * (FP4: of magnitude midpoints below |v|, sign bit set for v < 0 with a
@@ -179,10 +178,9 @@ BNB4_API int bnb_quantize_4bit(const void* x, int32_t x_dtype, const bnb4_qstate
  * Same method and bit-identical results as bnb_quantize_4bit with
  * st->double_quant = 1, except that the exact fp32 absmax is not returned:
  * st->absmax is ignored (may be NULL) and the intermediate absmax and the
- * bookkeeping of the grid-wide mean (a call counter, per-CTA tags and fp64
- * partial sums) live in a fixed array in the library's own device memory
- * (64 KiB + 4 MiB per GPU that loads the library, held until the process
- * exits).  The caller passes x and the outputs codes, absmax_q,
+ * per-CTA fp64 partial sums of the grid-wide mean live in a fixed array in
+ * the library's own device memory (32 KiB + 4 MiB per GPU that loads the
+ * library, held until the process exits).  The caller passes x and the outputs codes, absmax_q,
  * scale2 and offset, with the alignment rules of bnb_quantize_4bit.
  *  - Limit: at most BNB4_NOALLOC_MAX_BLOCKS blocks (ceil(n / blocksize));
  *    larger inputs return BNB4_ERR_SCRATCH_LIMIT and launch nothing.
@@ -198,8 +196,7 @@ BNB4_API int bnb_quantize_4bit(const void* x, int32_t x_dtype, const bnb4_qstate
  *    return BNB4_ERR_CUDA when the device is out of memory: make it at
  *    start-up, before any stream capture on the device.
  *  - Every call shares the one array.  A call overwrites all of the scratch
- *    it reads except the call counter of its grid-wide mean, which each call
- *    advances, so no result carries over from the previous call; calls that
+ *    it reads, so no result carries over from the previous call; calls that
  *    overlap on the GPU (different streams) race on it and must be
  *    serialized by the caller.
  * Allocates nothing and calls no allocating routine.

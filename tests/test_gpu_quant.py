@@ -172,7 +172,7 @@ def test_fast_reciprocal_exhaustive():
     assert first & 0xffffffff == 0xffffffff
 
 
-# ---- the grid-wide mean of double quantization inside one cooperative kernel
+# ---- the grid-wide mean of double quantization: workspace reuse and replay
 
 
 def _bits(x):
@@ -187,9 +187,9 @@ def _check_dq(st, x, bs=64, qtype=bnb4.NF4):
 
 
 def test_workspace_reused_across_inputs_and_sizes():
-    """One workspace, calls of different sizes and data in a row: the call
-    counter each call advances keeps a call from taking another call's
-    partial sums."""
+    """One workspace, calls of different sizes and data in a row: no call
+    takes another call's partial sums (a smaller grid leaves stale sums
+    beyond its own, which it must not read)."""
     ws = None
     xs = [synth.weight_bf16(4096, 4096, seed=s, outlier_frac=synth.OUTLIER_FRAC).cuda().view(-1)
           for s in (1, 2)] + [synth.normal_f32((100003,), seed=3, std=0.02).cuda()]
