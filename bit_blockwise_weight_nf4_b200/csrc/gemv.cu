@@ -102,12 +102,6 @@ constexpr int kSmallGroup = 4;   // one GEMV, or q/k/v, gate/up
 constexpr int kLargeGroup = 32;  // a longer list is launched in parts of 32
 static_assert(sizeof(Group<kLargeGroup>) <= 32000, "kernel parameter space");
 
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
 __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
 }
@@ -227,6 +221,14 @@ struct Fetch {
   int row0;             // first row of the row group within its problem
   int64_t blk0;         // block of row g at k = 0
   bool ok0, ok1, last;  // rows g, g + 8 exist; the problem's last row group
+  // the problem's scale arrays
+  const uint8_t* aq;
+  const float* s2;
+  int64_t nb;
+  // quad_sc: the row this lane copies a word of (g + 8 (t & 1)), as the
+  // block at the start of the current chunk, and whether that row exists
+  int64_t qb;
+  bool qv;
 
   __device__ Fetch(const Group<MAXP>& gp, int lane_, const Pos<MAXP>& start, int count)
       : grp(gp), lane(lane_), t(lane_ & 3), pos(start), left(count) {
@@ -241,6 +243,11 @@ struct Fetch {
     ok0 = n0 < a.N;
     ok1 = n0 + 8 < a.N;
     last = row0 + kRows >= a.N;
+    aq = a.absmax_q;
+    s2 = a.scale2;
+    nb = a.nb;
+    qb = blk0 + static_cast<int64_t>(8 * (t & 1)) * grp.kb + pos.kc * (kItemK / BS);
+    qv = (t & 1) ? ok1 : ok0;
   }
 
   __device__ void issue(uint8_t* tile, uint32_t* sc, uint32_t full) {
@@ -250,55 +257,58 @@ struct Fetch {
       mbar_arrive_expect_tx(full, kTileBytes);
       tma_load_2d(smem_u32(tile), &grp.maps[pos.p], pos.kc * (kItemK / 2), row0, full);
     }
+    if (quad_sc) {
+      // one word per lane, no branches: t < 2 the aligned absmax_q word of
+      // its row (cut at the end of the array in the last row group), t >= 2
+      // the row's scale2; a missing row copies nothing (zero-fill)
+      const int64_t wb = qb & ~int64_t(3);
+      const void* src = t < 2 ? static_cast<const void*>(aq + wb)
+                              : static_cast<const void*>(s2 + (qb >> 8));
+      uint32_t bytes = 4;
+      if (t < 2 && last) {
+        const int64_t rest = nb - wb;
+        bytes = static_cast<uint32_t>(rest < 4 ? rest : 4);
+      }
+      if (!qv) {
+        bytes = 0;
+        src = s2;
+      }
+      cp_async4_part(smem_u32(sc + lane), src, bytes);
+      qb += kItemK / BS;
+      if (pos.step(grp)) enter();
+      return;
+    }
     const int koff = pos.kc * kItemK + 64 * t;  // the lane's K segment
     const bool seg = koff < grp.K;
     const bool v0 = seg && ok0, v1 = seg && ok1;
     const int64_t b0 = blk0 + koff / BS;
     const int64_t b1 = b0 + static_cast<int64_t>(8) * grp.kb;
-    const Prob& a = grp.p[pos.p];
-    if (quad_sc) {
-      const int r = t & 1;  // the row this lane copies a word of
-      if (r ? v1 : v0) {
-        const int64_t b = r ? b1 : b0;
-        if (t < 2) {
-          const int64_t wb = b & ~int64_t(3);
-          if (last) {
-            const int64_t rest = a.nb - wb;
-            cp_async4_part(smem_u32(sc + lane), a.absmax_q + wb,
-                           static_cast<uint32_t>(rest < 4 ? rest : 4));
-          } else {
-            cp_async4(smem_u32(sc + lane), a.absmax_q + wb);
-          }
-        } else {
-          cp_async4(smem_u32(sc + lane), a.scale2 + (b >> 8));
-        }
-      }
-    } else {
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        if (!(r ? v1 : v0)) continue;
-        const int64_t b = r ? b1 : b0;
-        if constexpr (DQ) {
-          // the aligned 4-byte word holding u_b (and u_{b+1} at blocksize
-          // 32: b is even), cut at the end of the array in the last row group
-          const int64_t wb = b & ~int64_t(3);
-          if (last) {
-            const int64_t rest = a.nb - wb;
-            cp_async4_part(smem_u32(sc + r * 32 + lane), a.absmax_q + wb,
-                           static_cast<uint32_t>(rest < 4 ? rest : 4));
-          } else {
-            cp_async4(smem_u32(sc + r * 32 + lane), a.absmax_q + wb);
-          }
-          cp_async4(smem_u32(sc + (2 + r) * 32 + lane), a.scale2 + (b >> 8));
+    for (int r = 0; r < 2; ++r) {
+      if (!(r ? v1 : v0)) continue;
+      const int64_t b = r ? b1 : b0;
+      if constexpr (DQ) {
+        // the aligned 4-byte word holding u_b (and u_{b+1} at blocksize 32:
+        // b is even), cut at the end of the array in the last row group
+        const int64_t wb = b & ~int64_t(3);
+        if (last) {
+          const int64_t rest = nb - wb;
+          cp_async4_part(smem_u32(sc + r * 32 + lane), aq + wb,
+                         static_cast<uint32_t>(rest < 4 ? rest : 4));
         } else {
-          cp_async4(smem_u32(sc + r * 32 + lane), a.absmax + b);
-          if constexpr (BS == 32) cp_async4(smem_u32(sc + (2 + r) * 32 + lane), a.absmax + b + 1);
+          cp_async4(smem_u32(sc + r * 32 + lane), aq + wb);
         }
+        cp_async4(smem_u32(sc + (2 + r) * 32 + lane), s2 + (b >> 8));
+      } else {
+        const float* am = grp.p[pos.p].absmax;
+        cp_async4(smem_u32(sc + r * 32 + lane), am + b);
+        if constexpr (BS == 32) cp_async4(smem_u32(sc + (2 + r) * 32 + lane), am + b + 1);
       }
     }
     if (pos.step(grp)) enter();
   }
 };
+
 // Decoded scale of a block from its staged words (u at byte `sh` of the u
 // word); 0 for an invalid row / segment (its products are then 0 or
 // discarded).
@@ -346,10 +356,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     Pos<MAXP> cp;  // the item the math is on
     cp.seek(grp, rb + i0 / C, i0 % C, p_begin);
+    // Only the first item's copies start now: with every warp's whole ring
+    // requested at once the first tiles would arrive last among them, and
+    // the math waits for a tile while the rest of the ring is no use yet.
+    // The other stages fill once the first tile is in (kStages - 1 empty
+    // copy groups after the first keep the count of groups committed after
+    // each item's at kStages - 1 when it is consumed).
     Fetch<BS, DQ, MAXP> f(grp, lane, cp, cnt);
+    f.issue(sm.tiles[warp][0], &sm.sc[warp][0][0][0], smem_u32(&full[0]));
 #pragma unroll
-    for (int d = 0; d < kStages; ++d) {
-      f.issue(sm.tiles[warp][d], &sm.sc[warp][d][0][0], smem_u32(&full[d]));
+    for (int d = 0; d < kStages; ++d) cp_async_commit();
+    wait_tile(smem_u32(&full[0]), 0u, grp.err);
+#pragma unroll
+    for (int e = 1; e < kStages; ++e) {
+      f.issue(sm.tiles[warp][e], &sm.sc[warp][e][0][0], smem_u32(&full[e]));
       cp_async_commit();
     }
 
@@ -370,26 +390,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       cok0 = n0 < a.N;
       cok1 = n0 + 8 < a.N;
       off = DQ ? __ldg(a.offset) : 0.0f;
-      xrow = a.x + static_cast<int64_t>(g < grp.B ? g : 0) * grp.K;
+      xrow = a.x + static_cast<int64_t>(g) * grp.K;  // read by lanes g < B only
       blk_lo = static_cast<uint32_t>(n0) * static_cast<uint32_t>(grp.kb);
     };
     enter();
     float acc[2][4] = {};
     bool first = true;  // the row group is the run's first
+    uint4 xb[8];        // lanes of batch columns past B keep these zeros
+#pragma unroll
+    for (int q = 0; q < 8; ++q) xb[q] = make_uint4(0, 0, 0, 0);
 
     for (int j = 0; j < cnt; ++j) {
       const int d = j & (kStages - 1);
       const int koff = cp.kc * kItemK + 64 * t;  // the lane's K segment
       const bool seg = koff < grp.K;
-      // x of the segment (batch column g); columns past B stay zero
-      uint4 xb[8];
-      if (g < grp.B && seg) {
-        const uint4* xs = reinterpret_cast<const uint4*>(xrow + koff);
+      // x of the segment (batch column g; a segment past K reads zeros)
+      if (g < grp.B) {
+        const uint4* xs = reinterpret_cast<const uint4*>(xrow + (seg ? koff : 0));
 #pragma unroll
-        for (int q = 0; q < 8; ++q) xb[q] = __ldg(xs + q);
-      } else {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) xb[q] = make_uint4(0, 0, 0, 0);
+        for (int q = 0; q < 8; ++q) xb[q] = seg ? __ldg(xs + q) : make_uint4(0, 0, 0, 0);
       }
       wait_tile(smem_u32(&full[d]), static_cast<uint32_t>(j / kStages) & 1u, grp.err);
       cp_async_wait<kStages - 1>();  // this lane's scale copies of item j have landed
@@ -484,17 +503,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (cnt > 0 && i0 % C != 0 && i1 >= (i0 / C + 1) * C) {
     const int lrg = i0 / C;  // the row group, CTA-local
-    int w_lo = warp - 1;     // the run holding its first item
-    while (run(w_lo) > lrg * C) --w_lo;
+    const int first_item = lrg * C;
+    // the run holding its first item: the largest w with run(w) <= first_item
+    const int w_lo =
+        static_cast<int>((static_cast<int64_t>(first_item + 1) * kWarps - 1) / items);
     float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    int a0 = run(w_lo);
     for (int w = w_lo; w <= warp; ++w) {
-      const int a0 = run(w);
-      if (run(w + 1) == a0) continue;  // an empty run
-      const float4 q = sm.part[a0 / C == lrg ? 0 : 1][w][lane];
-      s.x += q.x;
-      s.y += q.y;
-      s.z += q.z;
-      s.w += q.w;
+      const int a1 = run(w + 1);
+      if (a1 != a0) {  // (an empty run deposited nothing)
+        // a run that starts inside the row group deposited it as its first
+        const float4 q = sm.part[a0 >= first_item ? 0 : 1][w][lane];
+        s.x += q.x;
+        s.y += q.y;
+        s.z += q.z;
+        s.w += q.w;
+      }
+      a0 = a1;
     }
     Pos<MAXP> rp;
     rp.seek(grp, rb + lrg, 0, p_begin);
