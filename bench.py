@@ -71,7 +71,23 @@ GEMV_WEIGHTS = 4
 # DRAM bytes (read + write) per launch of a kernel family, from one ncu
 # capture each, with the sources hashed at capture time: a figure is
 # reported only while the kernel's sources are the ones that were captured.
+# integer-ALU operations per weight of the decode kernel's exact lookup: per
+# 8 weights 16 byte permutes and 2 selector masks, and per 64-weight block
+# table 8 permutes and 8 bf16 packs -- 2.25 + 0.25
+ALU_OPS_PER_WEIGHT = 2.5
+
 TRAFFIC = {
+    # decode: DRAM bytes of one cold 11008 x 4096 launch over its algorithmic
+    # bytes (23.92 MB / 23.27 MB); the family's traffic per launch is that
+    # ratio times its algorithmic bytes per launch
+    "gemv": {"ratio": 23.922944 / 23.27,
+             "launch": "one decode launch (11008 x 4096, B = 1, captured cold), scaled by "
+                       "the algorithmic bytes per launch of the family",
+             "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemv.cu",
+                         "bit_blockwise_weight_nf4_b200/csrc/lut.cuh",
+                         "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
+                         "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
+             "sha256": "48f088efe3b179273161613bcbc1f8564a7e529a6698eb352113d58c7a0858f7"},
     "gemm": {"bytes": 37468818,
              "launch": "one prefill GEMM launch, averaged over the seven Llama-7B linears",
              "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemm.cu",
@@ -712,13 +728,32 @@ def run_ours(args):
         psrc = "%s HBM copy bandwidth" % peaks["source"]
     roofline = {
         "bound": dom["bound"], "kernel": dom_name, "achieved": ach, "peak": peak,
-        "unit": unit, "frac": ach / peak, "traffic": tr["bytes"] if tr else None,
+        "unit": unit, "frac": ach / peak,
+        "traffic": (tr["bytes"] if "bytes" in tr else tr["ratio"] * dom["work"] / dom["launches"])
+                   if tr else None,
         "traffic_launch": tr["launch"] if tr else None,
         "peak_source": psrc,
         "per_launch": "algorithmic work of the %d launches per step of this family "
                       "over their summed event time" % dom["launches"],
         "share_of_step": dom["s"] / (elapsed_max / args.steps),
     }
+    if dom_name == "gemv":
+        # the decode kernel's own bound: the integer ALU pipe of its exact
+        # table lookup (16 byte permutes + 2 logic ops per 8 weights, and one
+        # permute + one pack per 8 weights for the per-block tables), 16
+        # lanes per cycle per SM sub-partition
+        weights = sum(2.0 * r.extra["weight_bytes"] * len(r.calls)
+                      for r in rows if r.family == "gemv" and "weight_bytes" in r.extra)
+        s_w = sum(per_call[r.name] * len(r.calls)
+                  for r in rows if r.family == "gemv" and "weight_bytes" in r.extra)
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        mhz = clk["sm_max_mhz"] if clk else 1965.0
+        alu_peak = sms * 4 * 16 * mhz * 1e6 / 1e12
+        alu_ach = weights * ALU_OPS_PER_WEIGHT / s_w / 1e12
+        roofline["alu"] = {"achieved": alu_ach, "peak": alu_peak, "unit": "T lane-op/s",
+                           "frac": alu_ach / alu_peak, "ops_per_weight": ALU_OPS_PER_WEIGHT,
+                           "peak_source": "%d SMs x 4 sub-partitions x 16 ALU lanes x %.0f MHz"
+                                          % (sms, mhz)}
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": warm,

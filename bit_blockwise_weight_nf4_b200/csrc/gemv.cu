@@ -98,7 +98,7 @@ struct Group {
   uint32_t k16, k31;  // 2^16 and 2^31, opaque to the compiler (see dq8_fma)
   int* err;           // the library's device error word
 };
-constexpr int kSmallGroup = 4;   // one GEMV, or q/k/v, gate/up
+constexpr int kSmallGroup = 4;   // q/k/v, gate/up (one GEMV: a group of 1)
 constexpr int kLargeGroup = 32;  // a longer list is launched in parts of 32
 static_assert(sizeof(Group<kLargeGroup>) <= 32000, "kernel parameter space");
 
@@ -186,17 +186,24 @@ struct Pos {
   __device__ void seek(const Group<MAXP>& grp, int rg_, int kc_, int p_from) {
     rg = rg_;
     kc = kc_;
-    p = p_from;
-    while (p + 1 < grp.count && rg >= grp.p[p + 1].rg0) ++p;
-    next_rg0 = p + 1 < grp.count ? grp.p[p + 1].rg0 : 0x7fffffff;
+    p = 0;
+    next_rg0 = 0x7fffffff;
+    if constexpr (MAXP > 1) {
+      p = p_from;
+      while (p + 1 < grp.count && rg >= grp.p[p + 1].rg0) ++p;
+      next_rg0 = p + 1 < grp.count ? grp.p[p + 1].rg0 : 0x7fffffff;
+    }
   }
   // to the next item; true when that item begins a new row group
   __device__ bool step(const Group<MAXP>& grp) {
     if (++kc < grp.C) return false;
     kc = 0;
-    if (++rg >= next_rg0) {
-      ++p;
-      next_rg0 = p + 1 < grp.count ? grp.p[p + 1].rg0 : 0x7fffffff;
+    ++rg;
+    if constexpr (MAXP > 1) {
+      if (rg >= next_rg0) {
+        ++p;
+        next_rg0 = p + 1 < grp.count ? grp.p[p + 1].rg0 : 0x7fffffff;
+      }
     }
     return true;
   }
@@ -207,15 +214,10 @@ struct Pos {
 // every lane copies the words holding its two rows' block scales.  Rows past
 // N and segments past K copy no scales (the TMA fills their codes with
 // zeros).
-template <int BS, bool DQ, int MAXP>
+template <int BS, bool DQ, int MAXP, bool QUAD>
 struct Fetch {
   const Group<MAXP>& grp;
   int lane, t;
-  // double quant with blocksize >= 64 and K % 256 == 0: the blocks of one
-  // row of an item lie in one aligned 4-byte word of absmax_q and one scale2
-  // group, so the 4 lanes of a quad copy their two rows' words together
-  // (lane t: t = 0 the u word of row g, 1 of row g + 8, 2 / 3 their scale2)
-  bool quad_sc;
   Pos<MAXP> pos;
   int left;             // items not yet issued
   int row0;             // first row of the row group within its problem
@@ -225,14 +227,13 @@ struct Fetch {
   const uint8_t* aq;
   const float* s2;
   int64_t nb;
-  // quad_sc: the row this lane copies a word of (g + 8 (t & 1)), as the
+  // QUAD: the row this lane copies a word of (g + 8 (t & 1)), as the
   // block at the start of the current chunk, and whether that row exists
   int64_t qb;
   bool qv;
 
   __device__ Fetch(const Group<MAXP>& gp, int lane_, const Pos<MAXP>& start, int count)
       : grp(gp), lane(lane_), t(lane_ & 3), pos(start), left(count) {
-    quad_sc = DQ && BS >= 64 && grp.K % kItemK == 0;
     enter();
   }
   __device__ void enter() {
@@ -257,7 +258,7 @@ struct Fetch {
       mbar_arrive_expect_tx(full, kTileBytes);
       tma_load_2d(smem_u32(tile), &grp.maps[pos.p], pos.kc * (kItemK / 2), row0, full);
     }
-    if (quad_sc) {
+    if constexpr (QUAD) {
       // one word per lane, no branches: t < 2 the aligned absmax_q word of
       // its row (cut at the end of the array in the last row group), t >= 2
       // the row's scale2; a missing row copies nothing (zero-fill)
@@ -277,7 +278,7 @@ struct Fetch {
       qb += kItemK / BS;
       if (pos.step(grp)) enter();
       return;
-    }
+    } else {
     const int koff = pos.kc * kItemK + 64 * t;  // the lane's K segment
     const bool seg = koff < grp.K;
     const bool v0 = seg && ok0, v1 = seg && ok1;
@@ -306,6 +307,7 @@ struct Fetch {
       }
     }
     if (pos.step(grp)) enter();
+    }
   }
 };
 
@@ -324,7 +326,12 @@ __device__ __forceinline__ float scale_of(uint32_t w_u, uint32_t w_s, int sh, fl
   }
 }
 
-template <int BS, int QT, bool DQ, int F, int MAXP>
+// QUAD: double quant, blocksize >= 64 and K % 256 == 0 -- the blocks of one
+// row of an item lie in one aligned 4-byte word of absmax_q and one scale2
+// group, so the 4 lanes of a quad copy their two rows' words together (lane
+// t: t = 0 the u word of row g, 1 of row g + 8, 2 / 3 their scale2), and no
+// K segment is past K.
+template <int BS, int QT, bool DQ, int F, int MAXP, bool QUAD>
 __global__ void __launch_bounds__(kThreads, 1)
     gemv4_kernel(const __grid_constant__ Group<MAXP> grp) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -362,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // The other stages fill once the first tile is in (kStages - 1 empty
     // copy groups after the first keep the count of groups committed after
     // each item's at kStages - 1 when it is consumed).
-    Fetch<BS, DQ, MAXP> f(grp, lane, cp, cnt);
+    Fetch<BS, DQ, MAXP, QUAD> f(grp, lane, cp, cnt);
     f.issue(sm.tiles[warp][0], &sm.sc[warp][0][0][0], smem_u32(&full[0]));
 #pragma unroll
     for (int d = 0; d < kStages; ++d) cp_async_commit();
@@ -374,7 +381,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     const uint32_t k16 = grp.k16, k31 = grp.k31;
-    const bool quad_sc = f.quad_sc;
     // the row group being summed: its problem, row group within the problem,
     // this lane's rows, decoded-scale offset, x row and block-index low bits
     int cur_p = 0, rl = 0;
@@ -403,7 +409,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < cnt; ++j) {
       const int d = j & (kStages - 1);
       const int koff = cp.kc * kItemK + 64 * t;  // the lane's K segment
-      const bool seg = koff < grp.K;
+      const bool seg = QUAD || koff < grp.K;
       // x of the segment (batch column g; a segment past K reads zeros)
       if (g < grp.B) {
         const uint4* xs = reinterpret_cast<const uint4*>(xrow + (seg ? koff : 0));
@@ -420,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         c[q] = *reinterpret_cast<const uint4*>(tile + (g + 8 * (q >> 1)) * 128 +
                                                (((2 * t + (q & 1)) ^ g) << 4));
       uint32_t sw[4];
-      if (quad_sc) {
+      if constexpr (QUAD) {
         __syncwarp();  // the quad-mates' scale copies (each waited above) are visible
         const uint4 v = *reinterpret_cast<const uint4*>(&sm.sc[warp][d][0][lane & ~3]);
         sw[0] = v.x;
@@ -528,9 +534,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int BS, int QT, bool DQ, int F, int MAXP>
-cudaError_t launch_t(const Group<MAXP>& grp, int num_sms, cudaStream_t s) {
-  auto kern = gemv4_kernel<BS, QT, DQ, F, MAXP>;
+template <int BS, int QT, bool DQ, int F, int MAXP, bool QUAD>
+cudaError_t launch_k(const Group<MAXP>& grp, int num_sms, cudaStream_t s) {
+  auto kern = gemv4_kernel<BS, QT, DQ, F, MAXP, QUAD>;
   static bool attr_set[64] = {};  // per device
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -545,6 +551,14 @@ cudaError_t launch_t(const Group<MAXP>& grp, int num_sms, cudaStream_t s) {
   const int64_t grid = grp.n_rg < num_sms ? grp.n_rg : num_sms;
   return launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmemBytes, s,
                        false, grp);
+}
+
+template <int BS, int QT, bool DQ, int F, int MAXP>
+cudaError_t launch_t(const Group<MAXP>& grp, int num_sms, cudaStream_t s) {
+  if constexpr (DQ && BS >= 64) {
+    if (grp.K % kItemK == 0) return launch_k<BS, QT, DQ, F, MAXP, true>(grp, num_sms, s);
+  }
+  return launch_k<BS, QT, DQ, F, MAXP, false>(grp, num_sms, s);
 }
 
 // Fills the problem list from the linear layers' arguments (already checked
@@ -612,15 +626,17 @@ cudaError_t launch_gemv(const void* x, int64_t B, int64_t K, const bnb4_qstate& 
                         int64_t N, void* y, const void* bias, int fmt, int num_sms, int* err,
                         cudaStream_t s) {
   const GemvLinear one{x, &W, K, N, bias, y};
-  return launch_group<kSmallGroup>(&one, 1, B, fmt, num_sms, err, s);
+  return launch_group<1>(&one, 1, B, fmt, num_sms, err, s);
 }
 
 cudaError_t launch_gemv_group(const GemvLinear* lin, int count, int64_t B, int fmt,
                               int num_sms, int* err, cudaStream_t s) {
+  if (count == 1) return launch_group<1>(lin, count, B, fmt, num_sms, err, s);
   if (count <= kSmallGroup) return launch_group<kSmallGroup>(lin, count, B, fmt, num_sms, err, s);
   for (int i = 0; i < count; i += kLargeGroup) {
     const int c = count - i < kLargeGroup ? count - i : kLargeGroup;
-    const cudaError_t e = c <= kSmallGroup
+    const cudaError_t e = c == 1 ? launch_group<1>(lin + i, c, B, fmt, num_sms, err, s)
+                          : c <= kSmallGroup
                               ? launch_group<kSmallGroup>(lin + i, c, B, fmt, num_sms, err, s)
                               : launch_group<kLargeGroup>(lin + i, c, B, fmt, num_sms, err, s);
     if (e != cudaSuccess) return e;
