@@ -10,7 +10,7 @@
 // one output chunk of 16 bytes per row (4 fp32 or 8 bf16 elements), so a
 // warp's code load (64 or 128 contiguous bytes) and its output store (512
 // contiguous bytes) are both fully coalesced.  A warp streams whole tiles of
-// 8 rows; each row's register slots -- the code word and the raw scale
+// 4 rows; each row's register slots -- the code word and the raw scale
 // inputs of the chunk's block -- are refilled with the same row of the warp's
 // next tile as soon as the row is consumed, so neither the codes nor the
 // scales are waited for.  Lane pointers advance once per tile and rows are
@@ -26,7 +26,7 @@ namespace bnb4 {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kRows = 8;
+constexpr int kRows = 4;  // rows per tile (4 measured best of 2-16 on B200)
 constexpr int kCtasPerSm = 4;  // resident CTAs per SM (64 registers)
 
 // Output element type per format: fp32 (4 per 16-byte chunk) or a 16-bit
