@@ -78,16 +78,16 @@ ALU_OPS_PER_WEIGHT = 2.5
 
 TRAFFIC = {
     # decode: DRAM bytes of one cold 11008 x 4096 launch over its algorithmic
-    # bytes (23.92 MB / 23.27 MB); the family's traffic per launch is that
+    # bytes (23.30 MB / 23.27 MB); the family's traffic per launch is that
     # ratio times its algorithmic bytes per launch
-    "gemv": {"ratio": 23.922944 / 23.27,
+    "gemv": {"ratio": 23.30112 / 23.27,
              "launch": "one decode launch (11008 x 4096, B = 1, captured cold), scaled by "
                        "the algorithmic bytes per launch of the family",
              "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemv.cu",
                          "bit_blockwise_weight_nf4_b200/csrc/lut.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "48f088efe3b179273161613bcbc1f8564a7e529a6698eb352113d58c7a0858f7"},
+             "sha256": "dbf1605d6b8a6f8579c588df7eac0968562b5fac38f2065b649e5c9645d5d0cb"},
     "gemm": {"bytes": 37468818,
              "launch": "one prefill GEMM launch, averaged over the seven Llama-7B linears",
              "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemm.cu",

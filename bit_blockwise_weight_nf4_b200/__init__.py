@@ -366,7 +366,8 @@ def gemv_4bit_grouped(items, outs=None):
     """Several decode linears in one launch: ``items`` is a list of (x,
     state, N) or (x, state, N, bias) with x [B, K] (bf16 or fp16, the same B
     and dtype for all; x may be shared); returns the outputs [B, N] (or
-    writes ``outs``).  Bit-identical to calling linear_4bit on each."""
+    writes ``outs``).  Two or more linears run the persistent decode kernel,
+    whose fp32 sums may differ in the last bit from a single call's."""
     torch = _torch()
     if outs is None:
         outs = [torch.empty(it[0].shape[0], it[2], dtype=it[0].dtype, device=it[0].device)

@@ -4,6 +4,9 @@
 // h = round to the 16-bit compute format, bf16 or fp16 (nearest even); the
 // bias is optional.
 //
+// This kernel serves grouped launches of two or more weights; a single
+// weight runs the one-launch kernel of gemv_direct.cu (faster there).
+//
 // Method: bitsandbytes' gemv_4bit op (ossradar page, release notes 0.50.0)
 // over the blockwise NF4 / FP4 format of the CSDN article (section
 // "数学原理对比"), nested (double) quantization decoded in-kernel.
@@ -98,7 +101,7 @@ struct Group {
   uint32_t k16, k31;  // 2^16 and 2^31, opaque to the compiler (see dq8_fma)
   int* err;           // the library's device error word
 };
-constexpr int kSmallGroup = 4;   // q/k/v, gate/up (one GEMV: a group of 1)
+constexpr int kSmallGroup = 4;   // q/k/v, gate/up
 constexpr int kLargeGroup = 32;  // a longer list is launched in parts of 32
 static_assert(sizeof(Group<kLargeGroup>) <= 32000, "kernel parameter space");
 
@@ -625,17 +628,22 @@ cudaError_t launch_group(const GemvLinear* lin, int count, int64_t B, int fmt, i
 cudaError_t launch_gemv(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
                         int64_t N, void* y, const void* bias, int fmt, int num_sms, int* err,
                         cudaStream_t s) {
-  const GemvLinear one{x, &W, K, N, bias, y};
-  return launch_group<1>(&one, 1, B, fmt, num_sms, err, s);
+  // a single weight: the direct kernel is faster (gemv_direct.cu)
+  (void)num_sms;
+  (void)err;
+  return launch_gemv_direct(x, B, K, W, N, y, bias, fmt, s);
 }
 
 cudaError_t launch_gemv_group(const GemvLinear* lin, int count, int64_t B, int fmt,
                               int num_sms, int* err, cudaStream_t s) {
-  if (count == 1) return launch_group<1>(lin, count, B, fmt, num_sms, err, s);
+  if (count == 1)
+    return launch_gemv_direct(lin[0].x, B, lin[0].K, *lin[0].W, lin[0].N, lin[0].y,
+                              lin[0].bias, fmt, s);
   if (count <= kSmallGroup) return launch_group<kSmallGroup>(lin, count, B, fmt, num_sms, err, s);
   for (int i = 0; i < count; i += kLargeGroup) {
     const int c = count - i < kLargeGroup ? count - i : kLargeGroup;
-    const cudaError_t e = c == 1 ? launch_group<1>(lin + i, c, B, fmt, num_sms, err, s)
+    const cudaError_t e = c == 1 ? launch_gemv_direct(lin[i].x, B, lin[i].K, *lin[i].W, lin[i].N,
+                                                      lin[i].y, lin[i].bias, fmt, s)
                           : c <= kSmallGroup
                               ? launch_group<kSmallGroup>(lin + i, c, B, fmt, num_sms, err, s)
                               : launch_group<kLargeGroup>(lin + i, c, B, fmt, num_sms, err, s);

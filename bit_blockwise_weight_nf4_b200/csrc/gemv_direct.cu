@@ -1,0 +1,267 @@
+// gemv_direct.cu -- decode GEMV with 4-bit weights on sm_100a, one launch
+// per weight: the kernel behind single GEMV calls (grouped calls of two or
+// more weights use the persistent TMA-staged kernel of gemv.cu, which is
+// faster there; measured side by side on B200, this one is 10-17% faster for
+// a single weight at B = 1 and 28-32% at B = 8).
+//   y[b, n] = h( sum_k x[b, k] * What[n, k] + bias[n] ),  1 <= B <= 8,
+//   What[n, k] = h(RN(t[code] * a_hat))   (dequantized weight, exact),
+// h = round to the 16-bit compute format, bf16 or fp16 (nearest even); the
+// bias is optional.
+//
+// Method: bitsandbytes' gemv_4bit op (ossradar page, release notes 0.50.0)
+// over the blockwise NF4 / FP4 format of the CSDN article (section
+// "数学原理对比"), nested (double) quantization decoded in-kernel.
+//
+// Design:
+//  * One CTA (8 warps) per 16 weight rows, 2 CTAs resident per SM, as many
+//    CTAs as row groups: the block scheduler overlaps one CTA's start-up
+//    (first loads) with other CTAs' math.  The warps split K in 256-wide
+//    steps; the 4 lanes of a quad own two rows (g and g + 8) and a
+//    contiguous 64-element segment of each per step (2 x 2 128-bit loads
+//    straight into registers); every lane keeps 2 steps of loads (codes and
+//    raw scales) in flight.
+//  * Per (row, quant block) a lane builds the 16-entry table of
+//    h(RN(t[i] * a_hat)) and looks codes up with byte permutes (lut.cuh).
+//  * The products run on mma.sync m16n8k16 with the weight as the A operand
+//    (16 rows) and x as B (batch columns, read just in time from L1): K is
+//    permuted identically in both operands, which leaves the dot products
+//    unchanged; two accumulator chains keep consecutive MMAs independent;
+//    batch columns beyond B read a valid row whose outputs are discarded.
+//  * The 8 warps' partial sums are added in shared memory in a fixed order,
+//    the bias (if any) added in fp32, and rounded once.
+#include "common.cuh"
+#include "kernels.h"
+#include "lut.cuh"
+
+namespace bnb4 {
+namespace {
+
+constexpr int kWarps = 8;       // warps per CTA; they split K of one 16-row group
+constexpr int kThreads = kWarps * 32;
+constexpr int kRowsPerCta = 16;
+constexpr int kKStep = 256;  // K covered by one warp step (4 lanes x 64)
+constexpr int kChains = 2;   // independent MMA accumulators per warp
+
+// D[16 x 8] += A[16 x 16] (weight rows) * B[16 x 8] (x columns), bf16 or
+// fp16 in (format F), fp32 accumulate.
+template <int F>
+__device__ __forceinline__ void mma16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                      uint32_t a3, uint32_t b0, uint32_t b1) {
+  if constexpr (F == BNB4_F16)
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  else
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Raw scale inputs of one quant block, loaded ahead and decoded when used
+// (so the decode never waits on a load issued just before it).
+struct RawScale {
+  uint32_t u;  // absmax_q byte (double quant) or absmax bits
+  float s;     // scale2 of the block's group (double quant)
+};
+
+template <bool DQ>
+__device__ __forceinline__ RawScale load_scale(int64_t b, const float* absmax,
+                                               const uint8_t* absmax_q,
+                                               const float* scale2) {
+  RawScale r;
+  if constexpr (DQ) {
+    r.u = __ldg(absmax_q + b);
+    r.s = __ldg(scale2 + (b >> 8));
+  } else {
+    r.u = __float_as_uint(__ldg(absmax + b));
+    r.s = 0.0f;
+  }
+  return r;
+}
+
+template <bool DQ>
+__device__ __forceinline__ float decode(const RawScale& r, float off) {
+  if constexpr (DQ)
+    return __fmaf_rn(static_cast<float>(static_cast<int>(r.u) - 128), r.s, off);
+  else
+    return __uint_as_float(r.u);
+}
+
+// Loads of one K step of one lane: 64 codes of each of its two rows and the
+// scales of their blocks, issued kDepth steps ahead of their use.
+struct StepBuf {
+  uint4 c[2][2];       // [row g / g+8][16-byte half]
+  RawScale a[2][2];    // [row][block within the segment (blocksize 32)]
+};
+
+template <int BS, int QT, bool DQ, int kDepth, int F>
+__global__ void __launch_bounds__(kThreads, 2)
+    gemv4_direct_kernel(const uint16_t* __restrict__ x, int B, int64_t K,
+                 const uint8_t* __restrict__ codes,
+                 const float* __restrict__ absmax,
+                 const uint8_t* __restrict__ absmax_q,
+                 const float* __restrict__ scale2,
+                 const float* __restrict__ offset, int64_t N,
+                 const uint16_t* __restrict__ bias, uint16_t* __restrict__ y) {
+  __shared__ float red[kWarps][32][4];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int g = lane >> 2;  // rows g and g + 8 of the group; batch column g of x
+  const int t = lane & 3;   // K segment of the step
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRowsPerCta;
+  const int64_t n[2] = {row0 + g, row0 + g + 8};
+  const bool ok[2] = {n[0] < N, n[1] < N};
+  const float off = DQ ? __ldg(offset) : 0.0f;
+  const int64_t steps = (K + kKStep - 1) / kKStep;
+  const int my_steps =
+      warp < steps ? static_cast<int>((steps - warp + kWarps - 1) / kWarps) : 0;
+  // batch columns beyond B read row B-1 (valid memory); their outputs are
+  // never stored
+  const uint16_t* xrow = x + static_cast<int64_t>(g < B ? g : B - 1) * K;
+
+  auto issue = [&](int i, StepBuf& b) {
+    const int64_t k0 = (static_cast<int64_t>(i) * kWarps + warp) * kKStep + 64 * t;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      if (ok[r] && k0 < K) {
+        const uint8_t* src = codes + n[r] * (K / 2) + k0 / 2;
+        b.c[r][0] = ldg_stream_v4(src);
+        b.c[r][1] = ldg_stream_v4(src + 16);
+        const int64_t blk = (n[r] * K + k0) / BS;
+        b.a[r][0] = load_scale<DQ>(blk, absmax, absmax_q, scale2);
+        if constexpr (BS == 32) b.a[r][1] = load_scale<DQ>(blk + 1, absmax, absmax_q, scale2);
+      } else {
+        b.c[r][0] = make_uint4(0, 0, 0, 0);
+        b.c[r][1] = b.c[r][0];
+        b.a[r][0] = RawScale{0u, 0.0f};
+        b.a[r][1] = b.a[r][0];
+      }
+    }
+  };
+
+  float acc[kChains][4] = {};
+  StepBuf buf[kDepth];
+#pragma unroll
+  for (int d = 0; d < kDepth; ++d)
+    if (d < my_steps) issue(d, buf[d]);
+
+  for (int base = 0; base < my_steps; base += kDepth) {
+#pragma unroll
+    for (int d = 0; d < kDepth; ++d) {
+      const int i = base + d;
+      if (i < my_steps) {  // warp-uniform
+        const int64_t k0 = (static_cast<int64_t>(i) * kWarps + warp) * kKStep + 64 * t;
+        const bool seg = k0 < K;
+        // past a ragged K edge or the N edge the lane's rows are zero codes
+        // with a zero scale: mma.sync needs every lane of the warp
+        Lut lut[2][2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          lut[r][0] = make_lut<QT, F>(ok[r] && seg ? decode<DQ>(buf[d].a[r][0], off) : 0.0f);
+          lut[r][1] = BS == 32
+                          ? make_lut<QT, F>(ok[r] && seg ? decode<DQ>(buf[d].a[r][1], off) : 0.0f)
+                          : lut[r][0];
+        }
+        const int64_t kx = seg ? k0 : 0;  // x stays in bounds on a ragged edge
+#pragma unroll
+        for (int p = 0; p < 8; ++p) {  // codes k0 + 8p .. +7 of both rows: two MMAs
+          const uint4 xb = __ldg(reinterpret_cast<const uint4*>(xrow + kx + 8 * p));
+          const int h = p >> 2, wi = p & 3;
+          const uint32_t w0 = wi == 0 ? buf[d].c[0][h].x : wi == 1 ? buf[d].c[0][h].y
+                            : wi == 2 ? buf[d].c[0][h].z : buf[d].c[0][h].w;
+          const uint32_t w1 = wi == 0 ? buf[d].c[1][h].x : wi == 1 ? buf[d].c[1][h].y
+                            : wi == 2 ? buf[d].c[1][h].z : buf[d].c[1][h].w;
+          const uint4 o0 = dq8(lut[0][BS == 32 ? h : 0], w0);
+          const uint4 o1 = dq8(lut[1][BS == 32 ? h : 0], w1);
+          mma16<F>(acc[(2 * p) % kChains], o0.x, o1.x, o0.y, o1.y, xb.x, xb.y);
+          mma16<F>(acc[(2 * p + 1) % kChains], o0.z, o1.z, o0.w, o1.w, xb.z, xb.w);
+        }
+        if (i + kDepth < my_steps) issue(i + kDepth, buf[d]);
+      }
+    }
+  }
+
+  // acc[.]: rows g (0, 1) and g + 8 (2, 3) of the group, batch columns 2t and
+  // 2t + 1
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    float sum = 0.f;
+#pragma unroll
+    for (int c = 0; c < kChains; ++c) sum += acc[c][v];
+    red[warp][lane][v] = sum;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float s[4];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      s[v] = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) s[v] += red[w][lane][v];
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+#pragma unroll
+      for (int cb = 0; cb < 2; ++cb) {
+        const int bcol = 2 * t + cb;
+        if (ok[r] && bcol < B) {
+          float v = s[2 * r + cb];
+          if (bias) v = __fadd_rn(v, half_to_f32<F>(bias[n[r]]));
+          const uint32_t o = pack2<F>(v, 0.0f);
+          y[static_cast<int64_t>(bcol) * N + n[r]] = static_cast<uint16_t>(o);
+        }
+      }
+    }
+  }
+}
+
+template <int BS, int QT, bool DQ, int kDepth, int F>
+cudaError_t launch_t(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
+                     int64_t N, const void* bias, void* y, cudaStream_t s) {
+  const int64_t grid = (N + kRowsPerCta - 1) / kRowsPerCta;
+  return launch_kernel(gemv4_direct_kernel<BS, QT, DQ, kDepth, F>, dim3(static_cast<unsigned>(grid)),
+             dim3(kThreads), 0, s, false, static_cast<const uint16_t*>(x), static_cast<int>(B), K,
+             static_cast<const uint8_t*>(W.codes), static_cast<const float*>(W.absmax),
+             static_cast<const uint8_t*>(W.absmax_q), static_cast<const float*>(W.scale2),
+             static_cast<const float*>(W.offset), N, static_cast<const uint16_t*>(bias),
+             static_cast<uint16_t*>(y));
+}
+
+template <int BS, int QT, int F>
+cudaError_t launch_bs(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
+                      int64_t N, const void* bias, void* y, cudaStream_t s) {
+  // two K steps of loads in flight per lane (for K <= 4096 that is all of a
+  // warp's share), 2 CTAs of 8 warps resident per SM
+  if (W.double_quant) return launch_t<BS, QT, true, 2, F>(x, B, K, W, N, bias, y, s);
+  return launch_t<BS, QT, false, 2, F>(x, B, K, W, N, bias, y, s);
+}
+
+template <int QT, int F>
+cudaError_t launch_q(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
+                     int64_t N, const void* bias, void* y, cudaStream_t s) {
+  switch (W.blocksize) {
+    case 32: return launch_bs<32, QT, F>(x, B, K, W, N, bias, y, s);
+    case 64: return launch_bs<64, QT, F>(x, B, K, W, N, bias, y, s);
+    case 128: return launch_bs<128, QT, F>(x, B, K, W, N, bias, y, s);
+    default: return launch_bs<256, QT, F>(x, B, K, W, N, bias, y, s);
+  }
+}
+
+template <int F>
+cudaError_t launch_f(const void* x, int64_t B, int64_t K, const bnb4_qstate& W, int64_t N,
+                     const void* bias, void* y, cudaStream_t s) {
+  return W.qtype == kQtNF4 ? launch_q<kQtNF4, F>(x, B, K, W, N, bias, y, s)
+                           : launch_q<kQtFP4, F>(x, B, K, W, N, bias, y, s);
+}
+
+}  // namespace
+
+cudaError_t launch_gemv_direct(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
+                               int64_t N, void* y, const void* bias, int fmt, cudaStream_t s) {
+  return fmt == BNB4_F16 ? launch_f<BNB4_F16>(x, B, K, W, N, bias, y, s)
+                         : launch_f<BNB4_BF16>(x, B, K, W, N, bias, y, s);
+}
+
+}  // namespace bnb4

@@ -52,6 +52,11 @@ cudaError_t launch_gemv(const void* x, int64_t B, int64_t K,
                         const bnb4_qstate& W, int64_t N, void* y, const void* bias,
                         int fmt, int num_sms, int* err, cudaStream_t s);
 
+// The same GEMV in a launch of its own (one CTA per 16 rows, gemv_direct.cu):
+// faster than the persistent kernel for a single weight.
+cudaError_t launch_gemv_direct(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
+                               int64_t N, void* y, const void* bias, int fmt, cudaStream_t s);
+
 // One decode linear of a grouped launch (x [B, K], W [N, K], bias, y [B, N]).
 struct GemvLinear {
   const void* x;

@@ -253,10 +253,12 @@ BNB4_API int bnb_dequantize_4bit_2d(const bnb4_qstate* st, void* out, int32_t ou
  *  x  device bf16 [B, K], 16-byte aligned;   y  device bf16 [B, N].
  *  W  quantization state of the weight [N, K] (W->n == N*K).
  * Constraints: 1 <= B <= 256; K % 64 == 0; K % W->blocksize == 0; N, K <
- * 2^31.  B <= 8 runs the decode kernel (persistent, one CTA per SM; the
- * packed weight tiles staged in shared memory by TMA; mma.sync, one 8-column
- * group; partial sums over K added in a fixed order, so results are
- * bit-reproducible); larger batches run the small-batch tcgen05 kernel of
+ * 2^31.  B <= 8 runs the one-launch decode kernel (one CTA per 16 rows,
+ * packed codes loaded straight into registers two K steps ahead; mma.sync,
+ * one 8-column group; partial sums over K added in a fixed order, so
+ * results are bit-reproducible) -- measured faster for a single weight than
+ * the persistent TMA-staged kernel that bnb_gemv_4bit_grouped runs for two
+ * or more; larger batches run the small-batch tcgen05 kernel of
  * bnb_gemm_4bit.
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, SHAPE, CUDA.
  */
@@ -270,11 +272,14 @@ BNB4_API int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstat
  * for every problem i,
  *   y_i[b, n] = h( sum_k x_i[b, k] * What_i[n, k] + bias_i[n] ),
  * the arithmetic of bnb_linear_4bit with M = B (exact products, fp32
- * accumulation, one rounding).  One persistent grid streams all the weights,
- * so the start-up of a launch is paid once for the whole list.  The order of
- * the fp32 sums over K follows how the row groups of the whole list are
- * split over the SMs, so a problem's result can differ in the last bit from
- * a single call; the same list on the same device gives identical bits.
+ * accumulation, one rounding).  Two or more problems run one persistent
+ * grid (one CTA of 16 warps per SM, the packed weight tiles staged in shared
+ * memory by 2-D TMA copies) that streams all the weights, so the start-up of
+ * a launch is paid once for the whole list; a list of one runs the kernel of
+ * bnb_gemv_4bit.  The order of the fp32 sums over K follows how the row
+ * groups of the whole list are split over the SMs, so a problem's result can
+ * differ in the last bit from a single call; the same list on the same
+ * device gives identical bits.
  *  problems  host array of `count` descriptors (read during the call only):
  *            x device [B, K] of dtype, 16-byte aligned; W the quantization
  *            state of the weight [N, K] (W.n == N * K); bias device [N] of

@@ -14,7 +14,10 @@ from parity import check_linear, cpu_bits
 pytestmark = pytest.mark.gpu
 
 
-def case(N, K, B, bs, qtype, dq, seed):
+def case(N, K, B, bs, qtype, dq, seed, path="single"):
+    """path "single": one bnb_gemv_4bit call (the one-launch-per-weight
+    kernel); "grouped": the weight twice in one bnb_gemv_4bit_grouped call
+    (the persistent kernel), both outputs checked."""
     W = synth.weight_bf16(N, K, seed=seed)
     x = synth.activations_bf16(B, K, seed=seed + 1)
     st = oracle.quantize(synth.bf16_bits(W.view(-1)), bs, qtype, dq)
@@ -22,16 +25,24 @@ def case(N, K, B, bs, qtype, dq, seed):
     xb = synth.bf16_bits(x)
     y64 = oracle.linear_ref(xb, What)
     g = bnb4.state_from_arrays(st)
-    y = bnb4.gemv_4bit(x.cuda(), g, N)
-    return check_linear(cpu_bits(y), y64, xb, What)
+    if path == "single":
+        return check_linear(cpu_bits(bnb4.gemv_4bit(x.cuda(), g, N)), y64, xb, What)
+    xd = x.cuda()
+    for y in bnb4.gemv_4bit_grouped([(xd, g, N), (xd, g, N)]):
+        r = check_linear(cpu_bits(y), y64, xb, What)
+    return r
 
 
+PATHS = ["single", "grouped"]
+
+
+@pytest.mark.parametrize("path", PATHS)
 @pytest.mark.parametrize("N,K", [(11008, 4096), (4096, 11008)])
 @pytest.mark.parametrize("B", [1, 8])
-def test_llama_mlp_shapes(N, K, B):
+def test_llama_mlp_shapes(N, K, B, path):
     """Decode GEMV: x bf16 [B, K] ~ N(0, 1); NF4 weight ~ N(0, 0.02^2),
     blocksize 64, double quant (Llama-7B MLP shapes)."""
-    case(N, K, B, 64, bnb4.NF4, True, seed=N + K)
+    case(N, K, B, 64, bnb4.NF4, True, seed=N + K, path=path)
 
 
 @pytest.mark.parametrize("qtype", [bnb4.NF4, bnb4.FP4])
@@ -39,21 +50,23 @@ def test_llama_mlp_shapes(N, K, B):
 @pytest.mark.parametrize("dq", [True, False])
 @pytest.mark.parametrize("N,K,B", [(1, 256, 1), (13, 320, 3), (100, 576, 8),
                                    (257, 1024, 5), (8, 64, 2)])
-def test_small_ragged(qtype, bs, dq, N, K, B):
+@pytest.mark.parametrize("path", PATHS)
+def test_small_ragged(qtype, bs, dq, N, K, B, path):
     if K % bs:
         pytest.skip("K must be a multiple of the blocksize")
-    case(N, K, B, bs, qtype, dq, seed=N * 31 + K)
+    case(N, K, B, bs, qtype, dq, seed=N * 31 + K, path=path)
 
 
 @pytest.mark.parametrize("N,K,B", [(4099, 4096, 1), (1030, 2112, 2), (517, 11008, 4),
                                    (30001, 256, 8), (4096, 64, 1), (22, 1344, 2),
                                    (40003, 1024, 1), (38000, 2048, 3), (2400, 4352, 8)])
-def test_row_groups_and_warp_splits(N, K, B):
-    """16-row groups with ragged N; K split over the CTA's warps (K of at
-    least one 256-wide chunk per warp, or few row groups per CTA: 1 to 16
-    warps, a last chunk with empty segments) or whole row groups per warp
-    (short K and many row groups: 40003 x 1024, 38000 x 2048)."""
-    case(N, K, B, 64, bnb4.NF4, True, seed=N + 3 * K + B)
+@pytest.mark.parametrize("path", PATHS)
+def test_row_groups_and_warp_splits(N, K, B, path):
+    """16-row groups with ragged N; K split over a CTA's warps (few row
+    groups per CTA: runs that start and end inside row groups, a last chunk
+    with empty segments) or whole row groups per warp (short K and many row
+    groups: 40003 x 1024, 38000 x 2048)."""
+    case(N, K, B, 64, bnb4.NF4, True, seed=N + 3 * K + B, path=path)
 
 
 @pytest.mark.parametrize("N,K", [(11008, 4096), (4096, 11008), (40003, 1024)])
