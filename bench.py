@@ -77,17 +77,21 @@ GEMV_WEIGHTS = 4
 ALU_OPS_PER_WEIGHT = 2.5
 
 TRAFFIC = {
-    # decode: DRAM bytes of one cold 11008 x 4096 launch over its algorithmic
-    # bytes (23.30 MB / 23.27 MB); the family's traffic per launch is that
-    # ratio times its algorithmic bytes per launch
-    "gemv": {"ratio": 23.30112 / 23.27,
-             "launch": "one decode launch (11008 x 4096, B = 1, captured cold), scaled by "
-                       "the algorithmic bytes per launch of the family",
+    # decode: DRAM bytes over algorithmic bytes of cold launches of both
+    # decode kernels -- the single-weight one on 11008 x 4096 (23.29 / 23.27
+    # MB) and the persistent one on the q/k/v list (26.02 / 26.03 MB); the
+    # family's traffic per launch is that ratio times its algorithmic bytes
+    # per launch
+    "gemv": {"ratio": (23.293952 + 26.016768) / (23.27 + 26.03),
+             "launch": "cold captures of both decode kernels (11008 x 4096 single, "
+                       "3 x 4096 x 4096 grouped), scaled by the algorithmic bytes per "
+                       "launch of the family",
              "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemv.cu",
+                         "bit_blockwise_weight_nf4_b200/csrc/gemv_direct.cu",
                          "bit_blockwise_weight_nf4_b200/csrc/lut.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "dbf1605d6b8a6f8579c588df7eac0968562b5fac38f2065b649e5c9645d5d0cb"},
+             "sha256": "5d5032779593b7944dd421ffc27f87249c853eca5b80871e5900030a88c623e0"},
     "gemm": {"bytes": 37468818,
              "launch": "one prefill GEMM launch, averaged over the seven Llama-7B linears",
              "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemm.cu",
