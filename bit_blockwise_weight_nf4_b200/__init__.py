@@ -100,6 +100,8 @@ def load():
         "bnb_gemm_4bit": ([p, i64, i64, QP, i64, p, p], ctypes.c_int),
         "bnb_gemv_4bit_grouped": ([ctypes.POINTER(GemvProblem), i32, i64, i32, p],
                                   ctypes.c_int),
+        "bnb4_debug_gemv_grouped_persistent": ([ctypes.POINTER(GemvProblem), i32, i64, i32, p],
+                                               ctypes.c_int),
         "bnb_linear_4bit": ([p, i32, i64, i64, QP, i64, p, p, p], ctypes.c_int),
         "bnb4_device_status": ([p, i32], ctypes.c_int),
         "bnb4_debug_gemm_withhold": ([p, i64, i64, QP, i64, p, i32, p], ctypes.c_int),
@@ -172,6 +174,13 @@ def bnb_gemv_4bit_grouped(problems, B, dtype, stream):
     if not isinstance(problems, ctypes.Array):
         problems = (GemvProblem * len(problems))(*problems)
     return load().bnb_gemv_4bit_grouped(problems, len(problems), B, dtype, stream)
+
+
+def bnb4_debug_gemv_grouped_persistent(problems, B, dtype, stream):
+    """bnb_gemv_4bit_grouped forced onto the persistent kernel (tests)."""
+    if not isinstance(problems, ctypes.Array):
+        problems = (GemvProblem * len(problems))(*problems)
+    return load().bnb4_debug_gemv_grouped_persistent(problems, len(problems), B, dtype, stream)
 
 
 def bnb_linear_4bit(x, dtype, M, K, W, N, bias, y, stream):
@@ -362,12 +371,13 @@ def linear_4bit(x, state, N, bias=None, out=None):
     return out
 
 
-def gemv_4bit_grouped(items, outs=None):
+def gemv_4bit_grouped(items, outs=None, _persistent=False):
     """Several decode linears in one launch: ``items`` is a list of (x,
     state, N) or (x, state, N, bias) with x [B, K] (bf16 or fp16, the same B
     and dtype for all; x may be shared); returns the outputs [B, N] (or
-    writes ``outs``).  Two or more linears run the persistent decode kernel,
-    whose fp32 sums may differ in the last bit from a single call's."""
+    writes ``outs``).  With one row of x and four or more linears the list
+    runs the persistent decode kernel (``_persistent=True`` forces it, for
+    tests), whose fp32 sums may differ in the last bit from a single call's."""
     torch = _torch()
     if outs is None:
         outs = [torch.empty(it[0].shape[0], it[2], dtype=it[0].dtype, device=it[0].device)
@@ -381,7 +391,8 @@ def gemv_4bit_grouped(items, outs=None):
         bias = it[3] if len(it) > 3 else None
         probs[i] = GemvProblem(x.data_ptr(), state.cstruct(), x.shape[1], N,
                                None if bias is None else bias.data_ptr(), y.data_ptr())
-    rc = bnb_gemv_4bit_grouped(probs, items[0][0].shape[0], dt, _stream())
+    fn = bnb4_debug_gemv_grouped_persistent if _persistent else bnb_gemv_4bit_grouped
+    rc = fn(probs, items[0][0].shape[0], dt, _stream())
     _check(rc, "bnb_gemv_4bit_grouped")
     return outs
 

@@ -354,8 +354,9 @@ int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstate* W,
                                            static_cast<cudaStream_t>(stream)));
 }
 
-int bnb_gemv_4bit_grouped(const bnb4_gemv_problem* problems, int32_t count, int64_t B,
-                          int32_t dtype, void* stream) {
+namespace {
+int gemv_grouped_impl(const bnb4_gemv_problem* problems, int32_t count, int64_t B,
+                      int32_t dtype, void* stream, bool persistent) {
   if (!problems || count < 1) return BNB4_ERR_INVALID_ARG;
   if (count > BNB4_GROUP_MAX) return BNB4_ERR_SHAPE;
   if (dtype != BNB4_BF16 && dtype != BNB4_F16) return BNB4_ERR_UNSUPPORTED;
@@ -385,7 +386,18 @@ int bnb_gemv_4bit_grouped(const bnb4_gemv_problem* problems, int32_t count, int6
   int* err;
   if ((rc = error_word(&err)) != BNB4_OK) return rc;
   return from_cuda(bnb4::launch_gemv_group(lin, count, B, dtype, sms, err,
-                                           static_cast<cudaStream_t>(stream)));
+                                           static_cast<cudaStream_t>(stream), persistent));
+}
+}  // namespace
+
+int bnb_gemv_4bit_grouped(const bnb4_gemv_problem* problems, int32_t count, int64_t B,
+                          int32_t dtype, void* stream) {
+  return gemv_grouped_impl(problems, count, B, dtype, stream, false);
+}
+
+int bnb4_debug_gemv_grouped_persistent(const bnb4_gemv_problem* problems, int32_t count,
+                                       int64_t B, int32_t dtype, void* stream) {
+  return gemv_grouped_impl(problems, count, B, dtype, stream, true);
 }
 
 int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstate* W,

@@ -4,8 +4,9 @@
 // h = round to the 16-bit compute format, bf16 or fp16 (nearest even); the
 // bias is optional.
 //
-// This kernel serves grouped launches of two or more weights; a single
-// weight runs the one-launch kernel of gemv_direct.cu (faster there).
+// This kernel serves lists of four or more weights with one row of x; single
+// weights, short lists and B > 1 run the one-CTA-per-16-rows kernel of
+// gemv_direct.cu (faster there).
 //
 // Method: bitsandbytes' gemv_4bit op (ossradar page, release notes 0.50.0)
 // over the blockwise NF4 / FP4 format of the CSDN article (section
@@ -635,18 +636,21 @@ cudaError_t launch_gemv(const void* x, int64_t B, int64_t K, const bnb4_qstate& 
 }
 
 cudaError_t launch_gemv_group(const GemvLinear* lin, int count, int64_t B, int fmt,
-                              int num_sms, int* err, cudaStream_t s) {
-  if (count == 1)
-    return launch_gemv_direct(lin[0].x, B, lin[0].K, *lin[0].W, lin[0].N, lin[0].y,
-                              lin[0].bias, fmt, s);
-  if (count <= kSmallGroup) return launch_group<kSmallGroup>(lin, count, B, fmt, num_sms, err, s);
+                              int num_sms, int* err, cudaStream_t s, bool persistent) {
+  // Measured on B200 (µs per weight, rotating weights larger than L2): this
+  // kernel wins for single-row x over lists of 4 or more (11008 x 4096: 12.0
+  // against 13.9 over 16); the one-CTA-per-16-rows kernel of gemv_direct.cu
+  // wins for lists of 2 or 3 and at every size for B > 1 (16.9 against 22.8
+  // for two 11008 x 4096 weights at B = 8).
   for (int i = 0; i < count; i += kLargeGroup) {
     const int c = count - i < kLargeGroup ? count - i : kLargeGroup;
-    const cudaError_t e = c == 1 ? launch_gemv_direct(lin[i].x, B, lin[i].K, *lin[i].W, lin[i].N,
-                                                      lin[i].y, lin[i].bias, fmt, s)
-                          : c <= kSmallGroup
-                              ? launch_group<kSmallGroup>(lin + i, c, B, fmt, num_sms, err, s)
-                              : launch_group<kLargeGroup>(lin + i, c, B, fmt, num_sms, err, s);
+    cudaError_t e;
+    if (!persistent && (B > 1 || c < 4))
+      e = launch_gemv_direct_list(lin + i, c, B, fmt, s);
+    else if (c <= kSmallGroup)
+      e = launch_group<kSmallGroup>(lin + i, c, B, fmt, num_sms, err, s);
+    else
+      e = launch_group<kLargeGroup>(lin + i, c, B, fmt, num_sms, err, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

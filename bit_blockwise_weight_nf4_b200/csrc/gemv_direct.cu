@@ -43,6 +43,7 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kRowsPerCta = 16;
 constexpr int kKStep = 256;  // K covered by one warp step (4 lanes x 64)
 constexpr int kChains = 2;   // independent MMA accumulators per warp
+constexpr int kDirectListMax = 32;  // weights per launch of a list
 
 // D[16 x 8] += A[16 x 16] (weight rows) * B[16 x 8] (x columns), bf16 or
 // fp16 in (format F), fp32 accumulate.
@@ -98,21 +99,48 @@ struct StepBuf {
   RawScale a[2][2];    // [row][block within the segment (blocksize 32)]
 };
 
-template <int BS, int QT, bool DQ, int kDepth, int F>
+// The weights of a launch: problem i owns row groups [rg0, rg0 + ceil(N /
+// 16)) of the grid; all share K and the batch size.
+struct DirectProb {
+  const uint16_t* x;
+  const uint8_t* codes;
+  const float* absmax;
+  const uint8_t* absmax_q;
+  const float* scale2;
+  const float* offset;
+  const uint16_t* bias;
+  uint16_t* y;
+  int64_t N;
+  int rg0;
+};
+template <int MAXP>
+struct DirectList {
+  DirectProb p[MAXP];
+  int count;
+};
+
+template <int BS, int QT, bool DQ, int kDepth, int F, int MAXP>
 __global__ void __launch_bounds__(kThreads, 2)
-    gemv4_direct_kernel(const uint16_t* __restrict__ x, int B, int64_t K,
-                 const uint8_t* __restrict__ codes,
-                 const float* __restrict__ absmax,
-                 const uint8_t* __restrict__ absmax_q,
-                 const float* __restrict__ scale2,
-                 const float* __restrict__ offset, int64_t N,
-                 const uint16_t* __restrict__ bias, uint16_t* __restrict__ y) {
+    gemv4_direct_kernel(const __grid_constant__ DirectList<MAXP> L, int B, int64_t K) {
   __shared__ float red[kWarps][32][4];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int g = lane >> 2;  // rows g and g + 8 of the group; batch column g of x
   const int t = lane & 3;   // K segment of the step
-  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRowsPerCta;
+  int pi = 0;  // this CTA's problem
+  if constexpr (MAXP > 1)
+    while (pi + 1 < L.count && static_cast<int>(blockIdx.x) >= L.p[pi + 1].rg0) ++pi;
+  const DirectProb& P = L.p[pi];
+  const uint16_t* __restrict__ x = P.x;
+  const uint8_t* __restrict__ codes = P.codes;
+  const float* __restrict__ absmax = P.absmax;
+  const uint8_t* __restrict__ absmax_q = P.absmax_q;
+  const float* __restrict__ scale2 = P.scale2;
+  const float* __restrict__ offset = P.offset;
+  const uint16_t* __restrict__ bias = P.bias;
+  uint16_t* __restrict__ y = P.y;
+  const int64_t N = P.N;
+  const int64_t row0 = static_cast<int64_t>(static_cast<int>(blockIdx.x) - P.rg0) * kRowsPerCta;
   const int64_t n[2] = {row0 + g, row0 + g + 8};
   const bool ok[2] = {n[0] < N, n[1] < N};
   const float off = DQ ? __ldg(offset) : 0.0f;
@@ -219,51 +247,77 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-template <int BS, int QT, bool DQ, int kDepth, int F>
-cudaError_t launch_t(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
-                     int64_t N, const void* bias, void* y, cudaStream_t s) {
-  const int64_t grid = (N + kRowsPerCta - 1) / kRowsPerCta;
-  return launch_kernel(gemv4_direct_kernel<BS, QT, DQ, kDepth, F>, dim3(static_cast<unsigned>(grid)),
-             dim3(kThreads), 0, s, false, static_cast<const uint16_t*>(x), static_cast<int>(B), K,
-             static_cast<const uint8_t*>(W.codes), static_cast<const float*>(W.absmax),
-             static_cast<const uint8_t*>(W.absmax_q), static_cast<const float*>(W.scale2),
-             static_cast<const float*>(W.offset), N, static_cast<const uint16_t*>(bias),
-             static_cast<uint16_t*>(y));
-}
-
-template <int BS, int QT, int F>
-cudaError_t launch_bs(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
-                      int64_t N, const void* bias, void* y, cudaStream_t s) {
+template <int BS, int QT, bool DQ, int F, int MAXP>
+cudaError_t launch_t(const DirectList<MAXP>& L, int64_t grid, int64_t B, int64_t K,
+                     cudaStream_t s) {
   // two K steps of loads in flight per lane (for K <= 4096 that is all of a
   // warp's share), 2 CTAs of 8 warps resident per SM
-  if (W.double_quant) return launch_t<BS, QT, true, 2, F>(x, B, K, W, N, bias, y, s);
-  return launch_t<BS, QT, false, 2, F>(x, B, K, W, N, bias, y, s);
+  return launch_kernel(gemv4_direct_kernel<BS, QT, DQ, 2, F, MAXP>,
+                       dim3(static_cast<unsigned>(grid)), dim3(kThreads), 0, s, false, L,
+                       static_cast<int>(B), K);
 }
 
-template <int QT, int F>
-cudaError_t launch_q(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
-                     int64_t N, const void* bias, void* y, cudaStream_t s) {
-  switch (W.blocksize) {
-    case 32: return launch_bs<32, QT, F>(x, B, K, W, N, bias, y, s);
-    case 64: return launch_bs<64, QT, F>(x, B, K, W, N, bias, y, s);
-    case 128: return launch_bs<128, QT, F>(x, B, K, W, N, bias, y, s);
-    default: return launch_bs<256, QT, F>(x, B, K, W, N, bias, y, s);
+template <int MAXP>
+cudaError_t launch_list(const GemvLinear* lin, int count, int64_t B, int fmt, cudaStream_t s) {
+  DirectList<MAXP> L{};
+  L.count = count;
+  int64_t rg = 0;
+  for (int i = 0; i < count; ++i) {
+    const GemvLinear& l = lin[i];
+    DirectProb& p = L.p[i];
+    p.x = static_cast<const uint16_t*>(l.x);
+    p.codes = l.W->codes;
+    p.absmax = l.W->absmax;
+    p.absmax_q = l.W->absmax_q;
+    p.scale2 = l.W->scale2;
+    p.offset = l.W->offset;
+    p.bias = static_cast<const uint16_t*>(l.bias);
+    p.y = static_cast<uint16_t*>(l.y);
+    p.N = l.N;
+    p.rg0 = static_cast<int>(rg);
+    rg += (l.N + kRowsPerCta - 1) / kRowsPerCta;
   }
-}
-
-template <int F>
-cudaError_t launch_f(const void* x, int64_t B, int64_t K, const bnb4_qstate& W, int64_t N,
-                     const void* bias, void* y, cudaStream_t s) {
-  return W.qtype == kQtNF4 ? launch_q<kQtNF4, F>(x, B, K, W, N, bias, y, s)
-                           : launch_q<kQtFP4, F>(x, B, K, W, N, bias, y, s);
+  const bnb4_qstate& W = *lin[0].W;
+  const int64_t K = lin[0].K;
+  const bool dq = W.double_quant != 0;
+  const bool nf4 = W.qtype == kQtNF4;
+  const bool f16 = fmt == BNB4_F16;
+#define BNB4_DIRECT_LAUNCH(BSV)                                                            \
+  if (nf4)                                                                                 \
+    return dq ? (f16 ? launch_t<BSV, kQtNF4, true, BNB4_F16, MAXP>(L, rg, B, K, s)         \
+                     : launch_t<BSV, kQtNF4, true, BNB4_BF16, MAXP>(L, rg, B, K, s))       \
+              : (f16 ? launch_t<BSV, kQtNF4, false, BNB4_F16, MAXP>(L, rg, B, K, s)        \
+                     : launch_t<BSV, kQtNF4, false, BNB4_BF16, MAXP>(L, rg, B, K, s));     \
+  return dq ? (f16 ? launch_t<BSV, kQtFP4, true, BNB4_F16, MAXP>(L, rg, B, K, s)           \
+                   : launch_t<BSV, kQtFP4, true, BNB4_BF16, MAXP>(L, rg, B, K, s))         \
+            : (f16 ? launch_t<BSV, kQtFP4, false, BNB4_F16, MAXP>(L, rg, B, K, s)          \
+                   : launch_t<BSV, kQtFP4, false, BNB4_BF16, MAXP>(L, rg, B, K, s));
+  switch (W.blocksize) {
+    case 32: BNB4_DIRECT_LAUNCH(32)
+    case 64: BNB4_DIRECT_LAUNCH(64)
+    case 128: BNB4_DIRECT_LAUNCH(128)
+    default: BNB4_DIRECT_LAUNCH(256)
+  }
+#undef BNB4_DIRECT_LAUNCH
 }
 
 }  // namespace
 
 cudaError_t launch_gemv_direct(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
                                int64_t N, void* y, const void* bias, int fmt, cudaStream_t s) {
-  return fmt == BNB4_F16 ? launch_f<BNB4_F16>(x, B, K, W, N, bias, y, s)
-                         : launch_f<BNB4_BF16>(x, B, K, W, N, bias, y, s);
+  const GemvLinear one{x, &W, K, N, bias, y};
+  return launch_list<1>(&one, 1, B, fmt, s);
+}
+
+cudaError_t launch_gemv_direct_list(const GemvLinear* lin, int count, int64_t B, int fmt,
+                                    cudaStream_t s) {
+  if (count == 1) return launch_list<1>(lin, 1, B, fmt, s);
+  for (int i = 0; i < count; i += kDirectListMax) {
+    const int c = count - i < kDirectListMax ? count - i : kDirectListMax;
+    const cudaError_t e = launch_list<kDirectListMax>(lin + i, c, B, fmt, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace bnb4

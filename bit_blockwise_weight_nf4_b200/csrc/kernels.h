@@ -52,11 +52,6 @@ cudaError_t launch_gemv(const void* x, int64_t B, int64_t K,
                         const bnb4_qstate& W, int64_t N, void* y, const void* bias,
                         int fmt, int num_sms, int* err, cudaStream_t s);
 
-// The same GEMV in a launch of its own (one CTA per 16 rows, gemv_direct.cu):
-// faster than the persistent kernel for a single weight.
-cudaError_t launch_gemv_direct(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
-                               int64_t N, void* y, const void* bias, int fmt, cudaStream_t s);
-
 // One decode linear of a grouped launch (x [B, K], W [N, K], bias, y [B, N]).
 struct GemvLinear {
   const void* x;
@@ -65,10 +60,23 @@ struct GemvLinear {
   const void* bias;
   void* y;
 };
+
+// The same GEMV in a launch of its own (one CTA per 16 rows, gemv_direct.cu):
+// faster than the persistent kernel for a single weight.
+cudaError_t launch_gemv_direct(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
+                               int64_t N, void* y, const void* bias, int fmt, cudaStream_t s);
+// A list of decode linears (one K, one format), one CTA per 16 rows of any of
+// them, in launches of up to 32 weights.
+cudaError_t launch_gemv_direct_list(const GemvLinear* lin, int count, int64_t B, int fmt,
+                                    cudaStream_t s);
+
+
 // 1..BNB4_GROUP_MAX linears of one format (blocksize, code table, scale
-// format) and one batch size B <= 8 in one persistent launch.
+// format) and one batch size B <= 8: the persistent kernel for B = 1 and 4 or
+// more weights (or always, with `persistent`), else the one-CTA-per-16-rows
+// kernel; launches of up to 32 weights.
 cudaError_t launch_gemv_group(const GemvLinear* lin, int count, int64_t B, int fmt,
-                              int num_sms, int* err, cudaStream_t s);
+                              int num_sms, int* err, cudaStream_t s, bool persistent = false);
 
 // wait_limit_ns = 0 selects the normal bound of every mbarrier wait (2 s);
 // withhold_first_x != 0 is the failure-detection diagnostic (the first X

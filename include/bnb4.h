@@ -272,14 +272,16 @@ BNB4_API int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstat
  * for every problem i,
  *   y_i[b, n] = h( sum_k x_i[b, k] * What_i[n, k] + bias_i[n] ),
  * the arithmetic of bnb_linear_4bit with M = B (exact products, fp32
- * accumulation, one rounding).  Two or more problems run one persistent
- * grid (one CTA of 16 warps per SM, the packed weight tiles staged in shared
- * memory by 2-D TMA copies) that streams all the weights, so the start-up of
- * a launch is paid once for the whole list; a list of one runs the kernel of
- * bnb_gemv_4bit.  The order of the fp32 sums over K follows how the row
- * groups of the whole list are split over the SMs, so a problem's result can
- * differ in the last bit from a single call; the same list on the same
- * device gives identical bits.
+ * accumulation, one rounding).  With B = 1 and 4 or more problems the list
+ * runs one persistent grid (one CTA of 16 warps per SM, the packed weight
+ * tiles staged in shared memory by 2-D TMA copies) that streams all the
+ * weights, so the start-up of a launch is paid once for the whole list;
+ * shorter lists and B > 1 run one launch of the bnb_gemv_4bit kernel over
+ * the whole list (one CTA per 16 rows of any weight) -- each choice the
+ * faster one measured on B200.  With the persistent grid the order of the
+ * fp32 sums over K follows how the row groups of the whole list are split
+ * over the SMs, so a problem's result can differ in the last bit from a
+ * single call; the same list on the same device gives identical bits.
  *  problems  host array of `count` descriptors (read during the call only):
  *            x device [B, K] of dtype, 16-byte aligned; W the quantization
  *            state of the weight [N, K] (W.n == N * K); bias device [N] of
@@ -307,6 +309,16 @@ typedef struct bnb4_gemv_problem {
 } bnb4_gemv_problem;
 BNB4_API int bnb_gemv_4bit_grouped(const bnb4_gemv_problem* problems, int32_t count,
                                    int64_t B, int32_t dtype, void* stream);
+
+/*
+ * Test entry (no counterpart on the pages): bnb_gemv_4bit_grouped with the
+ * persistent TMA-staged kernel for every list, whatever its length and B,
+ * so that the parity tests cover that kernel on every shape.  Same arguments,
+ * results (within the tolerance) and errors.
+ */
+BNB4_API int bnb4_debug_gemv_grouped_persistent(const bnb4_gemv_problem* problems,
+                                                int32_t count, int64_t B, int32_t dtype,
+                                                void* stream);
 
 /*
  * Prefill GEMM with the dequantization fused in (release notes 0.50.0):

@@ -15,9 +15,10 @@ pytestmark = pytest.mark.gpu
 
 
 def case(N, K, B, bs, qtype, dq, seed, path="single"):
-    """path "single": one bnb_gemv_4bit call (the one-launch-per-weight
+    """path "single": one bnb_gemv_4bit call (the one-CTA-per-16-rows
     kernel); "grouped": the weight twice in one bnb_gemv_4bit_grouped call
-    (the persistent kernel), both outputs checked."""
+    (that kernel over a list); "persistent": the same list forced onto the
+    persistent TMA-staged kernel; every output checked."""
     W = synth.weight_bf16(N, K, seed=seed)
     x = synth.activations_bf16(B, K, seed=seed + 1)
     st = oracle.quantize(synth.bf16_bits(W.view(-1)), bs, qtype, dq)
@@ -28,12 +29,12 @@ def case(N, K, B, bs, qtype, dq, seed, path="single"):
     if path == "single":
         return check_linear(cpu_bits(bnb4.gemv_4bit(x.cuda(), g, N)), y64, xb, What)
     xd = x.cuda()
-    for y in bnb4.gemv_4bit_grouped([(xd, g, N), (xd, g, N)]):
+    for y in bnb4.gemv_4bit_grouped([(xd, g, N), (xd, g, N)], _persistent=path == "persistent"):
         r = check_linear(cpu_bits(y), y64, xb, What)
     return r
 
 
-PATHS = ["single", "grouped"]
+PATHS = ["single", "grouped", "persistent"]
 
 
 @pytest.mark.parametrize("path", PATHS)
