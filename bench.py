@@ -78,20 +78,20 @@ ALU_OPS_PER_WEIGHT = 2.5
 
 TRAFFIC = {
     # decode: DRAM bytes over algorithmic bytes of cold launches of both
-    # decode kernels -- the single-weight one on 11008 x 4096 (23.29 / 23.27
-    # MB) and the persistent one on the q/k/v list (26.02 / 26.03 MB); the
-    # family's traffic per launch is that ratio times its algorithmic bytes
-    # per launch
-    "gemv": {"ratio": (23.293952 + 26.016768) / (23.27 + 26.03),
-             "launch": "cold captures of both decode kernels (11008 x 4096 single, "
-                       "3 x 4096 x 4096 grouped), scaled by the algorithmic bytes per "
-                       "launch of the family",
+    # decode kernels -- the one-CTA-per-16-rows one on 11008 x 4096 (23.29 /
+    # 23.29 MB) and the persistent one on the six K = 4096 linears of a layer
+    # (81.28 / 81.27 MB); the family's traffic per launch is that ratio times
+    # its algorithmic bytes per launch
+    "gemv": {"ratio": (23.294208 + 81.275648) / (23.290112 + 81.265152),
+             "launch": "cold captures of both decode kernels (11008 x 4096 single; the "
+                       "six K = 4096 linears of a layer in one persistent launch), scaled "
+                       "by the algorithmic bytes per launch of the family",
              "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemv.cu",
                          "bit_blockwise_weight_nf4_b200/csrc/gemv_direct.cu",
                          "bit_blockwise_weight_nf4_b200/csrc/lut.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "5d5032779593b7944dd421ffc27f87249c853eca5b80871e5900030a88c623e0"},
+             "sha256": "d61b00920d6acca30e379dc6307dfa89c81efab52e2cd0a236a64877190e9a75"},
     "gemm": {"bytes": 37468818,
              "launch": "one prefill GEMM launch, averaged over the seven Llama-7B linears",
              "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemm.cu",
