@@ -91,7 +91,7 @@ TRAFFIC = {
                          "bit_blockwise_weight_nf4_b200/csrc/lut.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "d61b00920d6acca30e379dc6307dfa89c81efab52e2cd0a236a64877190e9a75"},
+             "sha256": "155c4583b331eefd7956298f06593264c63f75e4b1baabba5b731a58ed64d8f8"},
     "gemm": {"bytes": 37468818,
              "launch": "one prefill GEMM launch, averaged over the seven Llama-7B linears",
              "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemm.cu",

@@ -36,6 +36,8 @@
 //  * Every mbarrier wait is bounded in time; on expiry the CTA sets the
 //    library's device error word, drains what it started and exits.
 //  No TMA load uses cluster multicast.
+#include <atomic>
+
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -456,7 +458,8 @@ template <int BS, int QT, bool DQ, int F>
 cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W,
                      int64_t N, void* Y, const void* bias, int* err, uint64_t wait_limit_ns,
                      int withhold, cudaStream_t s) {
-  static bool attr_set[64] = {};  // per device
+  // per device; a race only repeats the (idempotent) attribute call
+  static std::atomic<bool> attr_set[64];
   auto kern = gemm4_kernel<BS, QT, DQ, F>;
   constexpr CUtensorMapDataType kT16 =
       F == BNB4_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
@@ -464,10 +467,10 @@ cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W,
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_relaxed)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_relaxed);
   }
   CUtensorMap mx, mw, my;
   if (!make_map_2d(&mx, kT16, X, K, M, K * 2, BK, BM,

@@ -38,6 +38,8 @@
 //    library's device error word, drains what it started and still reaches
 //    both cluster barriers, so its peers never wait on it.
 //  No TMA load uses cluster multicast.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100.cuh"
@@ -418,17 +420,18 @@ template <int BS, int QT, bool DQ, int F>
 cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W, int64_t N,
                      void* Y, const void* bias, int* err, int num_sms, uint64_t wait_limit_ns,
                      cudaStream_t s) {
-  static bool attr_set[64] = {};  // per device
+  // per device; a race only repeats the (idempotent) attribute call
+  static std::atomic<bool> attr_set[64];
   auto kern = gemm_small_kernel<BS, QT, DQ, F>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_relaxed)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem_bytes(kMaxNT));
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_relaxed);
   }
   const int nt = static_cast<int>((M + 15) / 16 * 16);
   uint32_t cols = 32;

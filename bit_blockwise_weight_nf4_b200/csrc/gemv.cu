@@ -36,6 +36,8 @@
 //    the A operand, 16 rows; x as B, batch columns): K is permuted
 //    identically in both operands, which leaves the dot products unchanged.
 //    Lanes of batch columns beyond B hold zeros and load nothing.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "lut.cuh"
@@ -541,16 +543,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int BS, int QT, bool DQ, int F, int MAXP, bool QUAD>
 cudaError_t launch_k(const Group<MAXP>& grp, int num_sms, cudaStream_t s) {
   auto kern = gemv4_kernel<BS, QT, DQ, F, MAXP, QUAD>;
-  static bool attr_set[64] = {};  // per device
+  // per device; a race only repeats the (idempotent) attribute call
+  static std::atomic<bool> attr_set[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!attr_set[dev]) {
+  if (!attr_set[dev].load(std::memory_order_relaxed)) {
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kSmemBytes));
     if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_relaxed);
   }
   const int64_t grid = grp.n_rg < num_sms ? grp.n_rg : num_sms;
   return launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmemBytes, s,
