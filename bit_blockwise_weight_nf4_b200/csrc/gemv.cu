@@ -192,24 +192,17 @@ struct Pos {
   __device__ void seek(const Group<MAXP>& grp, int rg_, int kc_, int p_from) {
     rg = rg_;
     kc = kc_;
-    p = 0;
-    next_rg0 = 0x7fffffff;
-    if constexpr (MAXP > 1) {
-      p = p_from;
-      while (p + 1 < grp.count && rg >= grp.p[p + 1].rg0) ++p;
-      next_rg0 = p + 1 < grp.count ? grp.p[p + 1].rg0 : 0x7fffffff;
-    }
+    p = p_from;
+    while (p + 1 < grp.count && rg >= grp.p[p + 1].rg0) ++p;
+    next_rg0 = p + 1 < grp.count ? grp.p[p + 1].rg0 : 0x7fffffff;
   }
   // to the next item; true when that item begins a new row group
   __device__ bool step(const Group<MAXP>& grp) {
     if (++kc < grp.C) return false;
     kc = 0;
-    ++rg;
-    if constexpr (MAXP > 1) {
-      if (rg >= next_rg0) {
-        ++p;
-        next_rg0 = p + 1 < grp.count ? grp.p[p + 1].rg0 : 0x7fffffff;
-      }
+    if (++rg >= next_rg0) {
+      ++p;
+      next_rg0 = p + 1 < grp.count ? grp.p[p + 1].rg0 : 0x7fffffff;
     }
     return true;
   }
