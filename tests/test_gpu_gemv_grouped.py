@@ -121,3 +121,15 @@ def test_outputs_do_not_spill(persist):
     xb = synth.bf16_bits(x)
     check_linear(cpu_bits(y1), oracle.linear_ref(xb, W1), xb, W1)
     check_linear(cpu_bits(y2), oracle.linear_ref(xb, W2), xb, W2)
+
+
+@pytest.mark.parametrize("B", [1, 8])
+def test_full_size_layer_lists(B, persist):
+    """A Llama-7B layer's decode launches at full size, as the bench makes
+    them: q / k / v (three 4096 x 4096, one x), gate / up (two 11008 x 4096,
+    one x), and the six K = 4096 linears in one list; every output checked
+    against the oracle."""
+    run_group([(4096, 4096)] * 3, B, share_x=True, seed=300 + B, persist=persist)
+    run_group([(11008, 4096)] * 2, B, share_x=True, seed=310 + B, persist=persist)
+    run_group([(4096, 4096)] * 4 + [(11008, 4096)] * 2, B, share_x=True, seed=320 + B,
+              persist=persist)
