@@ -580,6 +580,22 @@ def oracle_baseline():
     }, **host_description())
 
 
+def arm_config(args, world, stack_state_bytes):
+    """The `config` of both arms' lines (the reference arm times the same
+    metric, configuration 5's state bytes per second, on a sample)."""
+    return {"workload": WORKLOAD, "layers": args.layers,
+            "value": "configuration 5: 4-bit weight state bytes of the stack "
+                     "(codes + 8-bit scales + group scales, %.3f GB) per GEMV pass "
+                     "time, 4 launches per layer (q/k/v grouped, o, gate/up grouped, "
+                     "down)" % (stack_state_bytes / 1e9),
+            "weight_format": "nf4 unless named, blocksize 64 unless named, double quant",
+            "l2": "no flush: every row runs on its own buffers, each call on a "
+                  "different copy, and the 3.34 GB stack pass evicts L2 between steps",
+            "parallelism": "replicas x%d" % world,
+            "launch": "eager, one call per kernel" if args.eager
+                      else "the timed steps replayed as one CUDA graph"}
+
+
 def run_reference(args):
     """The oracle as the reference arm: each step is one linear of layers 0
     and 31 of the configuration-5 stack (dequantize + fp64 dot products),
@@ -607,11 +623,13 @@ def run_reference(args):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": wall / max(1, args.steps) * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": "configuration 5 (batch-1 GEMV through the Llama-7B-shaped "
-                               "NF4 stack), CPU oracle, one linear of layers 0 / 31 per step"},
+        "config": arm_config(args, world, sum(state_bytes(lin.N * lin.K)
+                                              for lin in synth.llama7b_layer()) * args.layers),
         "cpu_baseline": dict({"value": v, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                              "sample": "one linear of layers 0 / 31 per step, cycling "
-                                        "(%d steps)" % max(1, args.steps)},
+                              "sample": "configuration 5 through the CPU oracle "
+                                        "(dequantize + fp64 dot products): one linear of "
+                                        "layers 0 / 31 per step, cycling (%d steps)"
+                                        % max(1, args.steps)},
                              **host_description()),
         "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
@@ -770,17 +788,7 @@ def run_ours(args):
         "steps": args.steps, "warmup": warm,
         "ms_per_step": elapsed_max / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "layers": args.layers,
-                   "value": "configuration 5: 4-bit weight state bytes of the stack "
-                            "(codes + 8-bit scales + group scales, %.3f GB) per GEMV pass "
-                            "time, 4 launches per layer (q/k/v grouped, o, gate/up grouped, "
-                            "down)" % (stack["state_bytes"] / 1e9),
-                   "weight_format": "nf4 unless named, blocksize 64 unless named, double quant",
-                   "l2": "no flush: every row runs on its own buffers, each call on a "
-                         "different copy, and the 3.34 GB stack pass evicts L2 between steps",
-                   "parallelism": "replicas x%d" % world,
-                   "launch": "eager, one call per kernel" if args.eager
-                             else "the timed steps replayed as one CUDA graph"},
+        "config": arm_config(args, world, stack["state_bytes"]),
         "roofline": roofline,
         "rows": out_rows,
         "gpu_launches": step.kernels() * args.steps,
