@@ -92,12 +92,13 @@ TRAFFIC = {
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
              "sha256": "155c4583b331eefd7956298f06593264c63f75e4b1baabba5b731a58ed64d8f8"},
-    "gemm": {"bytes": 37468818,
-             "launch": "one prefill GEMM launch, averaged over the seven Llama-7B linears",
+    "gemm": {"bytes": 46747904,
+             "launch": "one prefill GEMM launch (M = 2048), averaged over the three "
+                       "Llama-7B shapes",
              "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemm.cu",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "82bff8b020a3a34fcf3c9d310104139b8333349765e4ae10d819569003c77780"},
+             "sha256": "430335f4939ab63719772ac4c187790daa3b6f8796b5302ae4904d1428671381"},
 }
 
 
