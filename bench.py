@@ -82,7 +82,7 @@ TRAFFIC = {
     # 23.29 MB) and the persistent one on the six K = 4096 linears of a layer
     # (81.28 / 81.27 MB); the family's traffic per launch is that ratio times
     # its algorithmic bytes per launch
-    "gemv": {"ratio": (23.294208 + 81.275648) / (23.290112 + 81.265152),
+    "gemv": {"ratio": (23.294208 + 81.26976) / (23.290112 + 81.265152),
              "launch": "cold captures of both decode kernels (11008 x 4096 single; the "
                        "six K = 4096 linears of a layer in one persistent launch), scaled "
                        "by the algorithmic bytes per launch of the family",
@@ -91,7 +91,7 @@ TRAFFIC = {
                          "bit_blockwise_weight_nf4_b200/csrc/lut.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "155c4583b331eefd7956298f06593264c63f75e4b1baabba5b731a58ed64d8f8"},
+             "sha256": "4f48759c00353cd1e3d085d2bfbe4357e535aa7c8547871ac8973d3f626ea7ab"},
     "gemm": {"bytes": 46747904,
              "launch": "one prefill GEMM launch (M = 2048), averaged over the three "
                        "Llama-7B shapes",
