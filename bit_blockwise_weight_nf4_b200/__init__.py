@@ -41,7 +41,7 @@ F32 = 0
 BF16 = 1
 F16 = 2
 
-ABI_VERSION = 3
+ABI_VERSION = 4
 GROUP_MAX = 256
 
 

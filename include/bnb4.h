@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define BNB4_ABI_VERSION 3
+#define BNB4_ABI_VERSION 4
 
 /* Every entry point is exported from the shared library (the library is
  * built with hidden visibility by default). */
