@@ -91,7 +91,7 @@ TRAFFIC = {
                          "bit_blockwise_weight_nf4_b200/csrc/lut.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "4f48759c00353cd1e3d085d2bfbe4357e535aa7c8547871ac8973d3f626ea7ab"},
+             "sha256": "dc9f9b3f31cdabf13a388f11b27b5f2cb4f077bc5be75e4054f962eac4ceffdf"},
     "gemm": {"bytes": 46747904,
              "launch": "one prefill GEMM launch (M = 2048), averaged over the three "
                        "Llama-7B shapes",

@@ -275,38 +275,36 @@ struct Fetch {
       }
       cp_async4_part(smem_u32(sc + lane), src, bytes);
       qb += kItemK / BS;
-      if (pos.step(grp)) enter();
-      return;
     } else {
-    const int koff = pos.kc * kItemK + 64 * t;  // the lane's K segment
-    const bool seg = koff < grp.K;
-    const bool v0 = seg && ok0, v1 = seg && ok1;
-    const int64_t b0 = blk0 + koff / BS;
-    const int64_t b1 = b0 + static_cast<int64_t>(8) * grp.kb;
+      const int koff = pos.kc * kItemK + 64 * t;  // the lane's K segment
+      const bool seg = koff < grp.K;
+      const bool v0 = seg && ok0, v1 = seg && ok1;
+      const int64_t b0 = blk0 + koff / BS;
+      const int64_t b1 = b0 + static_cast<int64_t>(8) * grp.kb;
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      if (!(r ? v1 : v0)) continue;
-      const int64_t b = r ? b1 : b0;
-      if constexpr (DQ) {
-        // the aligned 4-byte word holding u_b (and u_{b+1} at blocksize 32:
-        // b is even), cut at the end of the array in the last row group
-        const int64_t wb = b & ~int64_t(3);
-        if (last) {
-          const int64_t rest = nb - wb;
-          cp_async4_part(smem_u32(sc + r * 32 + lane), aq + wb,
-                         static_cast<uint32_t>(rest < 4 ? rest : 4));
+      for (int r = 0; r < 2; ++r) {
+        if (!(r ? v1 : v0)) continue;
+        const int64_t b = r ? b1 : b0;
+        if constexpr (DQ) {
+          // the aligned 4-byte word holding u_b (and u_{b+1} at blocksize 32:
+          // b is even), cut at the end of the array in the last row group
+          const int64_t wb = b & ~int64_t(3);
+          if (last) {
+            const int64_t rest = nb - wb;
+            cp_async4_part(smem_u32(sc + r * 32 + lane), aq + wb,
+                           static_cast<uint32_t>(rest < 4 ? rest : 4));
+          } else {
+            cp_async4(smem_u32(sc + r * 32 + lane), aq + wb);
+          }
+          cp_async4(smem_u32(sc + (2 + r) * 32 + lane), s2 + (b >> 8));
         } else {
-          cp_async4(smem_u32(sc + r * 32 + lane), aq + wb);
+          const float* am = grp.p[pos.p].absmax;
+          cp_async4(smem_u32(sc + r * 32 + lane), am + b);
+          if constexpr (BS == 32) cp_async4(smem_u32(sc + (2 + r) * 32 + lane), am + b + 1);
         }
-        cp_async4(smem_u32(sc + (2 + r) * 32 + lane), s2 + (b >> 8));
-      } else {
-        const float* am = grp.p[pos.p].absmax;
-        cp_async4(smem_u32(sc + r * 32 + lane), am + b);
-        if constexpr (BS == 32) cp_async4(smem_u32(sc + (2 + r) * 32 + lane), am + b + 1);
       }
     }
     if (pos.step(grp)) enter();
-    }
   }
 };
 
