@@ -77,12 +77,13 @@ GEMV_WEIGHTS = 4
 ALU_OPS_PER_WEIGHT = 2.5
 
 TRAFFIC = {
-    # decode: DRAM bytes over algorithmic bytes of cold launches of both
-    # decode kernels -- the one-CTA-per-16-rows one on 11008 x 4096 (23.29 /
-    # 23.29 MB) and the persistent one on the six K = 4096 linears of a layer
-    # (81.28 / 81.27 MB); the family's traffic per launch is that ratio times
-    # its algorithmic bytes per launch
-    "gemv": {"ratio": (23.294208 + 81.26976) / (23.290112 + 81.265152),
+    # decode: DRAM bytes (read + write) over algorithmic bytes of cold
+    # launches of both decode kernels -- the one-CTA-per-16-rows one on 11008
+    # x 4096 (23.30 MB read, none written / 23.29 MB) and the persistent one
+    # on the six K = 4096 linears of a layer (81.27 MB read + 1.85 MB written
+    # / 81.27 MB); the family's traffic per launch is that ratio times its
+    # algorithmic bytes per launch
+    "gemv": {"ratio": (23.295488 + 0.0 + 81.269248 + 1.85472) / (23.290112 + 81.265152),
              "launch": "cold captures of both decode kernels (11008 x 4096 single; the "
                        "six K = 4096 linears of a layer in one persistent launch), scaled "
                        "by the algorithmic bytes per launch of the family",
@@ -91,14 +92,14 @@ TRAFFIC = {
                          "bit_blockwise_weight_nf4_b200/csrc/lut.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "dc9f9b3f31cdabf13a388f11b27b5f2cb4f077bc5be75e4054f962eac4ceffdf"},
-    "gemm": {"bytes": 46747904,
+             "sha256": "339896f7449ea181d4597fd27726f811859820459be74ae9637b7ee653aa94b9"},
+    "gemm": {"bytes": 46757632,
              "launch": "one prefill GEMM launch (M = 2048), averaged over the three "
                        "Llama-7B shapes",
              "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemm.cu",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "430335f4939ab63719772ac4c187790daa3b6f8796b5302ae4904d1428671381"},
+             "sha256": "a54616d3a1b8727283a17c823e354e9f1845fb2872349884f2353fff5b5f0d72"},
 }
 
 

@@ -132,14 +132,16 @@ inline View2D make_view(int64_t cols, int64_t ld) {
   return View2D{cols, ld, ~0ull / static_cast<uint64_t>(cols) + 1ull};
 }
 
-// Programmatic dependent launch, used only inside one API call: a kernel
-// whose predecessor on the stream is the library's own previous kernel of the
-// same call (the double-quant kernel after the quantize kernel) is launched
-// with programmatic stream serialization, so it may be scheduled while that
-// kernel finishes; it waits for it with pdl_wait before touching global
-// memory.  The first kernel of every call launches normally: the caller's
-// previous work on the stream may be a copy, which a programmatic launch
-// would not wait for.  Both device calls are no-ops without such a launch.
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the kernel before it on the stream is still
+// running, but only once that kernel's CTAs have all called pdl_trigger (a
+// kernel that never calls it releases its dependent when it finishes); any
+// other predecessor (a copy, an event wait) stays a full dependency.  Such a
+// kernel must wait with pdl_wait -- which returns once the previous kernel
+// has completed and its writes are visible -- before it touches global
+// memory.  Used by the double-quant kernel (its predecessor is the quantize
+// kernel of the same call) and by the one-CTA-per-16-rows decode kernel
+// (any predecessor).  Both device calls are no-ops without such a launch.
 __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
