@@ -80,10 +80,10 @@ TRAFFIC = {
     # decode: DRAM bytes (read + write) over algorithmic bytes of cold
     # launches of both decode kernels -- the one-CTA-per-16-rows one on 11008
     # x 4096 (23.30 MB read, none written / 23.29 MB) and the persistent one
-    # on the six K = 4096 linears of a layer (81.27 MB read + 1.85 MB written
+    # on the six K = 4096 linears of a layer (81.27 MB read + 1.60 MB written
     # / 81.27 MB); the family's traffic per launch is that ratio times its
     # algorithmic bytes per launch
-    "gemv": {"ratio": (23.295488 + 0.0 + 81.269248 + 1.85472) / (23.290112 + 81.265152),
+    "gemv": {"ratio": (23.295744 + 0.0 + 81.270272 + 1.603584) / (23.290112 + 81.265152),
              "launch": "cold captures of both decode kernels (11008 x 4096 single; the "
                        "six K = 4096 linears of a layer in one persistent launch), scaled "
                        "by the algorithmic bytes per launch of the family",
@@ -92,14 +92,14 @@ TRAFFIC = {
                          "bit_blockwise_weight_nf4_b200/csrc/lut.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "339896f7449ea181d4597fd27726f811859820459be74ae9637b7ee653aa94b9"},
-    "gemm": {"bytes": 46757632,
+             "sha256": "fdbacc61c183ebb3cdf21dbfd638c57c2380f62d97b361ea4bb771f2720a81f4"},
+    "gemm": {"bytes": 46650539,
              "launch": "one prefill GEMM launch (M = 2048), averaged over the three "
                        "Llama-7B shapes",
              "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemm.cu",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "a54616d3a1b8727283a17c823e354e9f1845fb2872349884f2353fff5b5f0d72"},
+             "sha256": "d4118c9347efde041777b671106ba31eb1b5c6e2fa733c5403ff3dced1b8c0a5"},
 }
 
 

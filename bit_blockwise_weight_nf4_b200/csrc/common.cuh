@@ -139,9 +139,11 @@ inline View2D make_view(int64_t cols, int64_t ld) {
 // other predecessor (a copy, an event wait) stays a full dependency.  Such a
 // kernel must wait with pdl_wait -- which returns once the previous kernel
 // has completed and its writes are visible -- before it touches global
-// memory.  Used by the double-quant kernel (its predecessor is the quantize
-// kernel of the same call) and by the one-CTA-per-16-rows decode kernel
-// (any predecessor).  Both device calls are no-ops without such a launch.
+// memory.  Every kernel of the library (but the reciprocal check's) launches
+// this way and calls pdl_trigger at entry, so back-to-back calls overlap one
+// kernel's last wave with the next one's launch; the double-quant kernel's
+// predecessor is always the quantize kernel of the same call.  Both device
+// calls are no-ops without such a launch.
 __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }

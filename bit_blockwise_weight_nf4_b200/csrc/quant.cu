@@ -308,9 +308,13 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
   extern __shared__ uint2 lut[];
   __shared__ double red[kThreads / 32];
-  pdl_trigger();  // the double-quant kernel may be scheduled early
+  // programmatic dependent launch: the next kernel (the double-quant kernel)
+  // may be scheduled early; the table is built while the previous kernel on
+  // the stream finishes, and nothing global is touched before it has
+  pdl_trigger();
   build_lut<QT>(lut);
   __syncthreads();
+  pdl_wait();
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -422,10 +426,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 // Double quantization of the absmax array: one warp per group of 256 blocks
 // (grid-strided over the groups).  Every CTA first reduces the per-CTA
 // partial sums of the quantize kernel in the same fixed order -- thread i
-// adds partials i, i + 256, ... (independent loads, one round trip), then a
-// fixed xor tree per warp and the 8 warp sums in order -- so all CTAs agree
-// on the offset; the sum is exact whenever the absmax values span few
-// enough binades, and then equals the oracle's sequential sum.
+// adds partials i, i + 256, ... (independent loads, one round trip, shared
+// with the loads of the warp's first group), then a fixed xor tree per warp
+// and the 8 warp sums in order -- so all CTAs agree on the offset; the sum
+// is exact whenever the absmax values span few enough binades, and then
+// equals the oracle's sequential sum.
 constexpr int kDqThreads = 256;
 
 __global__ void __launch_bounds__(kDqThreads)
@@ -436,7 +441,23 @@ __global__ void __launch_bounds__(kDqThreads)
   __shared__ double red[kDqThreads / 32];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  const int64_t ng = (nb + 255) / 256;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * (kDqThreads / 32);
+  int64_t g = static_cast<int64_t>(blockIdx.x) * (kDqThreads / 32) + warp;
+  // entries g*256 + lane + 32 j of the warp's group (coalesced); 0 past nb
+  auto load_group = [&](int64_t grp, float (&a)[8]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t b = grp * 256 + lane + 32 * j;
+      a[j] = grp < ng && b < nb ? __ldg(absmax + b) : 0.0f;
+    }
+  };
+  pdl_trigger();
   pdl_wait();  // the quantize kernel's absmax and partial sums are complete
+  // the warp's first group is requested together with the partial sums, so
+  // the two loads share one round trip
+  float a[8];
+  load_group(g, a);
   double sum = 0.0;
   for (int i = threadIdx.x; i < n_partials; i += kDqThreads) sum += partials[i];
 #pragma unroll
@@ -449,18 +470,16 @@ __global__ void __launch_bounds__(kDqThreads)
   const float off = static_cast<float>(sum / static_cast<double>(nb));
   if (blockIdx.x == 0 && threadIdx.x == 0) offset[0] = off;
 
-  const int64_t ng = (nb + 255) / 256;
-  const int64_t stride = static_cast<int64_t>(gridDim.x) * (kDqThreads / 32);
-  for (int64_t g = static_cast<int64_t>(blockIdx.x) * (kDqThreads / 32) + warp; g < ng;
-       g += stride) {
+  for (; g < ng; g += stride) {
     float c[8];
     float m = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {  // entry g*256 + lane + 32 j (coalesced)
+    for (int j = 0; j < 8; ++j) {
       const int64_t b = g * 256 + lane + 32 * j;
-      c[j] = b < nb ? __fsub_rn(__ldg(absmax + b), off) : 0.0f;
+      c[j] = b < nb ? __fsub_rn(a[j], off) : 0.0f;
       m = fmaxf(m, fabsf(c[j]));
     }
+    load_group(g + stride, a);  // the next group of this warp (zeros past ng)
 #pragma unroll
     for (int o = 16; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     const float sg = __fdiv_rn(m, 127.0f);
@@ -519,9 +538,9 @@ cudaError_t launch_quant(const void* x, int64_t n, uint8_t* codes,
   const size_t smem = kLutEntries * 32 * sizeof(uint2);
   if (view)
     return launch_kernel(quant4_kernel<T, BS, QT, DQ, true>, dim3(grid), dim3(kThreads), smem,
-                         s, false, static_cast<const T*>(x), n, codes, absmax, partials, *view);
+                         s, true, static_cast<const T*>(x), n, codes, absmax, partials, *view);
   return launch_kernel(quant4_kernel<T, BS, QT, DQ, false>, dim3(grid), dim3(kThreads), smem, s,
-                       false, static_cast<const T*>(x), n, codes, absmax, partials, View2D{});
+                       true, static_cast<const T*>(x), n, codes, absmax, partials, View2D{});
 }
 
 template <typename T, int QT, bool DQ>
