@@ -56,17 +56,19 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "4-bit GEMV weight-GB/s & GEMM TFLOPS; quant/dequant GB/s; % of roofline"
-WORKLOAD = ("five workloads per step, each row isolated on its own buffers: "
+WORKLOAD = ("five configurations per step, each row isolated on its own buffers: "
             "cfg1 NF4 round trip fp32 2^20; cfg2 NF4/FP4 quantize+dequantize bf16 "
             "4096x4096 with outliers; cfg3 GEMV B=1,8 on 11008x4096 and 4096x11008; "
             "cfg4 GEMM M=2048 on the three Llama-7B shapes, NF4 bs64/bs128, FP4; "
             "cfg5 batch-1 GEMV through the 224 linears of a 32-layer "
-            "Llama-7B-shaped NF4 stack, per-layer launches (value)")
+            "Llama-7B-shaped NF4 stack, per-layer launches (value); plus the "
+            "small-batch linear (16 and 64 token rows) on the three Llama-7B shapes")
 GEMM_M = 2048
 BS = 64
 ROUNDTRIP_COPIES = 8
 MATRIX_COPIES = 4
 GEMV_WEIGHTS = 4
+SMALL_BATCH_ROWS = (16, 64)  # token rows of the small-batch linear rows
 
 # DRAM bytes (read + write) per launch of a kernel family, from one ncu
 # capture each, with the sources hashed at capture time: a figure is
@@ -79,11 +81,11 @@ ALU_OPS_PER_WEIGHT = 2.5
 TRAFFIC = {
     # decode: DRAM bytes (read + write) over algorithmic bytes of cold
     # launches of both decode kernels -- the one-CTA-per-16-rows one on 11008
-    # x 4096 (23.30 MB read, none written / 23.29 MB) and the persistent one
-    # on the six K = 4096 linears of a layer (81.27 MB read + 1.60 MB written
+    # x 4096 (23.29 MB read, none written / 23.29 MB) and the persistent one
+    # on the six K = 4096 linears of a layer (81.27 MB read + 2.18 MB written
     # / 81.27 MB); the family's traffic per launch is that ratio times its
     # algorithmic bytes per launch
-    "gemv": {"ratio": (23.295744 + 0.0 + 81.270272 + 1.603584) / (23.290112 + 81.265152),
+    "gemv": {"ratio": (23.294976 + 0.0 + 81.270528 + 2.18112) / (23.290112 + 81.265152),
              "launch": "cold captures of both decode kernels (11008 x 4096 single; the "
                        "six K = 4096 linears of a layer in one persistent launch), scaled "
                        "by the algorithmic bytes per launch of the family",
@@ -92,14 +94,14 @@ TRAFFIC = {
                          "bit_blockwise_weight_nf4_b200/csrc/lut.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "fdbacc61c183ebb3cdf21dbfd638c57c2380f62d97b361ea4bb771f2720a81f4"},
-    "gemm": {"bytes": 46650539,
+             "sha256": "d3a5f296dffea75f39e8a2519ea7ea9b9a6710c909f0b362592f23a426563805"},
+    "gemm": {"bytes": 46616405,
              "launch": "one prefill GEMM launch (M = 2048), averaged over the three "
                        "Llama-7B shapes",
              "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemm.cu",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "d4118c9347efde041777b671106ba31eb1b5c6e2fa733c5403ff3dced1b8c0a5"},
+             "sha256": "1763052f05d76596be2ee0e094e36538f220d72c9e50b22d1e12f01cf4fc2b44"},
 }
 
 
@@ -285,13 +287,15 @@ def gemv_bytes(N, K, B, bs=BS):
 
 # ---------------------------------------------------------------- rows
 class Call:
-    """One C-ABI launch: the entry point, its arguments (raw pointers) and
+    """One C-ABI call: the entry point, its arguments (raw pointers) and
     the tensors those pointers point into, held for as long as the call may
     run; the stream is torch's current one at call time (the capture stream
-    while a graph is being captured)."""
+    while a graph is being captured).  `launches`: how many times the call
+    launches its row's kernels (a grouped decode call launches once per 32
+    linears)."""
 
-    def __init__(self, fn, *args, keep=()):
-        self.fn, self.args, self.keep = fn, args, keep
+    def __init__(self, fn, *args, keep=(), launches=1):
+        self.fn, self.args, self.keep, self.launches = fn, args, keep, launches
 
     def __call__(self):
         import bit_blockwise_weight_nf4_b200 as b
@@ -385,6 +389,24 @@ def build_rows(dev, n_layers):
                             gemv_bytes(N, K, Bt), [gemv_call(x, s, N, y) for s in sts], 1,
                             weight_bytes=N * K // 2))
 
+    # the small-batch linear (16 and 64 token rows) on the three Llama-7B
+    # shapes, through bnb_gemm_4bit: 16 rows run the decode kernel's 16-row
+    # form, 64 the small-batch tcgen05 kernel
+    for M in SMALL_BATCH_ROWS:
+        for N, K in synth.GEMM_SHAPES:
+            X = synth.activations_bf16(M, K, seed=2, device=dev)
+            sts = []
+            for i in range(GEMV_WEIGHTS):
+                w = synth.weight_bf16(N, K, seed=500 + M + 10 * i + N // 1024, device=dev)
+                sts.append(b.quantize_4bit(w.view(-1), BS, b.NF4, True))
+                del w
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            rows.append(Row("f1_linear_m%d_%dx%d" % (M, N, K), "f1", "small", "hbm",
+                            gemv_bytes(N, K, M),
+                            [Call(b.bnb_gemm_4bit, X.data_ptr(), M, K, s.cstruct(), N,
+                                  Y.data_ptr(), keep=(X, s, Y)) for s in sts], 1,
+                            weight_bytes=N * K // 2))
+
     # cfg4: prefill GEMM
     def gemm_call(X, st, N, Y):
         M, K = X.shape
@@ -444,7 +466,8 @@ def build_rows(dev, n_layers):
             probs[j] = b.GemvProblem(xk[lin.K].data_ptr(), states[i].cstruct(), lin.K, lin.N,
                                      None, ys[i].data_ptr())
         return Call(b.bnb_gemv_4bit_grouped, probs, 1, b.BF16,
-                    keep=[states[i] for i in idx] + [ys[i] for i in idx] + list(xk.values()))
+                    keep=[states[i] for i in idx] + [ys[i] for i in idx] + list(xk.values()),
+                    launches=(len(idx) + 31) // 32)
 
     # the decoder's natural launches per layer: q/k/v (one input), o,
     # gate/up (one input), down
@@ -496,7 +519,7 @@ class Step:
             events[-1].record()
 
     def kernels(self):
-        return sum(r.kpc * len(r.calls) for r in self.rows)
+        return sum(r.kpc * sum(c.launches for c in r.calls) for r in self.rows)
 
 
 # ------------------------------------------------------------ CPU oracle
@@ -729,7 +752,8 @@ def run_ours(args):
         if r.cfg == "cfg5":
             t = per_call[r.name] * len(r.calls)
             out_rows[r.name].update({
-                "ms_per_pass": t * 1e3, "launches_per_pass": len(r.calls),
+                "ms_per_pass": t * 1e3,
+                "launches_per_pass": sum(c.launches for c in r.calls),
                 "state_GB/s": stack["state_bytes"] / t / 1e9,
                 "state_bytes_per_pass": stack["state_bytes"],
                 "target_ms_at_70pct_hbm":
@@ -747,7 +771,7 @@ def run_ours(args):
         f = fam.setdefault(r.family, {"s": 0.0, "work": 0.0, "launches": 0, "bound": r.bound})
         f["s"] += per_call[r.name] * len(r.calls)
         f["work"] += r.work * len(r.calls)
-        f["launches"] += len(r.calls)
+        f["launches"] += r.kpc * sum(c.launches for c in r.calls)
     dom_name = max(fam, key=lambda k: fam[k]["s"])
     dom = fam[dom_name]
     tr = traffic_of(dom_name)

@@ -254,11 +254,18 @@ int dequantize_impl(const bnb4_qstate* st, void* out, int32_t out_dtype, void* s
                                            static_cast<cudaStream_t>(stream), view));
 }
 
-// Kernel choice by the number of token rows: the mma.sync GEMV up to 8 (one
-// MMA column group), the small-M tcgen05 kernel (weight rows as the MMA's M,
-// K split over a cluster) up to 256, the 2-CTA tcgen05 GEMM above.
+// Kernel choice by the number of token rows: the mma.sync GEMV up to 8 (x
+// as the MMA's B operand), and from 9 to 16 when x and the codes are 32-byte
+// aligned (x as its A operand; measured faster than the small-M kernel on
+// the Llama-7B shapes), the small-M tcgen05 kernel (weight rows as the MMA's
+// M, K split over a cluster) up to 256, the 2-CTA tcgen05 GEMM above.
+// Grouped decode calls take up to 8 rows.
 constexpr int64_t kGemvMaxB = 8;
 constexpr int64_t kSmallMaxM = 256;
+
+bool use_gemv(const void* x, const bnb4_qstate& W, int64_t M) {
+  return M <= kGemvMaxB || bnb4::gemv_direct_takes(x, W, M);
+}
 
 }  // namespace
 
@@ -347,7 +354,7 @@ int bnb_gemv_4bit(const void* x, int64_t B, int64_t K, const bnb4_qstate* W,
   if ((rc = check_linear_memory(x, y, nullptr, W)) != BNB4_OK) return rc;
   int* err;
   if ((rc = error_word(&err)) != BNB4_OK) return rc;
-  if (B <= kGemvMaxB)
+  if (use_gemv(x, *W, B))
     return from_cuda(bnb4::launch_gemv(x, B, K, *W, N, y, nullptr, BNB4_BF16, sms, err,
                                        static_cast<cudaStream_t>(stream)));
   return from_cuda(bnb4::launch_gemm_small(x, B, K, *W, N, y, nullptr, BNB4_BF16, err, sms,
@@ -414,7 +421,7 @@ int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstate* W,
   if ((rc = check_linear_memory(X, Y, nullptr, W)) != BNB4_OK) return rc;
   int* err;
   if ((rc = error_word(&err)) != BNB4_OK) return rc;
-  if (M <= kGemvMaxB)
+  if (use_gemv(X, *W, M))
     return from_cuda(bnb4::launch_gemv(X, M, K, *W, N, Y, nullptr, BNB4_BF16, sms, err,
                                        static_cast<cudaStream_t>(stream)));
   if (M <= kSmallMaxM)
@@ -441,7 +448,7 @@ int bnb_linear_4bit(const void* x, int32_t dtype, int64_t M, int64_t K, const bn
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* err;
   if ((rc = error_word(&err)) != BNB4_OK) return rc;
-  if (M <= kGemvMaxB)
+  if (use_gemv(x, *W, M))
     return from_cuda(bnb4::launch_gemv(x, M, K, *W, N, y, bias, dtype, sms, err, s));
   if (M <= kSmallMaxM)
     return from_cuda(bnb4::launch_gemm_small(x, M, K, *W, N, y, bias, dtype, err, sms, s));

@@ -69,6 +69,27 @@ __device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
   return r;
 }
 
+// 256-bit loads (sm_100): the address must be 32-byte aligned.
+struct U8x32 {
+  uint32_t v[8];
+};
+__device__ __forceinline__ U8x32 ldg_v8(const void* p) {
+  U8x32 r;
+  asm volatile("ld.global.nc.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r.v[0]), "=r"(r.v[1]), "=r"(r.v[2]), "=r"(r.v[3]), "=r"(r.v[4]),
+                 "=r"(r.v[5]), "=r"(r.v[6]), "=r"(r.v[7])
+               : "l"(p));
+  return r;
+}
+__device__ __forceinline__ U8x32 ldg_stream_v8(const void* p) {
+  U8x32 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r.v[0]), "=r"(r.v[1]), "=r"(r.v[2]), "=r"(r.v[3]), "=r"(r.v[4]),
+                 "=r"(r.v[5]), "=r"(r.v[6]), "=r"(r.v[7])
+               : "l"(p));
+  return r;
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t w) {
   return __uint_as_float(w << 16);
 }
@@ -132,18 +153,16 @@ inline View2D make_view(int64_t cols, int64_t ld) {
   return View2D{cols, ld, ~0ull / static_cast<uint64_t>(cols) + 1ull};
 }
 
-// Programmatic dependent launch.  A kernel launched with programmatic stream
-// serialization may start while the kernel before it on the stream is still
-// running, but only once that kernel's CTAs have all called pdl_trigger (a
-// kernel that never calls it releases its dependent when it finishes); any
-// other predecessor (a copy, an event wait) stays a full dependency.  Such a
-// kernel must wait with pdl_wait -- which returns once the previous kernel
-// has completed and its writes are visible -- before it touches global
-// memory.  Every kernel of the library (but the reciprocal check's) launches
-// this way and calls pdl_trigger at entry, so back-to-back calls overlap one
-// kernel's last wave with the next one's launch; the double-quant kernel's
-// predecessor is always the quantize kernel of the same call.  Both device
-// calls are no-ops without such a launch.
+// Programmatic dependent launch, used only inside one API call: a kernel
+// whose predecessor on the stream is the library's own previous kernel of the
+// same call (the double-quant kernel after the quantize kernel) is launched
+// with programmatic stream serialization, so it may be scheduled while that
+// kernel finishes; it waits for it with pdl_wait before touching global
+// memory.  The first kernel of every call launches normally: the caller's
+// previous work on the stream may be a copy, which a programmatic launch
+// would not wait for (observed on B200: a pageable host-to-device copy
+// followed by programmatic launches gave intermittent mismatches).  Both
+// device calls are no-ops without such a launch.
 __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }

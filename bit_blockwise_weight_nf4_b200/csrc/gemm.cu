@@ -139,10 +139,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   Bars* bars = reinterpret_cast<Bars*>(smem + OFF_BARS);
-  // programmatic dependent launch: no global access (and no tensor memory
-  // allocated) before the previous kernel on the stream has completed
-  pdl_trigger();
-  pdl_wait();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cta_rank();
@@ -493,15 +489,13 @@ cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W,
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = SMEM_BYTES;
   cfg.stream = s;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, mx, mw, my, static_cast<int>(M), static_cast<int>(N),
                             static_cast<int>(K), n_pair_cols, W.absmax, W.absmax_q,
                             W.scale2, W.offset, static_cast<const uint16_t*>(bias), err,

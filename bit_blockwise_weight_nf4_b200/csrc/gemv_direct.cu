@@ -3,8 +3,9 @@
 // three weights at B = 1 and every grouped call at B > 1 (lists of four or
 // more weights at B = 1 run the persistent TMA-staged kernel of gemv.cu;
 // measured side by side on B200, this one is 10-17% faster for a single
-// weight at B = 1 and 28-32% at B = 8).
-//   y[b, n] = h( sum_k x[b, k] * What[n, k] + bias[n] ),  1 <= B <= 8,
+// weight at B = 1 and 28-32% at B = 8), and of single linears with 9 to 16
+// rows of x when x and the codes are 32-byte aligned.
+//   y[b, n] = h( sum_k x[b, k] * What[n, k] + bias[n] ),  1 <= B <= 16,
 //   What[n, k] = h(RN(t[code] * a_hat))   (dequantized weight, exact),
 // h = round to the 16-bit compute format, bf16 or fp16 (nearest even); the
 // bias is optional.
@@ -18,25 +19,24 @@
 //    CTAs as row groups: the block scheduler overlaps one CTA's start-up
 //    (first loads) with other CTAs' math.  The warps split K in 256-wide
 //    steps; the 4 lanes of a quad own two rows (g and g + 8) and a
-//    contiguous 64-element segment of each per step (2 x 2 128-bit loads
-//    straight into registers); every lane keeps 2 steps of loads (codes and
-//    raw scales) in flight.
+//    contiguous 64-element segment of each per step (a 256-bit load per
+//    row straight into registers when the codes are 32-byte aligned, else
+//    two 128-bit loads); every lane keeps 2 steps of loads (codes and raw
+//    scales) in flight.
 //  * Per (row, quant block) a lane builds the 16-entry table of
 //    h(RN(t[i] * a_hat)) and looks codes up with byte permutes (lut.cuh;
 //    shift-based selectors: the multiply-high form that helps the
 //    persistent kernel measured 2-6% slower here).
 //  * The products run on mma.sync m16n8k16 with the weight as the A operand
-//    (16 rows) and x as B (batch columns, read just in time from L1): K is
-//    permuted identically in both operands, which leaves the dot products
-//    unchanged; two accumulator chains keep consecutive MMAs independent;
-//    batch columns beyond B read a valid row whose outputs are discarded.
+//    (16 rows) and x as B (batch columns, read just in time from L1, 32
+//    bytes per load when aligned): K is permuted identically in both
+//    operands, which leaves the dot products unchanged; two accumulator
+//    chains keep consecutive MMAs independent; batch columns beyond B read a
+//    valid row whose outputs are discarded.  For 9 to 16 rows the operands
+//    swap (x the A operand, each weight row set the B operand), so every
+//    weight is still dequantized once.
 //  * The 8 warps' partial sums are added in shared memory in a fixed order,
 //    the bias (if any) added in fp32, and rounded once.
-//  * Programmatic dependent launch: each CTA lets the next kernel on the
-//    stream be scheduled at once and waits for the previous one before its
-//    first global access, so back-to-back decode launches (a decoder's
-//    linears) overlap one kernel's last wave with the next one's start
-//    (measured on B200: 2.6% on a 7B decoder pass, 3-7% on single weights).
 #include "common.cuh"
 #include "kernels.h"
 #include "lut.cuh"
@@ -125,13 +125,25 @@ struct DirectList {
   int count;
 };
 
-template <int BS, int QT, bool DQ, int kDepth, int F, int MAXP>
+// V8: every x and codes array of the launch is 32-byte aligned, so a lane
+// reads a row's 32 code bytes of a step, and x for two MMAs, with one 256-bit
+// load each (half the load instructions and, for B > 1, half the L1 lines
+// that the loads of x touch: measured 7-18% faster at B = 8, up to 15% for a
+// single weight at B = 1; not used for lists at B = 1, see launch_list).
+// T16 (V8 only): 9 to 16 rows of x.  The MMAs swap roles: x is the A operand
+// (16 rows: the lane's rows g and g + 8 of x), each of the lane's two weight
+// rows the B operand of its own MMA (rows 0-7 and 8-15 of the group, one
+// accumulator each, alternating); the lane dequantizes the same two rows as
+// for B <= 8.
+template <int BS, int QT, bool DQ, int kDepth, int F, int MAXP, bool V8, bool T16>
 __global__ void __launch_bounds__(kThreads, 2)
     gemv4_direct_kernel(const __grid_constant__ DirectList<MAXP> L, int B, int64_t K) {
-  __shared__ float red[kWarps][32][4];
+  static_assert(V8 || !T16, "the 16-row form reads x with 256-bit loads");
+  constexpr int kAcc = T16 ? 2 : kChains;  // accumulators (4 floats each) per lane
+  __shared__ float red[kWarps][32][T16 ? 8 : 4];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const int g = lane >> 2;  // rows g and g + 8 of the group; batch column g of x
+  const int g = lane >> 2;  // rows g and g + 8 of the group; row(s) g (and g + 8) of x
   const int t = lane & 3;   // K segment of the step
   int pi = 0;  // this CTA's problem
   if constexpr (MAXP > 1)
@@ -150,17 +162,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int64_t n[2] = {row0 + g, row0 + g + 8};
   const bool ok[2] = {n[0] < N, n[1] < N};
   const int64_t steps = (K + kKStep - 1) / kKStep;
-  // programmatic dependent launch: the next kernel on the stream may be
-  // scheduled now; this one touches no global memory before the previous
-  // kernel has completed (x may be its output)
-  pdl_trigger();
-  pdl_wait();
   const float off = DQ ? __ldg(offset) : 0.0f;
   const int my_steps =
       warp < steps ? static_cast<int>((steps - warp + kWarps - 1) / kWarps) : 0;
-  // batch columns beyond B read row B-1 (valid memory); their outputs are
-  // never stored
+  // rows of x beyond B read row B-1 (valid memory); their outputs are never
+  // stored
   const uint16_t* xrow = x + static_cast<int64_t>(g < B ? g : B - 1) * K;
+  const uint16_t* xrow8 = x + static_cast<int64_t>(g + 8 < B ? g + 8 : B - 1) * K;
 
   auto issue = [&](int i, StepBuf& b) {
     const int64_t k0 = (static_cast<int64_t>(i) * kWarps + warp) * kKStep + 64 * t;
@@ -168,8 +176,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (int r = 0; r < 2; ++r) {
       if (ok[r] && k0 < K) {
         const uint8_t* src = codes + n[r] * (K / 2) + k0 / 2;
-        b.c[r][0] = ldg_stream_v4(src);
-        b.c[r][1] = ldg_stream_v4(src + 16);
+        if constexpr (V8) {
+          const U8x32 cc = ldg_stream_v8(src);
+          b.c[r][0] = make_uint4(cc.v[0], cc.v[1], cc.v[2], cc.v[3]);
+          b.c[r][1] = make_uint4(cc.v[4], cc.v[5], cc.v[6], cc.v[7]);
+        } else {
+          b.c[r][0] = ldg_stream_v4(src);
+          b.c[r][1] = ldg_stream_v4(src + 16);
+        }
         const int64_t blk = (n[r] * K + k0) / BS;
         b.a[r][0] = load_scale<DQ>(blk, absmax, absmax_q, scale2);
         if constexpr (BS == 32) b.a[r][1] = load_scale<DQ>(blk + 1, absmax, absmax_q, scale2);
@@ -182,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   };
 
-  float acc[kChains][4] = {};
+  float acc[kAcc][4] = {};
   StepBuf buf[kDepth];
 #pragma unroll
   for (int d = 0; d < kDepth; ++d)
@@ -206,9 +220,21 @@ __global__ void __launch_bounds__(kThreads, 2)
                           : lut[r][0];
         }
         const int64_t kx = seg ? k0 : 0;  // x stays in bounds on a ragged edge
+        U8x32 xq, xq8;  // V8: x at k0 + 8p .. +15 (rows g and g + 8)
 #pragma unroll
         for (int p = 0; p < 8; ++p) {  // codes k0 + 8p .. +7 of both rows: two MMAs
-          const uint4 xb = __ldg(reinterpret_cast<const uint4*>(xrow + kx + 8 * p));
+          uint4 xb, xc;  // x at k0 + 8p .. +7: row g (and row g + 8)
+          if constexpr (V8) {
+            if ((p & 1) == 0) {
+              xq = ldg_v8(xrow + kx + 8 * p);
+              if constexpr (T16) xq8 = ldg_v8(xrow8 + kx + 8 * p);
+            }
+            const int q = (p & 1) * 4;
+            xb = make_uint4(xq.v[q], xq.v[q + 1], xq.v[q + 2], xq.v[q + 3]);
+            if constexpr (T16) xc = make_uint4(xq8.v[q], xq8.v[q + 1], xq8.v[q + 2], xq8.v[q + 3]);
+          } else {
+            xb = __ldg(reinterpret_cast<const uint4*>(xrow + kx + 8 * p));
+          }
           const int h = p >> 2, wi = p & 3;
           const uint32_t w0 = wi == 0 ? buf[d].c[0][h].x : wi == 1 ? buf[d].c[0][h].y
                             : wi == 2 ? buf[d].c[0][h].z : buf[d].c[0][h].w;
@@ -216,42 +242,74 @@ __global__ void __launch_bounds__(kThreads, 2)
                             : wi == 2 ? buf[d].c[1][h].z : buf[d].c[1][h].w;
           const uint4 o0 = dq8(lut[0][BS == 32 ? h : 0], w0);
           const uint4 o1 = dq8(lut[1][BS == 32 ? h : 0], w1);
-          mma16<F>(acc[(2 * p) % kChains], o0.x, o1.x, o0.y, o1.y, xb.x, xb.y);
-          mma16<F>(acc[(2 * p + 1) % kChains], o0.z, o1.z, o0.w, o1.w, xb.z, xb.w);
+          if constexpr (T16) {
+            mma16<F>(acc[0], xb.x, xc.x, xb.y, xc.y, o0.x, o0.y);
+            mma16<F>(acc[1], xb.x, xc.x, xb.y, xc.y, o1.x, o1.y);
+            mma16<F>(acc[0], xb.z, xc.z, xb.w, xc.w, o0.z, o0.w);
+            mma16<F>(acc[1], xb.z, xc.z, xb.w, xc.w, o1.z, o1.w);
+          } else {
+            mma16<F>(acc[(2 * p) % kChains], o0.x, o1.x, o0.y, o1.y, xb.x, xb.y);
+            mma16<F>(acc[(2 * p + 1) % kChains], o0.z, o1.z, o0.w, o1.w, xb.z, xb.w);
+          }
         }
         if (i + kDepth < my_steps) issue(i + kDepth, buf[d]);
       }
     }
   }
 
-  // acc[.]: rows g (0, 1) and g + 8 (2, 3) of the group, batch columns 2t and
-  // 2t + 1
+  if constexpr (T16) {
+    // acc[a]: rows 8a + 2t, 8a + 2t + 1 of the group (1, 3: the second) for
+    // rows g (0, 1) and g + 8 (2, 3) of x
 #pragma unroll
-  for (int v = 0; v < 4; ++v) {
-    float sum = 0.f;
+    for (int a = 0; a < 2; ++a)
 #pragma unroll
-    for (int c = 0; c < kChains; ++c) sum += acc[c][v];
-    red[warp][lane][v] = sum;
+      for (int v = 0; v < 4; ++v) red[warp][lane][4 * a + v] = acc[a][v];
+  } else {
+    // acc[.]: rows g (0, 1) and g + 8 (2, 3) of the group, batch columns 2t
+    // and 2t + 1
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < kChains; ++c) sum += acc[c][v];
+      red[warp][lane][v] = sum;
+    }
   }
   __syncthreads();
   if (warp == 0) {
-    float s[4];
+    if constexpr (T16) {
 #pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      s[v] = 0.f;
+      for (int e = 0; e < 8; ++e) {
+        float v = 0.f;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) s[v] += red[w][lane][v];
-    }
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-#pragma unroll
-      for (int cb = 0; cb < 2; ++cb) {
-        const int bcol = 2 * t + cb;
-        if (ok[r] && bcol < B) {
-          float v = s[2 * r + cb];
-          if (bias) v = __fadd_rn(v, half_to_f32<F>(bias[n[r]]));
+        for (int w = 0; w < kWarps; ++w) v += red[w][lane][e];
+        const int64_t row = row0 + 8 * (e >> 2) + 2 * t + (e & 1);
+        const int xr = g + 8 * ((e >> 1) & 1);
+        if (row < N && xr < B) {
+          if (bias) v = __fadd_rn(v, half_to_f32<F>(bias[row]));
           const uint32_t o = pack2<F>(v, 0.0f);
-          y[static_cast<int64_t>(bcol) * N + n[r]] = static_cast<uint16_t>(o);
+          y[static_cast<int64_t>(xr) * N + row] = static_cast<uint16_t>(o);
+        }
+      }
+    } else {
+      float s[4];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        s[v] = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) s[v] += red[w][lane][v];
+      }
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+#pragma unroll
+        for (int cb = 0; cb < 2; ++cb) {
+          const int bcol = 2 * t + cb;
+          if (ok[r] && bcol < B) {
+            float v = s[2 * r + cb];
+            if (bias) v = __fadd_rn(v, half_to_f32<F>(bias[n[r]]));
+            const uint32_t o = pack2<F>(v, 0.0f);
+            y[static_cast<int64_t>(bcol) * N + n[r]] = static_cast<uint16_t>(o);
+          }
         }
       }
     }
@@ -259,23 +317,34 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 template <int BS, int QT, bool DQ, int F, int MAXP>
-cudaError_t launch_t(const DirectList<MAXP>& L, int64_t grid, int64_t B, int64_t K,
+cudaError_t launch_t(const DirectList<MAXP>& L, int64_t grid, int64_t B, int64_t K, bool v8,
                      cudaStream_t s) {
   // two K steps of loads in flight per lane (for K <= 4096 that is all of a
-  // warp's share), 2 CTAs of 8 warps resident per SM; launched as a
-  // programmatic dependent of the previous kernel on the stream
-  return launch_kernel(gemv4_direct_kernel<BS, QT, DQ, 2, F, MAXP>,
-                       dim3(static_cast<unsigned>(grid)), dim3(kThreads), 0, s, true, L,
-                       static_cast<int>(B), K);
+  // warp's share), 2 CTAs of 8 warps resident per SM
+  const dim3 grd(static_cast<unsigned>(grid)), blk(kThreads);
+  if constexpr (MAXP == 1) {
+    if (B > 8)  // single weights only; the caller checked v8
+      return launch_kernel(gemv4_direct_kernel<BS, QT, DQ, 2, F, MAXP, true, true>, grd, blk,
+                           0, s, false, L, static_cast<int>(B), K);
+  }
+  if (v8)
+    return launch_kernel(gemv4_direct_kernel<BS, QT, DQ, 2, F, MAXP, true, false>, grd, blk, 0,
+                         s, false, L, static_cast<int>(B), K);
+  return launch_kernel(gemv4_direct_kernel<BS, QT, DQ, 2, F, MAXP, false, false>, grd, blk, 0, s,
+                       false, L, static_cast<int>(B), K);
 }
+
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 template <int MAXP>
 cudaError_t launch_list(const GemvLinear* lin, int count, int64_t B, int fmt, cudaStream_t s) {
   DirectList<MAXP> L{};
   L.count = count;
   int64_t rg = 0;
+  bool v8 = true;  // every x and codes array 32-byte aligned
   for (int i = 0; i < count; ++i) {
     const GemvLinear& l = lin[i];
+    v8 = v8 && aligned32(l.x) && aligned32(l.W->codes);
     DirectProb& p = L.p[i];
     p.x = static_cast<const uint16_t*>(l.x);
     p.codes = l.W->codes;
@@ -289,6 +358,12 @@ cudaError_t launch_list(const GemvLinear* lin, int count, int64_t B, int fmt, cu
     p.rg0 = static_cast<int>(rg);
     rg += (l.N + kRowsPerCta - 1) / kRowsPerCta;
   }
+  if (B > 8 && (MAXP != 1 || !v8)) return cudaErrorInvalidValue;  // see gemv_direct_takes
+  // lists at B = 1 keep the 128-bit loads: measured on B200, 256-bit ones
+  // cost them 1-3% (two 11008 x 4096 weights: 14.6 -> 15.0 us each) and a
+  // 7B decoder pass 2%, while single weights gain up to 15% (4096^2: 7.1 ->
+  // 6.1 us) and every B > 1 launch 7-18%
+  if (MAXP != 1 && B == 1) v8 = false;
   const bnb4_qstate& W = *lin[0].W;
   const int64_t K = lin[0].K;
   const bool dq = W.double_quant != 0;
@@ -296,14 +371,14 @@ cudaError_t launch_list(const GemvLinear* lin, int count, int64_t B, int fmt, cu
   const bool f16 = fmt == BNB4_F16;
 #define BNB4_DIRECT_LAUNCH(BSV)                                                            \
   if (nf4)                                                                                 \
-    return dq ? (f16 ? launch_t<BSV, kQtNF4, true, BNB4_F16, MAXP>(L, rg, B, K, s)         \
-                     : launch_t<BSV, kQtNF4, true, BNB4_BF16, MAXP>(L, rg, B, K, s))       \
-              : (f16 ? launch_t<BSV, kQtNF4, false, BNB4_F16, MAXP>(L, rg, B, K, s)        \
-                     : launch_t<BSV, kQtNF4, false, BNB4_BF16, MAXP>(L, rg, B, K, s));     \
-  return dq ? (f16 ? launch_t<BSV, kQtFP4, true, BNB4_F16, MAXP>(L, rg, B, K, s)           \
-                   : launch_t<BSV, kQtFP4, true, BNB4_BF16, MAXP>(L, rg, B, K, s))         \
-            : (f16 ? launch_t<BSV, kQtFP4, false, BNB4_F16, MAXP>(L, rg, B, K, s)          \
-                   : launch_t<BSV, kQtFP4, false, BNB4_BF16, MAXP>(L, rg, B, K, s));
+    return dq ? (f16 ? launch_t<BSV, kQtNF4, true, BNB4_F16, MAXP>(L, rg, B, K, v8, s)         \
+                     : launch_t<BSV, kQtNF4, true, BNB4_BF16, MAXP>(L, rg, B, K, v8, s))       \
+              : (f16 ? launch_t<BSV, kQtNF4, false, BNB4_F16, MAXP>(L, rg, B, K, v8, s)        \
+                     : launch_t<BSV, kQtNF4, false, BNB4_BF16, MAXP>(L, rg, B, K, v8, s));     \
+  return dq ? (f16 ? launch_t<BSV, kQtFP4, true, BNB4_F16, MAXP>(L, rg, B, K, v8, s)           \
+                   : launch_t<BSV, kQtFP4, true, BNB4_BF16, MAXP>(L, rg, B, K, v8, s))         \
+            : (f16 ? launch_t<BSV, kQtFP4, false, BNB4_F16, MAXP>(L, rg, B, K, v8, s)          \
+                   : launch_t<BSV, kQtFP4, false, BNB4_BF16, MAXP>(L, rg, B, K, v8, s));
   switch (W.blocksize) {
     case 32: BNB4_DIRECT_LAUNCH(32)
     case 64: BNB4_DIRECT_LAUNCH(64)
@@ -314,6 +389,10 @@ cudaError_t launch_list(const GemvLinear* lin, int count, int64_t B, int fmt, cu
 }
 
 }  // namespace
+
+bool gemv_direct_takes(const void* x, const bnb4_qstate& W, int64_t B) {
+  return B >= 1 && (B <= 8 || (B <= 16 && aligned32(x) && aligned32(W.codes)));
+}
 
 cudaError_t launch_gemv_direct(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
                                int64_t N, void* y, const void* bias, int fmt, cudaStream_t s) {

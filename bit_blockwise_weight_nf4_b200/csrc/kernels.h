@@ -62,11 +62,13 @@ struct GemvLinear {
 };
 
 // The same GEMV in a launch of its own (one CTA per 16 rows, gemv_direct.cu):
-// faster than the persistent kernel for a single weight.
+// faster than the persistent kernel for a single weight.  B <= 8, or B <= 16
+// when gemv_direct_takes(x, W, B) (x and the codes 32-byte aligned).
+bool gemv_direct_takes(const void* x, const bnb4_qstate& W, int64_t B);
 cudaError_t launch_gemv_direct(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
                                int64_t N, void* y, const void* bias, int fmt, cudaStream_t s);
-// A list of decode linears (one K, one format), one CTA per 16 rows of any of
-// them, in launches of up to 32 weights.
+// A list of decode linears (one K, one format, B <= 8), one CTA per 16 rows of
+// any of them, in launches of up to 32 weights.
 cudaError_t launch_gemv_direct_list(const GemvLinear* lin, int count, int64_t B, int fmt,
                                     cudaStream_t s);
 

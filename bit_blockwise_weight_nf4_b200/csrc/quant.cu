@@ -308,13 +308,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
 
   extern __shared__ uint2 lut[];
   __shared__ double red[kThreads / 32];
-  // programmatic dependent launch: the next kernel (the double-quant kernel)
-  // may be scheduled early; the table is built while the previous kernel on
-  // the stream finishes, and nothing global is touched before it has
-  pdl_trigger();
+  pdl_trigger();  // the double-quant kernel may be scheduled early
   build_lut<QT>(lut);
   __syncthreads();
-  pdl_wait();
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -452,7 +448,6 @@ __global__ void __launch_bounds__(kDqThreads)
       a[j] = grp < ng && b < nb ? __ldg(absmax + b) : 0.0f;
     }
   };
-  pdl_trigger();
   pdl_wait();  // the quantize kernel's absmax and partial sums are complete
   // the warp's first group is requested together with the partial sums, so
   // the two loads share one round trip
@@ -538,9 +533,9 @@ cudaError_t launch_quant(const void* x, int64_t n, uint8_t* codes,
   const size_t smem = kLutEntries * 32 * sizeof(uint2);
   if (view)
     return launch_kernel(quant4_kernel<T, BS, QT, DQ, true>, dim3(grid), dim3(kThreads), smem,
-                         s, true, static_cast<const T*>(x), n, codes, absmax, partials, *view);
+                         s, false, static_cast<const T*>(x), n, codes, absmax, partials, *view);
   return launch_kernel(quant4_kernel<T, BS, QT, DQ, false>, dim3(grid), dim3(kThreads), smem, s,
-                       true, static_cast<const T*>(x), n, codes, absmax, partials, View2D{});
+                       false, static_cast<const T*>(x), n, codes, absmax, partials, View2D{});
 }
 
 template <typename T, int QT, bool DQ>

@@ -257,8 +257,10 @@ BNB4_API int bnb_dequantize_4bit_2d(const bnb4_qstate* st, void* out, int32_t ou
  * packed codes loaded straight into registers two K steps ahead; mma.sync,
  * one 8-column group; partial sums over K added in a fixed order, so
  * results are bit-reproducible) -- measured faster for a single weight than
- * the persistent TMA-staged kernel that bnb_gemv_4bit_grouped runs for two
- * or more; larger batches run the small-batch tcgen05 kernel of
+ * the persistent TMA-staged kernel that bnb_gemv_4bit_grouped runs for long
+ * lists; so does 9 <= B <= 16 when x and W->codes are 32-byte aligned (x
+ * then the MMA's 16-row operand; measured faster than the small-batch
+ * kernel); other batches run the small-batch tcgen05 kernel of
  * bnb_gemm_4bit.
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, SHAPE, CUDA.
  */
@@ -328,10 +330,12 @@ BNB4_API int bnb4_debug_gemv_grouped_persistent(const bnb4_gemv_problem* problem
  *     16-byte aligned.
  *  W  quantization state of the weight [N, K] (W->n == N*K).
  * Constraints: M >= 1; N % 8 == 0; K % 64 == 0; K % W->blocksize == 0.
- * M <= 256 runs the small-batch kernel (the 128 weight rows of a CTA are
- * the MMA's M side and the tokens its N; K split over a cluster of up to 8
- * CTAs whose partial sums are added in rank order), larger M the 2-CTA
- * prefill kernel (512 x 256 output tiles).  Both are deterministic.
+ * M <= 8 -- and 9 <= M <= 16 when X and W->codes are 32-byte aligned -- runs
+ * the decode kernel of bnb_gemv_4bit, other M <= 256 the small-batch kernel
+ * (the 128 weight rows of a CTA are the MMA's M side and the tokens its N;
+ * K split over a cluster of up to 8 CTAs whose partial sums are added in
+ * rank order), larger M the 2-CTA prefill kernel (512 x 256 output tiles).
+ * All are deterministic.
  * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, SHAPE, CUDA.
  */
 BNB4_API int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstate* W,
@@ -353,7 +357,8 @@ BNB4_API int bnb_gemm_4bit(const void* X, int64_t M, int64_t K, const bnb4_qstat
  *  W     quantization state of the weight [N, K] (W->n == N*K).
  * Constraints: M >= 1; K % 64 == 0; K % W->blocksize == 0; N % 8 == 0 when
  * M > 256.  The kernel follows M as in bnb_gemm_4bit (the decode kernel up to
- * 8 rows, the small-batch kernel up to 256, the prefill kernel above); with
+ * 8 rows, or 16 with x and W->codes 32-byte aligned, the small-batch kernel
+ * up to 256, the prefill kernel above); with
  * dtype BNB4_BF16 and no bias the result equals that of bnb_gemm_4bit /
  * bnb_gemv_4bit bit for bit.
  * Errors: INVALID_ARG, UNSUPPORTED (dtype), ALIGNMENT, SHAPE, CUDA.

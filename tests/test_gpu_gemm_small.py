@@ -2,8 +2,10 @@
 weight rows on the MMA's M side and K split over a cluster of 1..8 CTAs)
 against the fp64 oracle over the dequantized bf16 weight, with the tolerance
 of the method's brief.  Reached through both linear entry points: the GEMM
-for 8 < M <= 256 (M <= 8 runs the decode kernel) and the GEMV for
-8 < B <= 256."""
+for 8 < M <= 256 and the GEMV for 8 < B <= 256 (M <= 8 runs the decode
+kernel, and so does 9..16 when x and the codes are 32-byte aligned: the
+cases with 9..16 rows run both, the small-batch kernel on a copy of x that
+is only 16-byte aligned)."""
 import numpy as np
 import pytest
 import torch
@@ -21,7 +23,7 @@ def status_ok():
     return bnb4.bnb4_device_status(torch.cuda.current_stream().cuda_stream) == 0
 
 
-def case(M, N, K, bs=64, qtype=bnb4.NF4, dq=True, seed=0, entry="gemm"):
+def case(M, N, K, bs=64, qtype=bnb4.NF4, dq=True, seed=0, entry="gemm", unaligned=False):
     W = synth.weight_bf16(N, K, seed=seed)
     X = synth.activations_bf16(M, K, seed=seed + 1)
     st = oracle.quantize(synth.bf16_bits(W.view(-1)), bs, qtype, dq)
@@ -29,10 +31,17 @@ def case(M, N, K, bs=64, qtype=bnb4.NF4, dq=True, seed=0, entry="gemm"):
     Xb = synth.bf16_bits(X)
     y64 = oracle.linear_ref(Xb, What)
     g = bnb4.state_from_arrays(st)
+    Xd = X.cuda()
+    if unaligned:  # a copy 16 bytes past a 32-byte boundary
+        buf = torch.empty(M * K + 32, dtype=Xd.dtype, device="cuda")
+        lead = ((16 - buf.data_ptr() % 32) % 32) // 2
+        Xd = buf[lead:lead + M * K].view(M, K)
+        Xd.copy_(X)
+        assert Xd.data_ptr() % 32 == 16
     if entry == "gemm":
-        Y = bnb4.gemm_4bit(X.cuda(), g, N)
+        Y = bnb4.gemm_4bit(Xd, g, N)
     else:
-        Y = bnb4.gemv_4bit(X.cuda(), g, N)
+        Y = bnb4.gemv_4bit(Xd, g, N)
     assert status_ok()
     return check_linear(cpu_bits(Y), y64, Xb, What)
 
@@ -46,6 +55,8 @@ def test_token_counts(M):
     last ragged) with 33 K steps split over a 7-CTA cluster (5 or 4 steps
     per rank)."""
     case(M, 1032, 2112, seed=M)
+    if 9 <= M <= 16:
+        case(M, 1032, 2112, seed=M, unaligned=True)
 
 
 @pytest.mark.parametrize("N,K", [(16384, 256),   # cluster of 2 / 1 (24 / 160 tokens)
@@ -87,7 +98,7 @@ def test_llama_shapes(N, K, M):
 def test_gemv_entry_large_batch(B, N):
     """bnb_gemv_4bit with more than 8 rows of x runs the same kernel; N need
     not be a multiple of 8 there (y is written element by element)."""
-    case(B, N, 1344, seed=B + N, entry="gemv")
+    case(B, N, 1344, seed=B + N, entry="gemv", unaligned=B <= 16)
 
 
 @pytest.mark.parametrize("M", [64, 256])

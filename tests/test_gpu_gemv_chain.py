@@ -1,14 +1,13 @@
 """Decode GEMVs chained through their outputs on one stream.
 
-The one-CTA-per-16-rows decode kernel is launched as a programmatic
-dependent of the previous kernel on the stream: it may be scheduled while
-that kernel still runs, and waits for it before its first global access.  A
-chain whose every link reads the output of the link before must therefore
-give exactly the results of the same links run one at a time with a
-synchronisation between them (the kernels are deterministic) -- eagerly,
-inside a CUDA graph whose first node copies the chain's input in, and for a
-decoder layer's grouped lists mixed with the persistent kernel (launched
-normally).  The last link is also checked against the fp64 oracle."""
+Each link reads the output of the link before, as a decoder's linears do.
+The chain must give exactly the results of the same links run one at a time
+with a synchronisation between them (the kernels are deterministic) --
+eagerly, inside a CUDA graph whose first node copies the chain's input in,
+and for a decoder layer's grouped lists mixing both decode kernels.  (A
+launch that overlaps its predecessor, as a programmatic dependent launch
+would, must still pass this.)  The last link is also checked against the
+fp64 oracle."""
 import pytest
 import torch
 

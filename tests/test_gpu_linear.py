@@ -2,7 +2,8 @@
 16-bit compute types (bf16, fp16) with an optional fused bias -- against the
 fp64 oracle over the weight dequantized in that compute type, with the
 tolerance of the method's brief.  Every kernel tier is reached: the decode
-kernel (M <= 8), the small-batch kernel (9..256) and the prefill kernel."""
+kernel (M <= 8, and 9..16 rows with x and the codes 32-byte aligned, as
+here), the small-batch kernel (up to 256) and the prefill kernel."""
 import numpy as np
 import pytest
 import torch
@@ -50,7 +51,7 @@ def case(M, N, K, dtype, with_bias, bs=64, qtype=bnb4.NF4, dq=True, seed=0, n_ro
 @pytest.mark.parametrize("with_bias", [False, True])
 @pytest.mark.parametrize("M", [1, 5, 8, 9, 40, 256, 257, 600])
 def test_every_tier(dtype, with_bias, M):
-    """Decode (1, 5, 8 rows), small-batch (9, 40, 256) and prefill (257, 600)
+    """Decode (1, 5, 8, 9 rows), small-batch (40, 256) and prefill (257, 600)
     kernels, ragged N (3 weight-row tiles of the small kernel, partial pair
     tiles of the prefill kernel) and several K steps."""
     case(M, 264 if M <= 256 else 520, 1280 if M <= 256 else 1024, dtype, with_bias,
