@@ -153,21 +153,42 @@ inline View2D make_view(int64_t cols, int64_t ld) {
   return View2D{cols, ld, ~0ull / static_cast<uint64_t>(cols) + 1ull};
 }
 
-// Programmatic dependent launch, used only inside one API call: a kernel
-// whose predecessor on the stream is the library's own previous kernel of the
-// same call (the double-quant kernel after the quantize kernel) is launched
-// with programmatic stream serialization, so it may be scheduled while that
-// kernel finishes; it waits for it with pdl_wait before touching global
-// memory.  The first kernel of every call launches normally: the caller's
-// previous work on the stream may be a copy, which a programmatic launch
-// would not wait for (observed on B200: a pageable host-to-device copy
-// followed by programmatic launches gave intermittent mismatches).  Both
-// device calls are no-ops without such a launch.
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may be scheduled while the kernel before it on the stream
+// finishes; it waits for that kernel with pdl_wait before touching global
+// memory.  Such a launch is made only where the predecessor is known to be a
+// kernel: the double-quant kernel after the quantize kernel of the same call,
+// and, while a stream is being captured into a CUDA graph, a library kernel
+// whose one dependency node is a kernel node (programmatic_after_kernel).
+// Eager launches of a call's first kernel are plain: the caller's previous
+// work on the stream may be a copy, which a programmatic launch would not
+// wait for (observed on B200: a pageable host-to-device copy followed by
+// programmatic launches gave intermittent mismatches).  Both device calls are
+// no-ops without such a launch.
 __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 __device__ __forceinline__ void pdl_wait() {
   asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// True while `s` is being captured and its single dependency is a kernel
+// node: a launch there may be programmatic (a kernel-to-kernel edge).
+inline bool programmatic_after_kernel(cudaStream_t s) {
+  cudaStreamCaptureStatus st = cudaStreamCaptureStatusNone;
+  const cudaGraphNode_t* deps = nullptr;
+  size_t n = 0;
+  if (cudaStreamGetCaptureInfo(s, &st, nullptr, nullptr, &deps, &n) != cudaSuccess) {
+    cudaGetLastError();  // not fatal: launch plainly
+    return false;
+  }
+  if (st != cudaStreamCaptureStatusActive || n != 1 || deps == nullptr) return false;
+  cudaGraphNodeType t;
+  if (cudaGraphNodeGetType(deps[0], &t) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return t == cudaGraphNodeTypeKernel;
 }
 
 template <typename... KArgs, typename... Args>

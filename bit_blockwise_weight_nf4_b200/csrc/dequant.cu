@@ -122,6 +122,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   __shared__ float table[16];
   if (threadIdx.x < 16) table[threadIdx.x] = code_value(qtype, threadIdx.x);
   __syncthreads();
+  // programmatic dependent launch (inside a captured graph after a kernel):
+  // no global access before the previous kernel has completed
+  pdl_trigger();
+  pdl_wait();
   const float off = DQ ? __ldg(offset) : 0.0f;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -205,12 +209,14 @@ cudaError_t launch(const bnb4_qstate& st, void* out, int grid, const View2D* vie
   using TO = typename Out<OF>::T;
   if (view)
     return launch_kernel(dequant4_kernel<OF, DQ, BS, true>, dim3(grid), dim3(kThreads), 0, s,
-                         false, static_cast<const uint8_t*>(st.codes), st.n,
+                         programmatic_after_kernel(s), static_cast<const uint8_t*>(st.codes),
+                         st.n,
                          static_cast<int>(st.qtype), static_cast<const float*>(st.absmax),
                          static_cast<const uint8_t*>(st.absmax_q),
                          static_cast<const float*>(st.scale2),
                          static_cast<const float*>(st.offset), static_cast<TO*>(out), *view);
-  return launch_kernel(dequant4_kernel<OF, DQ, BS, false>, dim3(grid), dim3(kThreads), 0, s, false,
+  return launch_kernel(dequant4_kernel<OF, DQ, BS, false>, dim3(grid), dim3(kThreads), 0, s,
+                       programmatic_after_kernel(s),
                        static_cast<const uint8_t*>(st.codes), st.n,
                        static_cast<int>(st.qtype), static_cast<const float*>(st.absmax),
                        static_cast<const uint8_t*>(st.absmax_q),

@@ -349,6 +349,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int cnt = i1 - i0;
   int p_begin = 0;
   while (p_begin + 1 < grp.count && rb >= grp.p[p_begin + 1].rg0) ++p_begin;
+  // programmatic dependent launch (inside a captured graph after a kernel):
+  // no global access before the previous kernel has completed
+  pdl_trigger();
+  pdl_wait();
 
   if (cnt > 0) {
     uint64_t* full = sm.full[warp];
@@ -548,7 +552,7 @@ cudaError_t launch_k(const Group<MAXP>& grp, int num_sms, cudaStream_t s) {
   }
   const int64_t grid = grp.n_rg < num_sms ? grp.n_rg : num_sms;
   return launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmemBytes, s,
-                       false, grp);
+                       programmatic_after_kernel(s), grp);
 }
 
 template <int BS, int QT, bool DQ, int F, int MAXP>

@@ -37,6 +37,10 @@
 //    weight is still dequantized once.
 //  * The 8 warps' partial sums are added in shared memory in a fixed order,
 //    the bias (if any) added in fp32, and rounded once.
+//  * Inside a captured CUDA graph, after a kernel node, the launch is a
+//    programmatic dependent of that kernel (common.cuh): it may be scheduled
+//    while the kernel's last wave runs and waits for it before its first
+//    global access (a 7B decoder pass replayed as a graph: 2.5% faster).
 #include "common.cuh"
 #include "kernels.h"
 #include "lut.cuh"
@@ -162,6 +166,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int64_t n[2] = {row0 + g, row0 + g + 8};
   const bool ok[2] = {n[0] < N, n[1] < N};
   const int64_t steps = (K + kKStep - 1) / kKStep;
+  // programmatic dependent launch (inside a captured graph after a kernel):
+  // the next kernel may be scheduled now; no global access before the
+  // previous kernel has completed (x may be its output)
+  pdl_trigger();
+  pdl_wait();
   const float off = DQ ? __ldg(offset) : 0.0f;
   const int my_steps =
       warp < steps ? static_cast<int>((steps - warp + kWarps - 1) / kWarps) : 0;
@@ -319,19 +328,20 @@ __global__ void __launch_bounds__(kThreads, 2)
 template <int BS, int QT, bool DQ, int F, int MAXP>
 cudaError_t launch_t(const DirectList<MAXP>& L, int64_t grid, int64_t B, int64_t K, bool v8,
                      cudaStream_t s) {
+  const bool prog = programmatic_after_kernel(s);
   // two K steps of loads in flight per lane (for K <= 4096 that is all of a
   // warp's share), 2 CTAs of 8 warps resident per SM
   const dim3 grd(static_cast<unsigned>(grid)), blk(kThreads);
   if constexpr (MAXP == 1) {
     if (B > 8)  // single weights only; the caller checked v8
       return launch_kernel(gemv4_direct_kernel<BS, QT, DQ, 2, F, MAXP, true, true>, grd, blk,
-                           0, s, false, L, static_cast<int>(B), K);
+                           0, s, prog, L, static_cast<int>(B), K);
   }
   if (v8)
     return launch_kernel(gemv4_direct_kernel<BS, QT, DQ, 2, F, MAXP, true, false>, grd, blk, 0,
-                         s, false, L, static_cast<int>(B), K);
+                         s, prog, L, static_cast<int>(B), K);
   return launch_kernel(gemv4_direct_kernel<BS, QT, DQ, 2, F, MAXP, false, false>, grd, blk, 0, s,
-                       false, L, static_cast<int>(B), K);
+                       prog, L, static_cast<int>(B), K);
 }
 
 bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }

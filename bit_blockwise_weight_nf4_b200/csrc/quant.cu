@@ -311,6 +311,9 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   pdl_trigger();  // the double-quant kernel may be scheduled early
   build_lut<QT>(lut);
   __syncthreads();
+  // launched programmatically (inside a captured graph after a kernel): no
+  // global access before the previous kernel has completed
+  pdl_wait();
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -448,7 +451,8 @@ __global__ void __launch_bounds__(kDqThreads)
       a[j] = grp < ng && b < nb ? __ldg(absmax + b) : 0.0f;
     }
   };
-  pdl_wait();  // the quantize kernel's absmax and partial sums are complete
+  pdl_trigger();  // a programmatic launch after this one may be scheduled early
+  pdl_wait();     // the quantize kernel's absmax and partial sums are complete
   // the warp's first group is requested together with the partial sums, so
   // the two loads share one round trip
   float a[8];
@@ -533,9 +537,10 @@ cudaError_t launch_quant(const void* x, int64_t n, uint8_t* codes,
   const size_t smem = kLutEntries * 32 * sizeof(uint2);
   if (view)
     return launch_kernel(quant4_kernel<T, BS, QT, DQ, true>, dim3(grid), dim3(kThreads), smem,
-                         s, false, static_cast<const T*>(x), n, codes, absmax, partials, *view);
+                         s, programmatic_after_kernel(s), static_cast<const T*>(x), n, codes,
+                         absmax, partials, *view);
   return launch_kernel(quant4_kernel<T, BS, QT, DQ, false>, dim3(grid), dim3(kThreads), smem, s,
-                       false, static_cast<const T*>(x), n, codes, absmax, partials, View2D{});
+                       programmatic_after_kernel(s), static_cast<const T*>(x), n, codes, absmax, partials, View2D{});
 }
 
 template <typename T, int QT, bool DQ>

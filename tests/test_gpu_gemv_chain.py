@@ -123,3 +123,54 @@ def test_decoder_layers_with_grouped_lists(B):
         got = layer_pass(x, sync=False)
         for i, (a, b) in enumerate(zip(got, ref)):
             assert torch.equal(a, b), "output %d differs from the serialised run" % i
+
+
+def test_graph_after_other_kernels():
+    """Inside a CUDA graph the library's kernels that follow a kernel node
+    are launched as programmatic dependents of it: here every input is the
+    output of a torch kernel captured just before (one that never lets its
+    dependents start early), so each call must still see that kernel's
+    finished output -- quantize, dequantize and a decode chain, compared bit
+    for bit with the same calls run eagerly."""
+    N, K, B = 1088, 4096, 1
+    w_src = synth.weight_bf16(N, K, seed=31, device="cuda").view(-1)
+    x_src = torch.empty(B, K, dtype=torch.bfloat16, device="cuda")
+    st = bnb4.QuantState(N * K, 64, bnb4.NF4, True)
+    ws = bnb4.workspace_for(st)
+    deq = torch.empty(N * K, dtype=torch.bfloat16, device="cuda")
+    y1 = torch.empty(B, N, dtype=torch.bfloat16, device="cuda")
+    sts2 = quantized([(K, N)], seed=32)
+
+    def body():
+        w = w_src * 1.0                      # a torch kernel produces the weight
+        bnb4.quantize_4bit(w, 64, bnb4.NF4, True, state=st, workspace=ws)
+        bnb4.dequantize_4bit(st, torch.bfloat16, out=deq)
+        x = x_src + 0.0                      # and another one the activations
+        bnb4.gemv_4bit(x, st, N, out=y1)
+        return bnb4.gemv_4bit(y1, sts2[0], K)
+
+    x_src.copy_(synth.activations_bf16(B, K, seed=33, device="cuda"))
+    body()  # warm-up outside capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s), torch.cuda.graph(g, stream=s):
+        y2 = body()
+    torch.cuda.current_stream().wait_stream(s)
+    for trial in range(3):
+        x_src.copy_(synth.activations_bf16(B, K, seed=40 + trial, device="cuda"))
+        w_src.mul_(-1.0 if trial % 2 else 1.0)
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        got = (st.codes.clone(), st.absmax_q.clone(), deq.clone(), y1.clone(), y2.clone())
+        ref_st = bnb4.quantize_4bit(w_src.clone(), 64, bnb4.NF4, True)
+        ref_deq = bnb4.dequantize_4bit(ref_st, torch.bfloat16)
+        ref_y1 = bnb4.gemv_4bit(x_src.clone(), ref_st, N)
+        ref_y2 = bnb4.gemv_4bit(ref_y1, sts2[0], K)
+        torch.cuda.synchronize()
+        for name, a, b in zip(("codes", "absmax_q", "dequantized", "y1", "y2"), got,
+                              (ref_st.codes, ref_st.absmax_q, ref_deq, ref_y1, ref_y2)):
+            assert torch.equal(a, b), "replay %d: %s differs" % (trial, name)
+    del g
