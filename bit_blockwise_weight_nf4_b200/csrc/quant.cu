@@ -45,50 +45,82 @@ constexpr int kThreads = 256;
 constexpr int kCtasPerSm = 3;       // resident CTAs per SM (register cap)
 constexpr int kRows = 8;            // 16-byte chunks per lane per tile
 constexpr int kLutEntries = 128;    // the fast path masks the bucket to 7 bits
-// v is bucketed as j = rint(32 v) + 32 (NF4) or rint(32 |v|) (FP4) with one
-// FMA against 1.5 * 2^23 (+32): the integer lands in the mantissa bits.
+// v is bucketed as j = rint(32 v) + 32 with one FMA against 1.5 * 2^23 + 32:
+// the integer lands in the mantissa bits.
 constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
 constexpr int kMagicBits = 0x4B400000;
-// FP4: the smallest magnitude midpoint, RN(RN(0 + 1/12) * 0.5).  A value
-// gets the sign bit exactly when v < -kFp4Mid0 (negative with a non-zero
-// magnitude index).
-constexpr float kFp4Mid0 = 0x1.555556p-5f;
+constexpr int kLutBuckets = 65;  // buckets reached by |v| <= 1 (+ rounding)
 
-template <int QT>
-__host__ __device__ constexpr int lut_buckets() {  // buckets reached by |v| <= 1 (+ rounding)
-  return QT == kQtNF4 ? 65 : 33;
+// The FP4 code of v (a finite value away from every decision point; used
+// only to label the table's buckets): the magnitude midpoints strictly below
+// |v|, plus the sign bit for a negative value with a non-zero magnitude.
+__device__ uint32_t fp4_code_at(float v) {
+  uint32_t m = 0;
+  const float a = fabsf(v);
+#pragma unroll
+  for (int i = 0; i < 7; ++i)
+    m += __fmul_rn(__fadd_rn(fp4_magnitude(i), fp4_magnitude(i + 1)), 0.5f) < a ? 1u : 0u;
+  return v < 0.0f && m != 0 ? m + 8u : m;
 }
 
-// Bucket table, replicated per lane: entry (j, lane) at lut[j * 32 + lane].
-// For every v whose bucket is j, code = base + (v > cand), where base counts
-// the midpoints below the bucket and cand is the only midpoint inside it (or
-// +inf).  Buckets are 1/32 wide; codebook midpoints are at least 0.08 apart, so
-// a bucket widened by 1e-3 on each side holds at most one.  Entries past the
-// reachable buckets are {+inf, 0}: only a NaN lands there, and its code is
-// 0 (no midpoint is below NaN).
+// Bucket table, replicated per lane: entry (j, lane) at lut[j * 32 + lane],
+// for buckets 1/32 wide over v in [-1, 1] (j = rint(32 v) + 32).  The code
+// of v changes at most once inside a bucket (decision points are at least
+// 0.08 apart; a bucket widened by 1e-3 on each side holds at most one), at
+// the candidate cand (+inf where there is none).
+//  NF4: entry {cand, base}; code = base + (v > cand), base counting the
+//       midpoints below the bucket.
+//  FP4: entry {cand, lo | hi << 8}; code = v > cand ? hi : lo.  Its codes
+//       are sign-magnitude: a positive midpoint m changes the code where
+//       v > m, a negative one (-m) where v >= -m, stored as the float just
+//       below -m so that the same comparison decides.
+// Entries past the reachable buckets are {+inf, 0}: only a NaN lands there,
+// and its code is 0 (no midpoint is below NaN).
 template <int QT>
 __device__ void build_lut(uint2* lut) {
-  constexpr int nm = QT == kQtNF4 ? 15 : 7;
   // one thread per entry computes it into lane slot 0 ...
   if (threadIdx.x < kLutEntries) {
     const int j = threadIdx.x;
-    int base = 0;
+    uint32_t word = 0;
     float cand = __int_as_float(0x7f800000);
-    if (j < lut_buckets<QT>()) {
-      const float center = QT == kQtNF4 ? static_cast<float>(j - 32)
-                                        : static_cast<float>(j);
+    if (j < kLutBuckets) {
+      const float center = static_cast<float>(j - 32);
       const float lo = (center - 0.5f) / 32.0f - 1e-3f;
       const float hi = (center + 0.5f) / 32.0f + 1e-3f;
+      if constexpr (QT == kQtNF4) {
+        int base = 0;
 #pragma unroll
-      for (int i = 0; i < nm; ++i) {
-        const float a = QT == kQtNF4 ? nf4_value(i) : fp4_magnitude(i);
-        const float b = QT == kQtNF4 ? nf4_value(i + 1) : fp4_magnitude(i + 1);
-        const float mid = __fmul_rn(__fadd_rn(a, b), 0.5f);
-        if (mid < lo) ++base;
-        else if (mid <= hi) cand = mid;
+        for (int i = 0; i < 15; ++i) {
+          const float mid = __fmul_rn(__fadd_rn(nf4_value(i), nf4_value(i + 1)), 0.5f);
+          if (mid < lo) ++base;
+          else if (mid <= hi) cand = mid;
+        }
+        word = static_cast<uint32_t>(base);
+      } else {
+        float d = 0.0f;  // the decision point in the bucket, if any
+        bool has = false;
+#pragma unroll
+        for (int i = 0; i < 7; ++i) {
+          const float mid = __fmul_rn(__fadd_rn(fp4_magnitude(i), fp4_magnitude(i + 1)), 0.5f);
+          if (mid >= lo && mid <= hi) {
+            cand = mid;
+            d = mid;
+            has = true;
+          }
+          if (-mid >= lo && -mid <= hi) {  // v >= -mid  <=>  v > (the float below -mid)
+            cand = __int_as_float(__float_as_int(-mid) + 1);
+            d = -mid;
+            has = true;
+          }
+        }
+        // the codes on either side of the decision point (other decision
+        // points are >= 0.08 away), or the bucket's one code at its center
+        const uint32_t c_lo = fp4_code_at(has ? d - 1e-4f : center / 32.0f);
+        const uint32_t c_hi = has ? fp4_code_at(d + 1e-4f) : c_lo;
+        word = c_lo | (c_hi << 8);
       }
     }
-    lut[j * 32] = make_uint2(__float_as_uint(cand), static_cast<uint32_t>(base));
+    lut[j * 32] = make_uint2(__float_as_uint(cand), word);
   }
   __syncthreads();
   // ... and every thread replicates entries to the other lane slots
@@ -97,36 +129,34 @@ __device__ void build_lut(uint2* lut) {
 }
 
 // Exact nearest code for any v (infinite and NaN included): the bucket is
-// clamped in the float domain (maxNum drops a NaN), which reproduces the
-// midpoint count.
+// clamped in the float domain.  A NaN (maxNum drops it) lands in bucket 0,
+// whose NF4 base is the NaN's code 0 (no midpoint is below NaN); FP4's
+// bucket 0 holds the code of v near -1, so a NaN returns 0 first.
 template <int QT>
 __device__ __forceinline__ uint32_t code_of(float v, const uint2* lut_lane) {
-  if constexpr (QT == kQtNF4) {
-    const float f = fminf(fmaxf(__fmaf_rn(v, 32.0f, kMagic + 32.0f), kMagic),
-                          kMagic + 64.0f);
-    const int j = __float_as_int(f) - kMagicBits;
-    const uint2 e = lut_lane[j * 32];
-    return e.y + (v > __uint_as_float(e.x) ? 1u : 0u);
-  } else {
-    const float a = fabsf(v);
-    const float f =
-        fminf(fmaxf(__fmaf_rn(a, 32.0f, kMagic), kMagic), kMagic + 32.0f);
-    const int j = __float_as_int(f) - kMagicBits;
-    const uint2 e = lut_lane[j * 32];
-    const uint32_t m = e.y + (a > __uint_as_float(e.x) ? 1u : 0u);
-    return m + (v < -kFp4Mid0 ? 8u : 0u);
-  }
+  if constexpr (QT == kQtFP4)
+    if (v != v) return 0u;
+  const float f = fminf(fmaxf(__fmaf_rn(v, 32.0f, kMagic + 32.0f), kMagic),
+                        kMagic + 64.0f);
+  const int j = __float_as_int(f) - kMagicBits;
+  const uint2 e = lut_lane[j * 32];
+  const bool above = v > __uint_as_float(e.x);
+  if constexpr (QT == kQtNF4)
+    return e.y + (above ? 1u : 0u);
+  else
+    return above ? (e.y >> 8) & 0xffu : e.y & 0xffu;
 }
 
 // One Horner step of the fast path, p * 16 + code(v), for |v| <= 1 + 2^-23
 // (finite block, absmax in the normal range) or NaN: the bucket index is then
 // 0..64 (127 for the canonical NaN) without clamping, the 7-bit mask only
-// keeps the address inside the table, and code = base + (v > cand) as in
+// keeps the address inside the table, and the code follows the entry as in
 // code_of.  lut_addr = shared address of this lane's slot of bucket 0.
-// Written out in PTX so that a step is 7 instructions (NF4; 11 for FP4):
-// bucket FMA, mask, table address, 64-bit table read, compare to the
-// candidate midpoint as a 0 / -1 mask, multiply-add of the base count,
-// subtract the mask.
+// Written out in PTX so that a step is 7 instructions (NF4: bucket FMA,
+// mask, table address, 64-bit table read, compare to the candidate as a 0 /
+// -1 mask, multiply-add of the base count, subtract the mask) or 8 (FP4: the
+// compare's low bit picks the lo or hi byte of the entry with one byte
+// permute).
 template <int QT>
 __device__ __forceinline__ uint32_t horner_code(uint32_t p, float v, uint32_t lut_addr) {
   uint32_t out;
@@ -142,18 +172,16 @@ __device__ __forceinline__ uint32_t horner_code(uint32_t p, float v, uint32_t lu
         : "=r"(out)
         : "f"(v), "r"(lut_addr), "r"(p));
   } else {
-    asm("{\n\t.reg .b32 av, f, j, a, c, b, m, s, t;\n\t"
-        "abs.f32 av, %1;\n\t"
-        "fma.rn.f32 f, av, 0f42000000, 0f4B400000;\n\t"  // |v| * 32 + 1.5 * 2^23
+    asm("{\n\t.reg .b32 f, j, a, c, b, m, s, k;\n\t"
+        "fma.rn.f32 f, %1, 0f42000000, 0f4B400020;\n\t"  // v * 32 + 1.5 * 2^23 + 32
         "and.b32 j, f, 127;\n\t"
         "mad.lo.u32 a, j, 256, %2;\n\t"
         "ld.shared.v2.u32 {c, b}, [a];\n\t"
-        "set.gt.u32.f32 m, av, c;\n\t"
-        "set.lt.u32.f32 s, %1, 0fBD2AAAAB;\n\t"  // v < -kFp4Mid0: sign bit
-        "and.b32 s, s, 8;\n\t"
-        "mad.lo.u32 t, %3, 16, b;\n\t"
-        "sub.u32 t, t, m;\n\t"
-        "add.u32 %0, t, s;\n\t}"
+        "set.gt.u32.f32 m, %1, c;\n\t"
+        "and.b32 s, m, 1;\n\t"
+        "xor.b32 s, s, 0x4440;\n\t"  // byte 1 (hi) or 0 (lo) of b, upper bytes 0
+        "prmt.b32 k, b, 0, s;\n\t"
+        "mad.lo.u32 %0, %3, 16, k;\n\t}"
         : "=r"(out)
         : "f"(v), "r"(lut_addr), "r"(p));
   }
