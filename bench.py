@@ -82,10 +82,10 @@ TRAFFIC = {
     # decode: DRAM bytes (read + write) over algorithmic bytes of cold
     # launches of both decode kernels -- the one-CTA-per-16-rows one on 11008
     # x 4096 (23.29 MB read, none written / 23.29 MB) and the persistent one
-    # on the six K = 4096 linears of a layer (81.27 MB read + 2.18 MB written
+    # on the six K = 4096 linears of a layer (81.28 MB read + 2.21 MB written
     # / 81.27 MB); the family's traffic per launch is that ratio times its
     # algorithmic bytes per launch
-    "gemv": {"ratio": (23.294976 + 0.0 + 81.270528 + 2.18112) / (23.290112 + 81.265152),
+    "gemv": {"ratio": (23.294976 + 0.0 + 81.27744 + 2.209536) / (23.290112 + 81.265152),
              "launch": "cold captures of both decode kernels (11008 x 4096 single; the "
                        "six K = 4096 linears of a layer in one persistent launch), scaled "
                        "by the algorithmic bytes per launch of the family",
@@ -94,14 +94,14 @@ TRAFFIC = {
                          "bit_blockwise_weight_nf4_b200/csrc/lut.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "d3a5f296dffea75f39e8a2519ea7ea9b9a6710c909f0b362592f23a426563805"},
-    "gemm": {"bytes": 46616405,
+             "sha256": "f049c995cce56a53409b4a9491add36de3da2e98bd4ffbdf923b39d608d7f493"},
+    "gemm": {"bytes": 46406315,
              "launch": "one prefill GEMM launch (M = 2048), averaged over the three "
                        "Llama-7B shapes",
              "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemm.cu",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "1763052f05d76596be2ee0e094e36538f220d72c9e50b22d1e12f01cf4fc2b44"},
+             "sha256": "a4d455f160c1d22171a989b30e5f54ed374eecb17d3cbdd84bbbdd515bb19baf"},
 }
 
 
