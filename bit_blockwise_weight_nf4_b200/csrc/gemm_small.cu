@@ -143,6 +143,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint8_t* smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
   const int xs_bytes = x_stage_bytes(nt);
   Bars* bars = reinterpret_cast<Bars*>(smem + bars_offset(nt, SX));
+  // programmatic dependent launch (inside a captured graph after a kernel):
+  // no global access and no tensor memory taken before the previous kernel
+  // has completed
+  pdl_trigger();
+  pdl_wait();
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t rank = cta_rank();
@@ -471,13 +476,15 @@ cudaError_t launch_t(const void* X, int64_t M, int64_t K, const bnb4_qstate& W, 
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem_bytes(nt, sx);
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(S);
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = programmatic_after_kernel(s) ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, mx, static_cast<int>(M), static_cast<int>(N),
                             static_cast<int>(K), nt, idesc_for(nt, F), cols,
                             static_cast<const uint8_t*>(W.codes),

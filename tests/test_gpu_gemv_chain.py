@@ -130,11 +130,13 @@ def test_graph_after_other_kernels():
     are launched as programmatic dependents of it: here every input is the
     output of a torch kernel captured just before (one that never lets its
     dependents start early), so each call must still see that kernel's
-    finished output -- quantize, dequantize and a decode chain, compared bit
-    for bit with the same calls run eagerly."""
+    finished output -- quantize, dequantize, a decode chain and a 64-token
+    linear (the small-batch kernel), compared bit for bit with the same
+    calls run eagerly."""
     N, K, B = 1088, 4096, 1
     w_src = synth.weight_bf16(N, K, seed=31, device="cuda").view(-1)
     x_src = torch.empty(B, K, dtype=torch.bfloat16, device="cuda")
+    X_src = torch.empty(64, K, dtype=torch.bfloat16, device="cuda")
     st = bnb4.QuantState(N * K, 64, bnb4.NF4, True)
     ws = bnb4.workspace_for(st)
     deq = torch.empty(N * K, dtype=torch.bfloat16, device="cuda")
@@ -147,30 +149,35 @@ def test_graph_after_other_kernels():
         bnb4.dequantize_4bit(st, torch.bfloat16, out=deq)
         x = x_src + 0.0                      # and another one the activations
         bnb4.gemv_4bit(x, st, N, out=y1)
-        return bnb4.gemv_4bit(y1, sts2[0], K)
+        y2 = bnb4.gemv_4bit(y1, sts2[0], K)
+        return y2, bnb4.gemm_4bit(X_src * 1.0, st, N)
 
     x_src.copy_(synth.activations_bf16(B, K, seed=33, device="cuda"))
+    X_src.copy_(synth.activations_bf16(64, K, seed=34, device="cuda"))
     body()  # warm-up outside capture
     torch.cuda.synchronize()
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s), torch.cuda.graph(g, stream=s):
-        y2 = body()
+        y2, Y3 = body()
     torch.cuda.current_stream().wait_stream(s)
     for trial in range(3):
         x_src.copy_(synth.activations_bf16(B, K, seed=40 + trial, device="cuda"))
+        X_src.copy_(synth.activations_bf16(64, K, seed=50 + trial, device="cuda"))
         w_src.mul_(-1.0 if trial % 2 else 1.0)
         torch.cuda.synchronize()
         g.replay()
         torch.cuda.synchronize()
-        got = (st.codes.clone(), st.absmax_q.clone(), deq.clone(), y1.clone(), y2.clone())
+        got = (st.codes.clone(), st.absmax_q.clone(), deq.clone(), y1.clone(), y2.clone(),
+               Y3.clone())
         ref_st = bnb4.quantize_4bit(w_src.clone(), 64, bnb4.NF4, True)
         ref_deq = bnb4.dequantize_4bit(ref_st, torch.bfloat16)
         ref_y1 = bnb4.gemv_4bit(x_src.clone(), ref_st, N)
         ref_y2 = bnb4.gemv_4bit(ref_y1, sts2[0], K)
+        ref_Y3 = bnb4.gemm_4bit(X_src.clone(), ref_st, N)
         torch.cuda.synchronize()
-        for name, a, b in zip(("codes", "absmax_q", "dequantized", "y1", "y2"), got,
-                              (ref_st.codes, ref_st.absmax_q, ref_deq, ref_y1, ref_y2)):
+        for name, a, b in zip(("codes", "absmax_q", "dequantized", "y1", "y2", "Y64"), got,
+                              (ref_st.codes, ref_st.absmax_q, ref_deq, ref_y1, ref_y2, ref_Y3)):
             assert torch.equal(a, b), "replay %d: %s differs" % (trial, name)
     del g
