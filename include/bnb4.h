@@ -45,10 +45,10 @@
  *    once to bf16 at the end.
  *  - Every call is ordered after the stream's earlier work as a plain launch
  *    would be.  While the stream is being captured into a CUDA graph, the
- *    quantize, dequantize, decode and small-batch kernels that follow a kernel node are
- *    captured as programmatic dependents of it (they may start while it
- *    finishes and wait for it before touching memory); eagerly, and after
- *    any other node, they launch plainly.
+ *    quantize, dequantize, decode and small-batch kernels that follow a
+ *    kernel node are captured as programmatic dependents of it (they may
+ *    start while it finishes and wait for it before touching memory);
+ *    eagerly, and after any other node, they launch plainly.
  */
 #ifndef BNB4_H_
 #define BNB4_H_
