@@ -196,6 +196,24 @@ class ClockSampler:
         self.path = None
         self.dev = device_index
         self.interval = interval_ms
+        self.skip = 0  # lines written before the timed region
+
+    def _lines(self):
+        try:
+            with open(self.path) as f:
+                return sum(1 for _ in f)
+        except OSError:
+            return 0
+
+    def ready(self, timeout_s=5.0):
+        """Wait until the sampler writes (nvidia-smi can take a second to
+        start), then mark where the timed region's samples begin."""
+        if self.proc is None:
+            return
+        t0 = time.time()
+        while self._lines() == 0 and time.time() - t0 < timeout_s and self.proc.poll() is None:
+            time.sleep(0.02)
+        self.skip = self._lines()
 
     def start(self):
         try:
@@ -220,7 +238,9 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
                  "sw_power_cap"]
         with open(self.path) as f:
-            for line in f:
+            for n, line in enumerate(f):
+                if n < self.skip:
+                    continue
                 p = [c.strip() for c in line.split(",")]
                 if len(p) < 9:
                     continue
@@ -699,7 +719,7 @@ def run_ours(args):
         torch.cuda.synchronize()
     clocks = ClockSampler(physical_gpu_index(local))
     clocks.start()
-    time.sleep(0.1)
+    clocks.ready()
     barrier(world)
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)

@@ -152,34 +152,36 @@ __device__ __forceinline__ uint32_t code_of(float v, const uint2* lut_lane) {
 // 0..64 (127 for the canonical NaN) without clamping, the 7-bit mask only
 // keeps the address inside the table, and the code follows the entry as in
 // code_of.  lut_addr = shared address of this lane's slot of bucket 0.
-// Written out in PTX so that a step is 7 instructions (NF4: bucket FMA,
-// mask, table address, 64-bit table read, compare to the candidate as a 0 /
-// -1 mask, multiply-add of the base count, subtract the mask) or 8 (FP4: the
-// compare's low bit picks the lo or hi byte of the entry with one byte
-// permute).
+// "v > cand" is the sign bit of cand - v (exact: both are floats, the
+// difference of distinct ones is never rounded to zero, an infinite cand
+// gives +inf, and a NaN -- the canonical one, sign clear -- compares false),
+// so the compare runs on the FMA pipe as a subtraction.  Written out in PTX:
+// NF4 adds the sign bit to base + 16 p; FP4 uses it to pick the entry's lo or
+// hi byte with one byte permute.
 template <int QT>
 __device__ __forceinline__ uint32_t horner_code(uint32_t p, float v, uint32_t lut_addr) {
   uint32_t out;
   if constexpr (QT == kQtNF4) {
-    asm("{\n\t.reg .b32 f, j, a, c, b, m, t;\n\t"
+    asm("{\n\t.reg .b32 f, j, a, c, b, d, s, t;\n\t"
         "fma.rn.f32 f, %1, 0f42000000, 0f4B400020;\n\t"  // v * 32 + 1.5 * 2^23 + 32
         "and.b32 j, f, 127;\n\t"
         "mad.lo.u32 a, j, 256, %2;\n\t"
         "ld.shared.v2.u32 {c, b}, [a];\n\t"
-        "set.gt.u32.f32 m, %1, c;\n\t"
+        "sub.rn.f32 d, c, %1;\n\t"    // negative exactly when v > cand
         "mad.lo.u32 t, %3, 16, b;\n\t"
-        "sub.u32 %0, t, m;\n\t}"
+        "shr.u32 s, d, 31;\n\t"
+        "add.u32 %0, t, s;\n\t}"
         : "=r"(out)
         : "f"(v), "r"(lut_addr), "r"(p));
   } else {
-    asm("{\n\t.reg .b32 f, j, a, c, b, m, s, k;\n\t"
+    asm("{\n\t.reg .b32 f, j, a, c, b, d, s, k;\n\t"
         "fma.rn.f32 f, %1, 0f42000000, 0f4B400020;\n\t"  // v * 32 + 1.5 * 2^23 + 32
         "and.b32 j, f, 127;\n\t"
         "mad.lo.u32 a, j, 256, %2;\n\t"
         "ld.shared.v2.u32 {c, b}, [a];\n\t"
-        "set.gt.u32.f32 m, %1, c;\n\t"
-        "and.b32 s, m, 1;\n\t"
-        "xor.b32 s, s, 0x4440;\n\t"  // byte 1 (hi) or 0 (lo) of b, upper bytes 0
+        "sub.rn.f32 d, c, %1;\n\t"    // negative exactly when v > cand
+        "shr.u32 s, d, 31;\n\t"
+        "or.b32 s, s, 0x4440;\n\t"    // byte 1 (hi) or 0 (lo) of b, upper bytes 0
         "prmt.b32 k, b, 0, s;\n\t"
         "mad.lo.u32 %0, %3, 16, k;\n\t}"
         : "=r"(out)
