@@ -91,6 +91,7 @@ TRAFFIC = {
                        "by the algorithmic bytes per launch of the family",
              "sources": ("bit_blockwise_weight_nf4_b200/csrc/gemv.cu",
                          "bit_blockwise_weight_nf4_b200/csrc/gemv_direct.cu",
+                         "bit_blockwise_weight_nf4_b200/csrc/l2warm.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/lut.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),

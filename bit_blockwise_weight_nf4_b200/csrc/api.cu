@@ -129,8 +129,9 @@ int from_cuda(cudaError_t e) { return e == cudaSuccess ? BNB4_OK : BNB4_ERR_CUDA
 // the middle of capturing a stream into a CUDA graph, whose default (global)
 // mode forbids such calls.  The query therefore runs with this thread's
 // capture interaction mode switched to relaxed and restored right after, so
-// the checks behave the same inside and outside a capture.
-int bnb4::resolve_ptr(const void* p, Residency where, const void** dev) {
+// the checks behave the same inside and outside a capture.  *on_device (if
+// given) tells whether p is plain device memory.
+int bnb4::resolve_ptr(const void* p, Residency where, const void** dev, bool* on_device) {
   cudaPointerAttributes a;
   cudaStreamCaptureMode mode = cudaStreamCaptureModeRelaxed;
   const bool swapped = cudaThreadExchangeStreamCaptureMode(&mode) == cudaSuccess;
@@ -140,6 +141,7 @@ int bnb4::resolve_ptr(const void* p, Residency where, const void** dev) {
     cudaGetLastError();  // clear the (non-sticky) error the failed query recorded
     return BNB4_ERR_INVALID_ARG;
   }
+  if (on_device) *on_device = a.type == cudaMemoryTypeDevice;
   if (a.type == cudaMemoryTypeDevice) {
     *dev = p;
     return BNB4_OK;
@@ -222,7 +224,9 @@ int quantize_impl(const void* x, int32_t x_dtype, const bnb4_qstate* st, void* w
   int sms;
   if ((rc = num_sms(&sms)) != BNB4_OK) return rc;
   const void *xd, *ws_dev;
-  if ((rc = bnb4::resolve_ptr(x, bnb4::Residency::kDeviceOrPinnedHost, &xd)) != BNB4_OK)
+  bool x_dev = false;
+  if ((rc = bnb4::resolve_ptr(x, bnb4::Residency::kDeviceOrPinnedHost, &xd, &x_dev)) !=
+      BNB4_OK)
     return rc;
   if ((rc = check_state_memory(st, false)) != BNB4_OK) return rc;
   if (st->double_quant &&
@@ -232,7 +236,7 @@ int quantize_impl(const void* x, int32_t x_dtype, const bnb4_qstate* st, void* w
   int* err = nullptr;
   if (st->double_quant && (rc = error_word(&err)) != BNB4_OK) return rc;
   return from_cuda(bnb4::launch_quantize(xd, x_dtype, *st, workspace, err, sms,
-                                         static_cast<cudaStream_t>(stream), view));
+                                         static_cast<cudaStream_t>(stream), view, x_dev));
 }
 
 int dequantize_impl(const bnb4_qstate* st, void* out, int32_t out_dtype, void* stream,

@@ -628,9 +628,8 @@ cudaError_t launch_gemv(const void* x, int64_t B, int64_t K, const bnb4_qstate& 
                         int64_t N, void* y, const void* bias, int fmt, int num_sms, int* err,
                         cudaStream_t s) {
   // a single weight: the direct kernel is faster (gemv_direct.cu)
-  (void)num_sms;
   (void)err;
-  return launch_gemv_direct(x, B, K, W, N, y, bias, fmt, s);
+  return launch_gemv_direct(x, B, K, W, N, y, bias, fmt, num_sms, s);
 }
 
 cudaError_t launch_gemv_group(const GemvLinear* lin, int count, int64_t B, int fmt,
@@ -644,7 +643,7 @@ cudaError_t launch_gemv_group(const GemvLinear* lin, int count, int64_t B, int f
     const int c = count - i < kLargeGroup ? count - i : kLargeGroup;
     cudaError_t e;
     if (!persistent && (B > 1 || c < 4))
-      e = launch_gemv_direct_list(lin + i, c, B, fmt, s);
+      e = launch_gemv_direct_list(lin + i, c, B, fmt, num_sms, s);
     else if (c <= kSmallGroup)
       e = launch_group<kSmallGroup>(lin + i, c, B, fmt, num_sms, err, s);
     else

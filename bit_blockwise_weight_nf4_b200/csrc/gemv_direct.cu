@@ -37,12 +37,19 @@
 //    weight is still dequantized once.
 //  * The 8 warps' partial sums are added in shared memory in a fixed order,
 //    the bias (if any) added in fp32, and rounded once.
+//  * Before waiting on the previous kernel, each CTA warms L2 with its own
+//    weight rows and with the rows of the CTA one wave (the CTAs resident at
+//    once) later, which starts when a CTA retires: every CTA's first loads
+//    then find their codes in L2 (measured on B200: 2-5% faster for a single
+//    MLP weight and 7% over a 7B decoder pass of single calls with the own
+//    rows alone).
 //  * Inside a captured CUDA graph, after a kernel node, the launch is a
 //    programmatic dependent of that kernel (common.cuh): it may be scheduled
 //    while the kernel's last wave runs and waits for it before its first
 //    global access (a 7B decoder pass replayed as a graph: 2.5% faster).
 #include "common.cuh"
 #include "kernels.h"
+#include "l2warm.cuh"
 #include "lut.cuh"
 
 namespace bnb4 {
@@ -129,6 +136,32 @@ struct DirectList {
   int count;
 };
 
+// L2 warm-up of row group `cta` of the launch (its problem found from the
+// list's row-group offsets), by one warp: lanes 0-15 the codes of one row
+// each (K / 2 bytes: K is a multiple of 64 and the codes 16-byte aligned),
+// lanes 16-31 the group's block scales line by line.
+template <int BS, bool DQ, int MAXP>
+__device__ __forceinline__ void warm_rows(const DirectList<MAXP>& L, int cta, int64_t K,
+                                          int lane) {
+  int q = 0;
+  if constexpr (MAXP > 1)
+    while (q + 1 < L.count && cta >= L.p[q + 1].rg0) ++q;
+  const DirectProb& P = L.p[q];
+  const int64_t row0 = static_cast<int64_t>(cta - P.rg0) * kRowsPerCta;
+  const int64_t rows = P.N - row0 < kRowsPerCta ? P.N - row0 : kRowsPerCta;
+  if (lane < kRowsPerCta) {
+    if (lane < rows) prefetch_l2_range(P.codes + (row0 + lane) * (K / 2), K / 2);
+  } else {
+    const int64_t b0 = row0 * K / BS, nblk = rows * K / BS;
+    const char* s = DQ ? reinterpret_cast<const char*>(P.absmax_q + b0)
+                       : reinterpret_cast<const char*>(P.absmax + b0);
+    const int64_t bytes = DQ ? nblk : 4 * nblk;
+    for (int64_t o = static_cast<int64_t>(lane - kRowsPerCta) * 128; o < bytes;
+         o += (32 - kRowsPerCta) * 128)
+      prefetch_l2_line(s + o);
+  }
+}
+
 // V8: every x and codes array of the launch is 32-byte aligned, so a lane
 // reads a row's 32 code bytes of a step, and x for two MMAs, with one 256-bit
 // load each (half the load instructions and, for B > 1, half the L1 lines
@@ -141,7 +174,8 @@ struct DirectList {
 // for B <= 8.
 template <int BS, int QT, bool DQ, int kDepth, int F, int MAXP, bool V8, bool T16>
 __global__ void __launch_bounds__(kThreads, 2)
-    gemv4_direct_kernel(const __grid_constant__ DirectList<MAXP> L, int B, int64_t K) {
+    gemv4_direct_kernel(const __grid_constant__ DirectList<MAXP> L, int B, int64_t K,
+                        int64_t ahead) {
   static_assert(V8 || !T16, "the 16-row form reads x with 256-bit loads");
   constexpr int kAcc = T16 ? 2 : kChains;  // accumulators (4 floats each) per lane
   __shared__ float red[kWarps][32][T16 ? 8 : 4];
@@ -170,6 +204,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   // the next kernel may be scheduled now; no global access before the
   // previous kernel has completed (x may be its output)
   pdl_trigger();
+  // Warm L2 (l2warm.cuh) with this CTA's weight rows, while the previous
+  // kernel may still run, and with the rows of the CTA `ahead` places later,
+  // which an SM will most likely start when this one (or its neighbour)
+  // retires: every CTA after the first `ahead` then finds its codes in L2.
+  if (warp == 0) warm_rows<BS, DQ>(L, static_cast<int>(blockIdx.x), K, lane);
+  if (warp == 1 && static_cast<int64_t>(blockIdx.x) + ahead < gridDim.x)
+    warm_rows<BS, DQ>(L, static_cast<int>(blockIdx.x) + ahead, K, lane);
   pdl_wait();
   const float off = DQ ? __ldg(offset) : 0.0f;
   const int my_steps =
@@ -327,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 template <int BS, int QT, bool DQ, int F, int MAXP>
 cudaError_t launch_t(const DirectList<MAXP>& L, int64_t grid, int64_t B, int64_t K, bool v8,
-                     cudaStream_t s) {
+                     int64_t ahead, cudaStream_t s) {
   const bool prog = programmatic_after_kernel(s);
   // two K steps of loads in flight per lane (for K <= 4096 that is all of a
   // warp's share), 2 CTAs of 8 warps resident per SM
@@ -335,19 +376,20 @@ cudaError_t launch_t(const DirectList<MAXP>& L, int64_t grid, int64_t B, int64_t
   if constexpr (MAXP == 1) {
     if (B > 8)  // single weights only; the caller checked v8
       return launch_kernel(gemv4_direct_kernel<BS, QT, DQ, 2, F, MAXP, true, true>, grd, blk,
-                           0, s, prog, L, static_cast<int>(B), K);
+                           0, s, prog, L, static_cast<int>(B), K, ahead);
   }
   if (v8)
     return launch_kernel(gemv4_direct_kernel<BS, QT, DQ, 2, F, MAXP, true, false>, grd, blk, 0,
-                         s, prog, L, static_cast<int>(B), K);
+                         s, prog, L, static_cast<int>(B), K, ahead);
   return launch_kernel(gemv4_direct_kernel<BS, QT, DQ, 2, F, MAXP, false, false>, grd, blk, 0, s,
-                       prog, L, static_cast<int>(B), K);
+                       prog, L, static_cast<int>(B), K, ahead);
 }
 
 bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 template <int MAXP>
-cudaError_t launch_list(const GemvLinear* lin, int count, int64_t B, int fmt, cudaStream_t s) {
+cudaError_t launch_list(const GemvLinear* lin, int count, int64_t B, int fmt, int num_sms,
+                        cudaStream_t s) {
   DirectList<MAXP> L{};
   L.count = count;
   int64_t rg = 0;
@@ -376,19 +418,22 @@ cudaError_t launch_list(const GemvLinear* lin, int count, int64_t B, int fmt, cu
   if (MAXP != 1 && B == 1) v8 = false;
   const bnb4_qstate& W = *lin[0].W;
   const int64_t K = lin[0].K;
+  // CTAs resident at once (2 per SM): the distance of the row group a CTA
+  // warms L2 for, one wave ahead
+  const int64_t ahead = 2 * static_cast<int64_t>(num_sms);
   const bool dq = W.double_quant != 0;
   const bool nf4 = W.qtype == kQtNF4;
   const bool f16 = fmt == BNB4_F16;
-#define BNB4_DIRECT_LAUNCH(BSV)                                                            \
-  if (nf4)                                                                                 \
-    return dq ? (f16 ? launch_t<BSV, kQtNF4, true, BNB4_F16, MAXP>(L, rg, B, K, v8, s)         \
-                     : launch_t<BSV, kQtNF4, true, BNB4_BF16, MAXP>(L, rg, B, K, v8, s))       \
-              : (f16 ? launch_t<BSV, kQtNF4, false, BNB4_F16, MAXP>(L, rg, B, K, v8, s)        \
-                     : launch_t<BSV, kQtNF4, false, BNB4_BF16, MAXP>(L, rg, B, K, v8, s));     \
-  return dq ? (f16 ? launch_t<BSV, kQtFP4, true, BNB4_F16, MAXP>(L, rg, B, K, v8, s)           \
-                   : launch_t<BSV, kQtFP4, true, BNB4_BF16, MAXP>(L, rg, B, K, v8, s))         \
-            : (f16 ? launch_t<BSV, kQtFP4, false, BNB4_F16, MAXP>(L, rg, B, K, v8, s)          \
-                   : launch_t<BSV, kQtFP4, false, BNB4_BF16, MAXP>(L, rg, B, K, v8, s));
+#define BNB4_DIRECT_LAUNCH(BSV)                                                                    \
+  if (nf4)                                                                                         \
+    return dq ? (f16 ? launch_t<BSV, kQtNF4, true, BNB4_F16, MAXP>(L, rg, B, K, v8, ahead, s)      \
+                     : launch_t<BSV, kQtNF4, true, BNB4_BF16, MAXP>(L, rg, B, K, v8, ahead, s))    \
+              : (f16 ? launch_t<BSV, kQtNF4, false, BNB4_F16, MAXP>(L, rg, B, K, v8, ahead, s)     \
+                     : launch_t<BSV, kQtNF4, false, BNB4_BF16, MAXP>(L, rg, B, K, v8, ahead, s));  \
+  return dq ? (f16 ? launch_t<BSV, kQtFP4, true, BNB4_F16, MAXP>(L, rg, B, K, v8, ahead, s)        \
+                   : launch_t<BSV, kQtFP4, true, BNB4_BF16, MAXP>(L, rg, B, K, v8, ahead, s))      \
+            : (f16 ? launch_t<BSV, kQtFP4, false, BNB4_F16, MAXP>(L, rg, B, K, v8, ahead, s)       \
+                   : launch_t<BSV, kQtFP4, false, BNB4_BF16, MAXP>(L, rg, B, K, v8, ahead, s));
   switch (W.blocksize) {
     case 32: BNB4_DIRECT_LAUNCH(32)
     case 64: BNB4_DIRECT_LAUNCH(64)
@@ -405,17 +450,18 @@ bool gemv_direct_takes(const void* x, const bnb4_qstate& W, int64_t B) {
 }
 
 cudaError_t launch_gemv_direct(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
-                               int64_t N, void* y, const void* bias, int fmt, cudaStream_t s) {
+                               int64_t N, void* y, const void* bias, int fmt, int num_sms,
+                               cudaStream_t s) {
   const GemvLinear one{x, &W, K, N, bias, y};
-  return launch_list<1>(&one, 1, B, fmt, s);
+  return launch_list<1>(&one, 1, B, fmt, num_sms, s);
 }
 
 cudaError_t launch_gemv_direct_list(const GemvLinear* lin, int count, int64_t B, int fmt,
-                                    cudaStream_t s) {
-  if (count == 1) return launch_list<1>(lin, 1, B, fmt, s);
+                                    int num_sms, cudaStream_t s) {
+  if (count == 1) return launch_list<1>(lin, 1, B, fmt, num_sms, s);
   for (int i = 0; i < count; i += kDirectListMax) {
     const int c = count - i < kDirectListMax ? count - i : kDirectListMax;
-    const cudaError_t e = launch_list<kDirectListMax>(lin + i, c, B, fmt, s);
+    const cudaError_t e = launch_list<kDirectListMax>(lin + i, c, B, fmt, num_sms, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -18,7 +18,8 @@ enum class Residency { kDevice, kDeviceOrManaged, kDeviceOrPinnedHost };
 // BNB4_OK with the address the device uses in *dev, or BNB4_ERR_INVALID_ARG
 // (pageable host memory, a pointer the runtime does not know, or a kind of
 // memory `where` excludes).  Host-only; launches nothing.
-int resolve_ptr(const void* p, Residency where, const void** dev);
+int resolve_ptr(const void* p, Residency where, const void** dev,
+                bool* on_device = nullptr);
 
 // Upper bound on the quantize grid.  The double-quant workspace holds one
 // fp64 partial sum of the blocks' absmax per CTA.
@@ -29,9 +30,11 @@ int quant_grid(int64_t n, int x_dtype, int num_sms);
 // workspace: kDqWorkspaceBytes, 16-byte aligned (double quant only); err:
 // the device error word (unused: the quantize kernels have no waits).  view: x is a row-major 2-D view with a row stride
 // (see View2D), or null for a contiguous x.
+// warm_x: x is device memory, which the quantize kernel may warm in L2
+// before waiting on the previous kernel of a programmatic launch.
 cudaError_t launch_quantize(const void* x, int x_dtype, const bnb4_qstate& st,
                             void* workspace, int* err, int num_sms, cudaStream_t s,
-                            const View2D* view = nullptr);
+                            const View2D* view = nullptr, bool warm_x = false);
 
 // The library's device error word on the current device (api.cu).
 int device_error_word(int** out);
@@ -66,11 +69,12 @@ struct GemvLinear {
 // when gemv_direct_takes(x, W, B) (x and the codes 32-byte aligned).
 bool gemv_direct_takes(const void* x, const bnb4_qstate& W, int64_t B);
 cudaError_t launch_gemv_direct(const void* x, int64_t B, int64_t K, const bnb4_qstate& W,
-                               int64_t N, void* y, const void* bias, int fmt, cudaStream_t s);
+                               int64_t N, void* y, const void* bias, int fmt, int num_sms,
+                               cudaStream_t s);
 // A list of decode linears (one K, one format, B <= 8), one CTA per 16 rows of
 // any of them, in launches of up to 32 weights.
 cudaError_t launch_gemv_direct_list(const GemvLinear* lin, int count, int64_t B, int fmt,
-                                    cudaStream_t s);
+                                    int num_sms, cudaStream_t s);
 
 
 // 1..BNB4_GROUP_MAX linears of one format (blocksize, code table, scale

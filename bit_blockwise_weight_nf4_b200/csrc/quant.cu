@@ -37,6 +37,7 @@
 // fp64 partial sums in a fixed order.
 #include "common.cuh"
 #include "kernels.h"
+#include "l2warm.cuh"
 
 namespace bnb4 {
 namespace {
@@ -327,7 +328,7 @@ template <typename T, int BS, int QT, bool DQ, bool STR>
 __global__ void __launch_bounds__(kThreads, kCtasPerSm)
     quant4_kernel(const T* __restrict__ x, int64_t n,
                   uint8_t* __restrict__ codes, float* __restrict__ absmax,
-                  double* __restrict__ partials, View2D v) {
+                  double* __restrict__ partials, View2D v, bool warm) {
   constexpr int EPL = Elem<T>::kPerChunk;  // elements per 16-byte chunk
   constexpr int LPB = BS / EPL;            // lanes (chunks) per block
   constexpr int ROW = 32 * EPL;            // elements per warp row
@@ -339,6 +340,14 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   extern __shared__ uint2 lut[];
   __shared__ double red[kThreads / 32];
   pdl_trigger();  // the double-quant kernel may be scheduled early
+  // Warm L2 (l2warm.cuh) with the warp's first tile of x, one 128-byte line
+  // per lane (a tile is 32 lanes x 8 chunks of 16 bytes), while a previous
+  // kernel may still run; device memory only (`warm`).
+  if (!STR && warm) {
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
+    if (t0 < n / TILE)
+      prefetch_l2_line(reinterpret_cast<const char*>(x + t0 * TILE) + (threadIdx.x & 31) * 128);
+  }
   build_lut<QT>(lut);
   __syncthreads();
   // launched programmatically (inside a captured graph after a kernel): no
@@ -563,37 +572,46 @@ __global__ void __launch_bounds__(256) check_rcp_kernel(unsigned long long* res)
 template <typename T, int BS, int QT, bool DQ>
 cudaError_t launch_quant(const void* x, int64_t n, uint8_t* codes,
                          float* absmax, double* partials, int grid, const View2D* view,
-                         cudaStream_t s) {
+                         bool warm, cudaStream_t s) {
   const size_t smem = kLutEntries * 32 * sizeof(uint2);
   if (view)
     return launch_kernel(quant4_kernel<T, BS, QT, DQ, true>, dim3(grid), dim3(kThreads), smem,
                          s, programmatic_after_kernel(s), static_cast<const T*>(x), n, codes,
-                         absmax, partials, *view);
+                         absmax, partials, *view, false);
   return launch_kernel(quant4_kernel<T, BS, QT, DQ, false>, dim3(grid), dim3(kThreads), smem, s,
-                       programmatic_after_kernel(s), static_cast<const T*>(x), n, codes, absmax, partials, View2D{});
+                       programmatic_after_kernel(s), static_cast<const T*>(x), n, codes, absmax,
+                       partials, View2D{}, warm);
 }
 
 template <typename T, int QT, bool DQ>
 cudaError_t dispatch_bs(int bs, const void* x, int64_t n, uint8_t* codes,
                         float* absmax, double* partials, int grid, const View2D* view,
-                        cudaStream_t s) {
+                        bool warm, cudaStream_t s) {
   switch (bs) {
-    case 32: return launch_quant<T, 32, QT, DQ>(x, n, codes, absmax, partials, grid, view, s);
-    case 64: return launch_quant<T, 64, QT, DQ>(x, n, codes, absmax, partials, grid, view, s);
-    case 128: return launch_quant<T, 128, QT, DQ>(x, n, codes, absmax, partials, grid, view, s);
-    default: return launch_quant<T, 256, QT, DQ>(x, n, codes, absmax, partials, grid, view, s);
+    case 32:
+      return launch_quant<T, 32, QT, DQ>(x, n, codes, absmax, partials, grid, view, warm, s);
+    case 64:
+      return launch_quant<T, 64, QT, DQ>(x, n, codes, absmax, partials, grid, view, warm, s);
+    case 128:
+      return launch_quant<T, 128, QT, DQ>(x, n, codes, absmax, partials, grid, view, warm, s);
+    default:
+      return launch_quant<T, 256, QT, DQ>(x, n, codes, absmax, partials, grid, view, warm, s);
   }
 }
 
 template <typename T>
 cudaError_t dispatch_q(int qt, bool dq, int bs, const void* x, int64_t n,
                        uint8_t* codes, float* absmax, double* partials,
-                       int grid, const View2D* view, cudaStream_t s) {
+                       int grid, const View2D* view, bool warm, cudaStream_t s) {
   if (qt == kQtNF4)
-    return dq ? dispatch_bs<T, kQtNF4, true>(bs, x, n, codes, absmax, partials, grid, view, s)
-              : dispatch_bs<T, kQtNF4, false>(bs, x, n, codes, absmax, partials, grid, view, s);
-  return dq ? dispatch_bs<T, kQtFP4, true>(bs, x, n, codes, absmax, partials, grid, view, s)
-            : dispatch_bs<T, kQtFP4, false>(bs, x, n, codes, absmax, partials, grid, view, s);
+    return dq ? dispatch_bs<T, kQtNF4, true>(bs, x, n, codes, absmax, partials, grid, view,
+                                             warm, s)
+              : dispatch_bs<T, kQtNF4, false>(bs, x, n, codes, absmax, partials, grid, view,
+                                              warm, s);
+  return dq ? dispatch_bs<T, kQtFP4, true>(bs, x, n, codes, absmax, partials, grid, view, warm,
+                                           s)
+            : dispatch_bs<T, kQtFP4, false>(bs, x, n, codes, absmax, partials, grid, view,
+                                            warm, s);
 }
 
 }  // namespace
@@ -622,7 +640,7 @@ int quant_grid(int64_t n, int x_dtype, int num_sms) {
 
 cudaError_t launch_quantize(const void* x, int x_dtype, const bnb4_qstate& st,
                             void* workspace, int* err, int num_sms, cudaStream_t s,
-                            const View2D* view) {
+                            const View2D* view, bool warm_x) {
   (void)err;  // no bounded waits here
   const bool dq = st.double_quant != 0;
   const int grid = quant_grid(st.n, x_dtype, num_sms);
@@ -630,12 +648,12 @@ cudaError_t launch_quantize(const void* x, int x_dtype, const bnb4_qstate& st,
   cudaError_t e =
       x_dtype == BNB4_F32
           ? dispatch_q<float>(st.qtype, dq, st.blocksize, x, st.n, st.codes,
-                              st.absmax, partials, grid, view, s)
+                              st.absmax, partials, grid, view, warm_x, s)
       : x_dtype == BNB4_F16
           ? dispatch_q<Half16>(st.qtype, dq, st.blocksize, x, st.n, st.codes,
-                               st.absmax, partials, grid, view, s)
+                               st.absmax, partials, grid, view, warm_x, s)
           : dispatch_q<uint16_t>(st.qtype, dq, st.blocksize, x, st.n, st.codes,
-                                 st.absmax, partials, grid, view, s);
+                                 st.absmax, partials, grid, view, warm_x, s);
   if (e != cudaSuccess || !dq) return e;
   const int64_t nb = (st.n + st.blocksize - 1) / st.blocksize;
   const int64_t ng = (nb + 255) / 256;
