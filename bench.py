@@ -81,11 +81,11 @@ ALU_OPS_PER_WEIGHT = 2.5
 TRAFFIC = {
     # decode: DRAM bytes (read + write) over algorithmic bytes of cold
     # launches of both decode kernels -- the one-CTA-per-16-rows one on 11008
-    # x 4096 (23.29 MB read, none written / 23.29 MB) and the persistent one
-    # on the six K = 4096 linears of a layer (81.28 MB read + 2.21 MB written
+    # x 4096 (23.30 MB read, none written / 23.29 MB) and the persistent one
+    # on the six K = 4096 linears of a layer (81.26 MB read + 2.09 MB written
     # / 81.27 MB); the family's traffic per launch is that ratio times its
     # algorithmic bytes per launch
-    "gemv": {"ratio": (23.294976 + 0.0 + 81.27744 + 2.209536) / (23.290112 + 81.265152),
+    "gemv": {"ratio": (23.304448 + 0.0 + 81.260544 + 2.088448) / (23.290112 + 81.265152),
              "launch": "cold captures of both decode kernels (11008 x 4096 single; the "
                        "six K = 4096 linears of a layer in one persistent launch), scaled "
                        "by the algorithmic bytes per launch of the family",
@@ -95,7 +95,7 @@ TRAFFIC = {
                          "bit_blockwise_weight_nf4_b200/csrc/lut.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/common.cuh",
                          "bit_blockwise_weight_nf4_b200/csrc/sm100.cuh"),
-             "sha256": "f049c995cce56a53409b4a9491add36de3da2e98bd4ffbdf923b39d608d7f493"},
+             "sha256": "86e2dfca955d480d8ef1d629b19bd09c6d590179dbca7cb57a9c9e00583d0958"},
     "gemm": {"bytes": 46406315,
              "launch": "one prefill GEMM launch (M = 2048), averaged over the three "
                        "Llama-7B shapes",

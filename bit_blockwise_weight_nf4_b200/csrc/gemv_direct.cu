@@ -37,12 +37,12 @@
 //    weight is still dequantized once.
 //  * The 8 warps' partial sums are added in shared memory in a fixed order,
 //    the bias (if any) added in fp32, and rounded once.
-//  * Before waiting on the previous kernel, each CTA warms L2 with its own
-//    weight rows and with the rows of the CTA one wave (the CTAs resident at
-//    once) later, which starts when a CTA retires: every CTA's first loads
-//    then find their codes in L2 (measured on B200: 2-5% faster for a single
-//    MLP weight and 7% over a 7B decoder pass of single calls with the own
-//    rows alone).
+//  * In a programmatic launch (below), before waiting on the previous
+//    kernel, each CTA warms L2 with its own weight rows and with the rows of
+//    the CTA one wave (the CTAs resident at once) later, which starts when a
+//    CTA retires: every CTA's first loads then find their codes in L2
+//    (measured on B200: 2-5% faster for a single MLP weight, 7% over a 7B
+//    decoder pass of single calls).
 //  * Inside a captured CUDA graph, after a kernel node, the launch is a
 //    programmatic dependent of that kernel (common.cuh): it may be scheduled
 //    while the kernel's last wave runs and waits for it before its first
@@ -208,9 +208,12 @@ __global__ void __launch_bounds__(kThreads, 2)
   // kernel may still run, and with the rows of the CTA `ahead` places later,
   // which an SM will most likely start when this one (or its neighbour)
   // retires: every CTA after the first `ahead` then finds its codes in L2.
-  if (warp == 0) warm_rows<BS, DQ>(L, static_cast<int>(blockIdx.x), K, lane);
-  if (warp == 1 && static_cast<int64_t>(blockIdx.x) + ahead < gridDim.x)
-    warm_rows<BS, DQ>(L, static_cast<int>(blockIdx.x) + ahead, K, lane);
+  // ahead == 0 (a plain launch): no warm-up.
+  if (ahead > 0) {
+    if (warp == 0) warm_rows<BS, DQ>(L, static_cast<int>(blockIdx.x), K, lane);
+    if (warp == 1 && static_cast<int64_t>(blockIdx.x) + ahead < gridDim.x)
+      warm_rows<BS, DQ>(L, static_cast<int>(blockIdx.x) + ahead, K, lane);
+  }
   pdl_wait();
   const float off = DQ ? __ldg(offset) : 0.0f;
   const int my_steps =
@@ -370,6 +373,11 @@ template <int BS, int QT, bool DQ, int F, int MAXP>
 cudaError_t launch_t(const DirectList<MAXP>& L, int64_t grid, int64_t B, int64_t K, bool v8,
                      int64_t ahead, cudaStream_t s) {
   const bool prog = programmatic_after_kernel(s);
+  // L2 warm-up only in a programmatic launch, where it overlaps the previous
+  // kernel: in a plain launch the first wave's prefetches of the next wave's
+  // rows compete with its own first loads (measured on B200: a 7B decoder
+  // pass of eager launches 2.56 -> 2.80 ms with the warm-up on)
+  if (!prog) ahead = 0;
   // two K steps of loads in flight per lane (for K <= 4096 that is all of a
   // warp's share), 2 CTAs of 8 warps resident per SM
   const dim3 grd(static_cast<unsigned>(grid)), blk(kThreads);

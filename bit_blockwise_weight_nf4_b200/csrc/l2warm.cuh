@@ -4,7 +4,9 @@
 // coherently: a later write to the same bytes by another kernel still reaches
 // the loads that follow it.  So a kernel may warm its read-only operands
 // before waiting on the kernel it depends on (pdl_wait), and a CTA may warm
-// the operands of a CTA that will start after it.
+// the operands of a CTA that will start after it.  The kernels do so only in
+// a programmatic launch, where the prefetches overlap the previous kernel; in
+// a plain launch they would compete with the kernel's own first loads.
 //
 // Only for plain device memory: the linear entry points accept nothing else
 // for the weight state, and the quantize entry points warm their input only

@@ -342,7 +342,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   pdl_trigger();  // the double-quant kernel may be scheduled early
   // Warm L2 (l2warm.cuh) with the warp's first tile of x, one 128-byte line
   // per lane (a tile is 32 lanes x 8 chunks of 16 bytes), while a previous
-  // kernel may still run; device memory only (`warm`).
+  // kernel may still run (`warm`: a programmatic launch on device memory).
   if (!STR && warm) {
     const int64_t t0 = static_cast<int64_t>(blockIdx.x) * (kThreads / 32) + (threadIdx.x >> 5);
     if (t0 < n / TILE)
@@ -574,13 +574,15 @@ cudaError_t launch_quant(const void* x, int64_t n, uint8_t* codes,
                          float* absmax, double* partials, int grid, const View2D* view,
                          bool warm, cudaStream_t s) {
   const size_t smem = kLutEntries * 32 * sizeof(uint2);
+  const bool prog = programmatic_after_kernel(s);
   if (view)
     return launch_kernel(quant4_kernel<T, BS, QT, DQ, true>, dim3(grid), dim3(kThreads), smem,
-                         s, programmatic_after_kernel(s), static_cast<const T*>(x), n, codes,
-                         absmax, partials, *view, false);
+                         s, prog, static_cast<const T*>(x), n, codes, absmax, partials, *view,
+                         false);
+  // the L2 warm-up only where it overlaps a previous kernel
   return launch_kernel(quant4_kernel<T, BS, QT, DQ, false>, dim3(grid), dim3(kThreads), smem, s,
-                       programmatic_after_kernel(s), static_cast<const T*>(x), n, codes, absmax,
-                       partials, View2D{}, warm);
+                       prog, static_cast<const T*>(x), n, codes, absmax, partials, View2D{},
+                       warm && prog);
 }
 
 template <typename T, int QT, bool DQ>
