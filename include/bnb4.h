@@ -47,7 +47,9 @@
  *    would be.  While the stream is being captured into a CUDA graph, the
  *    quantize, dequantize, decode and small-batch kernels that follow a
  *    kernel node are captured as programmatic dependents of it (they may
- *    start while it finishes and wait for it before touching memory);
+ *    start while it finishes and wait for it before reading or writing
+ *    memory; only L2 prefetches of their inputs come earlier, and since L2
+ *    is coherent across the GPU a prefetch never yields stale data);
  *    eagerly, and after any other node, they launch plainly.
  */
 #ifndef BNB4_H_
